@@ -1,0 +1,19 @@
+"""B200 (sm_100a) kernels for the clip-parallel temporal modules of Video-Infinity.
+
+The latent video [P positions][F frames][C channels] is cut into N clips along
+the frame axis, and three CUDA kernels, reached through the C ABI in
+include/vi.h, compute the temporal modules with the clip partition inside the
+kernel grid:
+
+  dual_attn         dual-domain temporal attention (own clip + neighbour
+                    context + uniformly sampled global frames)
+  temporal_conv     temporal conv1d with neighbour padding, zeros at the ends
+  groupnorm_global  GroupNorm with statistics aggregated over every clip
+
+Python here only marshals arguments; see _binding.py.
+"""
+from ._binding import (LIB_PATH, ViError, dual_attn, groupnorm_global, lib,  # noqa: F401
+                       take_device_errors, temporal_conv)
+
+__all__ = ["dual_attn", "temporal_conv", "groupnorm_global", "take_device_errors", "lib",
+           "ViError", "LIB_PATH"]

@@ -1,0 +1,135 @@
+"""ctypes binding of libvi (include/vi.h): argument marshalling only.
+
+Every step of the temporal modules runs in the CUDA kernels behind the C ABI;
+this module checks that tensors are what the ABI expects (device, dtype,
+contiguity, shape), passes raw pointers and the current CUDA stream, and turns
+a negative status into an exception.  There is no CPU path: if libvi.so is
+missing the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libvi.so")
+
+VI_OK = 0
+STATUS = {0: "VI_OK", -1: "VI_ERR_INVALID_ARG", -2: "VI_ERR_ALIGNMENT", -3: "VI_ERR_UNSUPPORTED",
+          -4: "VI_ERR_CUDA", -5: "VI_ERR_DEVICE_TIMEOUT"}
+
+# name -> argument types (all return int status)
+_vp, _i, _f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+SIGNATURES = {
+    "vi_dual_attn": [_vp, _vp, _vp, _vp] + [_i] * 8 + [_vp],
+    "vi_dual_attn_f32": [_vp, _vp, _vp, _vp] + [_i] * 8 + [_vp],
+    "vi_temporal_conv": [_vp, _vp, _vp, _vp] + [_i] * 5 + [_vp],
+    "vi_temporal_conv_f32": [_vp, _vp, _vp, _vp] + [_i] * 5 + [_vp],
+    "vi_groupnorm_global": [_vp, _vp, _vp, _vp] + [_i] * 5 + [_f, _vp],
+    "vi_groupnorm_global_f32": [_vp, _vp, _vp, _vp] + [_i] * 5 + [_f, _vp],
+    "vi_version": [],
+    "vi_take_device_errors": [],
+}
+
+
+class ViError(RuntimeError):
+    def __init__(self, name: str, status: int):
+        super().__init__(f"{name} returned {status} ({STATUS.get(status, 'unknown')})")
+        self.status = status
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libvi.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libvi.so not built at {LIB_PATH}; run __graft_entry__.build()")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, args in SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = ctypes.c_int
+        L.vi_status_string.argtypes = [ctypes.c_int]
+        L.vi_status_string.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def _check(name: str, status: int) -> None:
+    if status != VI_OK:
+        raise ViError(name, status)
+
+
+def _stream_ptr(stream) -> int:
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return int(s.cuda_stream)
+
+
+def _suffix(t) -> str:
+    import torch
+    if t.dtype == torch.bfloat16:
+        return ""
+    if t.dtype == torch.float32:
+        return "_f32"
+    raise TypeError(f"libvi takes bfloat16 or float32 tensors, got {t.dtype}")
+
+
+def _dev(*ts):
+    for t in ts:
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("libvi takes contiguous CUDA tensors")
+    if len({t.dtype for t in ts}) != 1:
+        raise TypeError("all tensors of one call share a dtype")
+
+
+def dual_attn(q, k, v, out=None, *, N: int, heads: int, n_pre: int = 8, n_post: int = 8,
+              n_global: int = 16, stream=None):
+    """Dual-domain temporal attention; q, k, v, out are [P][F][heads*d] CUDA tensors."""
+    import torch
+    if out is None:
+        out = torch.empty_like(q)
+    _dev(q, k, v, out)
+    P, F, C = q.shape
+    name = "vi_dual_attn" + _suffix(q)
+    _check(name, getattr(lib(), name)(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                      F, N, P, heads, C // heads, n_pre, n_post, n_global,
+                                      _stream_ptr(stream)))
+    return out
+
+
+def temporal_conv(x, w, b, out=None, *, N: int, stream=None):
+    """Clip-padded temporal conv; x, out [P][F][C], w [C][C][k], b [C] CUDA tensors."""
+    import torch
+    if out is None:
+        out = torch.empty_like(x)
+    _dev(x, w, b, out)
+    P, F, C = x.shape
+    k = w.shape[2]
+    name = "vi_temporal_conv" + _suffix(x)
+    _check(name, getattr(lib(), name)(x.data_ptr(), w.data_ptr(), b.data_ptr(), out.data_ptr(),
+                                      F, N, P, C, k, _stream_ptr(stream)))
+    return out
+
+
+def groupnorm_global(x, gamma, beta, out=None, *, N: int, groups: int, eps: float = 1e-5,
+                     stream=None):
+    """Global-statistics GroupNorm; x, out [P][F][C] (out may be x), gamma/beta [C]."""
+    import torch
+    if out is None:
+        out = torch.empty_like(x)
+    _dev(x, gamma, beta, out)
+    P, F, C = x.shape
+    name = "vi_groupnorm_global" + _suffix(x)
+    _check(name, getattr(lib(), name)(x.data_ptr(), gamma.data_ptr(), beta.data_ptr(),
+                                      out.data_ptr(), F, N, P, C, groups, float(eps),
+                                      _stream_ptr(stream)))
+    return out
+
+
+def take_device_errors() -> None:
+    """Synchronise and raise if a kernel's bounded wait ran out since the last call."""
+    _check("vi_take_device_errors", lib().vi_take_device_errors())

@@ -1,0 +1,348 @@
+// Dual-domain temporal attention with all N clips of the video on one GPU.
+//
+// Source: "Video-Infinity: Distributed Long Video Generation" (news.43zhubao.com
+// write-up), attention-module paragraph.  Every query frame of clip i attends,
+// per spatial position and head, over one fixed key/value list: the clip's own
+// L frames, the last n_pre frames of clip i-1 and the first n_post frames of
+// clip i+1 (local context, absent at the video ends), and n_global frames
+// sampled every floor(F/n_global) frames over the whole video (global
+// context).  Duplicates are kept; the scale is 1/sqrt(d).
+//
+// On the pages each clip sits on its own GPU and the context frames arrive by
+// an all_gather plus two neighbour exchanges.  Here the clip partition is the
+// kernel grid: a CTA owns a run of clips of one (position, head), and the
+// neighbours' frames are simply the adjacent rows of the [P][F][C] layout.
+//
+// Fast path (bf16, L = 16, d = 64, n_pre, n_post <= 8, n_global <= 16):
+//   CTA = (position p, block of 8 clips = 128 frames, head h), 8 warps.
+//   One thread issues five TMA loads (128B-swizzled, one mbarrier):
+//     Q   rows f0 .. f0+127                       16 KB
+//     K,V rows f0-8 .. f0+135 ("window")          18 KB each
+//     K,V rows j*stride, j < 16 ("global")         2 KB each
+//   Rows outside [0, F) arrive as zeros and are masked out of the softmax.
+//   Warp w owns clip 8*blk + w: its 48 keys are window rows 16w .. 16w+31
+//   (C_pre | own | C_post) plus the 16 global rows.  S = Q K^T and O = P V
+//   run on tensor cores (mma.sync m16n8k16, bf16 in, fp32 accumulate: 24 +
+//   24 instructions per warp), the softmax in fp32 registers with quad
+//   shuffles; P is rounded to bf16 for the PV product and the row sums use
+//   the rounded values.  O goes back through the Q buffer and one TMA store.
+//   HBM traffic per token and head: q, k, v, out once each (4 x 128 B); the
+//   halo and global rows are re-read by neighbouring CTAs from L2.
+// Generic path (fp32 I/O, or shapes outside the fast path): one warp per
+//   (position, head, query frame), keys streamed with an online softmax in
+//   fp32, expf, and the exact key list walked in order.
+#include "ptx.cuh"
+#include "vi_internal.cuh"
+
+namespace vi {
+
+// ---------------------------------------------------------------------------
+// Generic path.
+
+// Frame of entry t in clip i's key list (own, C_pre, C_post, C_global).
+__device__ __forceinline__ int key_frame(int t, int i, int L, int N, int n_pre, int n_post,
+                                         int gstride) {
+  const int s = i * L;
+  if (t < L) return s + t;
+  t -= L;
+  if (i > 0) {
+    if (t < n_pre) return s - n_pre + t;
+    t -= n_pre;
+  }
+  if (i < N - 1) {
+    if (t < n_post) return s + L + t;
+    t -= n_post;
+  }
+  return t * gstride;
+}
+
+template <typename T, int DPL>
+__global__ void __launch_bounds__(256) dual_attn_generic(const T* __restrict__ q,
+                                                         const T* __restrict__ k,
+                                                         const T* __restrict__ v,
+                                                         T* __restrict__ out, int F, int N, int P,
+                                                         int heads, int n_pre, int n_post,
+                                                         int n_global, float scale) {
+  constexpr int D = 32 * DPL;
+  const int lane = threadIdx.x & 31;
+  const int64_t wid = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (wid >= (int64_t)P * heads * F) return;
+  const int f = (int)(wid % F);
+  const int h = (int)((wid / F) % heads);
+  const int64_t p = wid / ((int64_t)F * heads);
+  const int C = heads * D, L = F / N, i = f / L;
+  const int64_t pbase = p * F * C + (int64_t)h * D + lane * DPL;
+  const int gstride = n_global > 0 ? F / n_global : 1;
+  const int nk = L + (i > 0 ? n_pre : 0) + (i < N - 1 ? n_post : 0) + n_global;
+
+  float qv[DPL], acc[DPL];
+#pragma unroll
+  for (int e = 0; e < DPL; ++e) {
+    qv[e] = to_f32(q[pbase + (int64_t)f * C + e]);
+    acc[e] = 0.f;
+  }
+  float m = -INFINITY, l = 0.f;
+  for (int t = 0; t < nk; ++t) {
+    const int64_t off = pbase + (int64_t)key_frame(t, i, L, N, n_pre, n_post, gstride) * C;
+    float dot = 0.f;
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) dot = fmaf(qv[e], to_f32(k[off + e]), dot);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+    const float s = dot * scale;
+    const float mn = fmaxf(m, s);
+    const float alpha = expf(m - mn);      // exp(-inf) = 0 on the first key
+    const float pe = expf(s - mn);
+    l = l * alpha + pe;
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) acc[e] = fmaf(pe, to_f32(v[off + e]), acc[e] * alpha);
+    m = mn;
+  }
+  const float inv = 1.f / l;
+#pragma unroll
+  for (int e = 0; e < DPL; ++e) out[pbase + (int64_t)f * C + e] = from_f32<T>(acc[e] * inv);
+}
+
+template <typename T>
+int dual_attn_generic_launch(const T* q, const T* k, const T* v, T* out, int F, int N, int P,
+                             int heads, int d, int n_pre, int n_post, int n_global,
+                             cudaStream_t stream) {
+  const int64_t warps = (int64_t)P * heads * F;
+  const int64_t blocks = (warps + 7) / 8;
+  if (blocks > 0x7fffffff) return VI_ERR_UNSUPPORTED;
+  const float scale = 1.0f / sqrtf((float)d);
+  if (d == 64)
+    dual_attn_generic<T, 2><<<(unsigned)blocks, 256, 0, stream>>>(q, k, v, out, F, N, P, heads,
+                                                                  n_pre, n_post, n_global, scale);
+  else
+    return VI_ERR_UNSUPPORTED;
+  VI_CUDA_TRY(cudaGetLastError());
+  return VI_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Fast path: TMA staging + mma.sync tensor-core tiles.
+
+constexpr int FA_CLIPS = 8;                       // clips per CTA (one per warp)
+constexpr int FA_L = 16;                          // frames per clip
+constexpr int FA_HALO = 8;                        // max n_pre / n_post
+constexpr int FA_NG = 16;                         // max n_global
+constexpr int FA_ROWS_Q = FA_CLIPS * FA_L;        // 128 query rows
+constexpr int FA_ROWS_W = FA_ROWS_Q + 2 * FA_HALO;  // 144 window rows
+constexpr int FA_ROW_BYTES = 128;                 // 64 bf16 channels of one head
+constexpr uint32_t FA_OFF_Q = 0;
+constexpr uint32_t FA_OFF_KW = FA_OFF_Q + FA_ROWS_Q * FA_ROW_BYTES;     // 16384
+constexpr uint32_t FA_OFF_VW = FA_OFF_KW + FA_ROWS_W * FA_ROW_BYTES;    // 34816
+constexpr uint32_t FA_OFF_KG = FA_OFF_VW + FA_ROWS_W * FA_ROW_BYTES;    // 53248
+constexpr uint32_t FA_OFF_VG = FA_OFF_KG + FA_NG * FA_ROW_BYTES;        // 55296
+constexpr uint32_t FA_OFF_BAR = FA_OFF_VG + FA_NG * FA_ROW_BYTES;       // 57344
+constexpr uint32_t FA_SMEM_BYTES = FA_OFF_BAR + 16 + 1024;  // + slack for 1024B alignment
+static_assert(FA_OFF_KW % 1024 == 0 && FA_OFF_VW % 1024 == 0 && FA_OFF_KG % 1024 == 0 &&
+                  FA_OFF_VG % 1024 == 0,
+              "128B-swizzled regions must start on 1024-byte boundaries");
+
+// Byte address of 16-byte chunk `chunk` of row `row` in a 128B-swizzled region.
+__device__ __forceinline__ uint32_t sw128(uint32_t region, int row, int chunk) {
+  return region + row * FA_ROW_BYTES + (((chunk ^ (row & 7)) & 7) << 4);
+}
+
+struct FaMaps {
+  CUtensorMap q, k, v, kg, vg, o;
+};
+
+__global__ void __launch_bounds__(256) dual_attn_bf16_mma(const __grid_constant__ FaMaps maps,
+                                                          int F, int N, int heads, int nblk,
+                                                          int n_pre, int n_post, int n_global,
+                                                          float scale_log2,
+                                                          unsigned int* err_word) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  const uint32_t sQ = base + FA_OFF_Q, sKW = base + FA_OFF_KW, sVW = base + FA_OFF_VW;
+  const uint32_t sKG = base + FA_OFF_KG, sVG = base + FA_OFF_VG, bar = base + FA_OFF_BAR;
+
+  const int blk = blockIdx.x % nblk;
+  const int h = (blockIdx.x / nblk) % heads;
+  const int p = blockIdx.x / (nblk * heads);
+  const int f0 = blk * FA_ROWS_Q;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const uint32_t bytes = (FA_ROWS_Q + 2 * FA_ROWS_W) * FA_ROW_BYTES +
+                           (n_global > 0 ? 2 * FA_NG * FA_ROW_BYTES : 0);
+    mbar_arrive_expect_tx(bar, bytes);
+    tma_load_3d(sQ, &maps.q, h * 64, f0, p, bar);
+    tma_load_3d(sKW, &maps.k, h * 64, f0 - FA_HALO, p, bar);
+    tma_load_3d(sVW, &maps.v, h * 64, f0 - FA_HALO, p, bar);
+    if (n_global > 0) {
+      tma_load_3d(sKG, &maps.kg, h * 64, 0, p, bar);
+      tma_load_3d(sVG, &maps.vg, h * 64, 0, p, bar);
+    }
+  }
+  if (!mbar_wait_bounded(bar, 0, err_word, VI_DEV_ERR_TMA_TIMEOUT)) return;
+
+  const int clip = blk * FA_CLIPS + warp;
+  if (clip < N) {
+    const int g = lane >> 2, qd = lane & 3;
+    // ---- S = Q K^T over 48 keys (6 n-tiles of 8), 4 k-steps of 16 dims ----
+    uint32_t qa[4][4];
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks)
+      ldsm_x4(sw128(sQ, warp * 16 + (lane & 15), 2 * ks + (lane >> 4)), qa[ks][0], qa[ks][1],
+              qa[ks][2], qa[ks][3]);
+    float s[6][4];
+#pragma unroll
+    for (int nt = 0; nt < 6; ++nt) {
+      s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+      const uint32_t region = nt < 4 ? sKW : sKG;
+      const int row = nt < 4 ? warp * 16 + nt * 8 + (lane & 7) : (nt - 4) * 8 + (lane & 7);
+#pragma unroll
+      for (int kp = 0; kp < 2; ++kp) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(sw128(region, row, 4 * kp + (lane >> 3)), b0, b1, b2, b3);
+        mma_bf16_16816(s[nt], qa[2 * kp], b0, b1);
+        mma_bf16_16816(s[nt], qa[2 * kp + 1], b2, b3);
+      }
+    }
+    // ---- mask absent keys, softmax in log2 units ----
+    float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+    for (int nt = 0; nt < 6; ++nt) {
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const int kk = nt * 8 + 2 * qd + c;     // key index in the warp's list
+        bool valid;
+        if (kk < FA_HALO) valid = clip > 0 && kk >= FA_HALO - n_pre;
+        else if (kk < FA_HALO + FA_L) valid = true;
+        else if (kk < 32) valid = clip < N - 1 && kk - (FA_HALO + FA_L) < n_post;
+        else valid = kk - 32 < n_global;
+        s[nt][c] = valid ? s[nt][c] * scale_log2 : -INFINITY;
+        s[nt][c + 2] = valid ? s[nt][c + 2] * scale_log2 : -INFINITY;
+        mx0 = fmaxf(mx0, s[nt][c]);
+        mx1 = fmaxf(mx1, s[nt][c + 2]);
+      }
+    }
+#pragma unroll
+    for (int o = 1; o <= 2; o <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+    }
+    // P in bf16 as mma A fragments: k-step ks covers keys 16ks .. 16ks+15.
+    uint32_t pa[3][4];
+    float l0 = 0.f, l1 = 0.f;
+#pragma unroll
+    for (int nt = 0; nt < 6; ++nt) {
+      const uint32_t lo = pack2_bf16(exp2f(s[nt][0] - mx0), exp2f(s[nt][1] - mx0));
+      const uint32_t hi = pack2_bf16(exp2f(s[nt][2] - mx1), exp2f(s[nt][3] - mx1));
+      l0 += __uint_as_float(lo << 16) + __uint_as_float(lo & 0xFFFF0000u);
+      l1 += __uint_as_float(hi << 16) + __uint_as_float(hi & 0xFFFF0000u);
+      pa[nt >> 1][(nt & 1) * 2 + 0] = lo;
+      pa[nt >> 1][(nt & 1) * 2 + 1] = hi;
+    }
+#pragma unroll
+    for (int o = 1; o <= 2; o <<= 1) {
+      l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+    }
+    // ---- O = P V: 3 k-steps of 16 keys x 8 n-tiles of 8 dims ----
+    float o[8][4];
+#pragma unroll
+    for (int nd = 0; nd < 8; ++nd) o[nd][0] = o[nd][1] = o[nd][2] = o[nd][3] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < 3; ++ks) {
+      const uint32_t region = ks < 2 ? sVW : sVG;
+      const int row = (ks < 2 ? warp * 16 + ks * 16 : 0) + (lane & 15);
+#pragma unroll
+      for (int nd = 0; nd < 8; nd += 2) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(sw128(region, row, nd + (lane >> 4)), b0, b1, b2, b3);
+        mma_bf16_16816(o[nd], pa[ks], b0, b1);
+        mma_bf16_16816(o[nd + 1], pa[ks], b2, b3);
+      }
+    }
+    // ---- normalise, round, write this warp's 16 rows into the Q buffer ----
+    const float inv0 = 1.f / l0, inv1 = 1.f / l1;
+    const int r0 = warp * 16 + g, r1 = r0 + 8;
+#pragma unroll
+    for (int nd = 0; nd < 8; ++nd) {
+      const uint32_t w0 = pack2_bf16(o[nd][0] * inv0, o[nd][1] * inv0);
+      const uint32_t w1 = pack2_bf16(o[nd][2] * inv1, o[nd][3] * inv1);
+      asm volatile("st.shared.b32 [%0], %1;" ::"r"(sw128(sQ, r0, nd) + 4 * qd), "r"(w0));
+      asm volatile("st.shared.b32 [%0], %1;" ::"r"(sw128(sQ, r1, nd) + 4 * qd), "r"(w1));
+    }
+  }
+  fence_proxy_async_smem();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    tma_store_3d(&maps.o, sQ, h * 64, f0, p);
+    tma_store_commit_and_drain();
+  }
+}
+
+// Host: tensor maps over [P][F][C] bf16 with 128B swizzle.
+bool encode_tmap(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                 const uint64_t* strides_bytes, const uint32_t* box, CUtensorMapSwizzle swz,
+                 CUtensorMapDataType dt);
+
+int dual_attn_bf16_fast(const bf16* q, const bf16* k, const bf16* v, bf16* out, int F, int N,
+                        int P, int heads, int n_pre, int n_post, int n_global,
+                        cudaStream_t stream) {
+  const int C = heads * 64;
+  FaMaps maps;
+  const uint64_t dims[3] = {(uint64_t)C, (uint64_t)F, (uint64_t)P};
+  const uint64_t strides[2] = {(uint64_t)C * 2, (uint64_t)F * C * 2};
+  const uint32_t boxQ[3] = {64, FA_ROWS_Q, 1}, boxW[3] = {64, FA_ROWS_W, 1};
+  const CUtensorMapDataType BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const CUtensorMapSwizzle SW = CU_TENSOR_MAP_SWIZZLE_128B;
+  bool ok = encode_tmap(&maps.q, q, 3, dims, strides, boxQ, SW, BF) &&
+            encode_tmap(&maps.k, k, 3, dims, strides, boxW, SW, BF) &&
+            encode_tmap(&maps.v, v, 3, dims, strides, boxW, SW, BF) &&
+            encode_tmap(&maps.o, out, 3, dims, strides, boxQ, SW, BF);
+  if (n_global > 0) {
+    const int gs = F / n_global;
+    const uint64_t gdims[3] = {(uint64_t)C, (uint64_t)n_global, (uint64_t)P};
+    const uint64_t gstrides[2] = {(uint64_t)gs * C * 2, (uint64_t)F * C * 2};
+    const uint32_t boxG[3] = {64, FA_NG, 1};
+    ok = ok && encode_tmap(&maps.kg, k, 3, gdims, gstrides, boxG, SW, BF) &&
+         encode_tmap(&maps.vg, v, 3, gdims, gstrides, boxG, SW, BF);
+  } else {
+    maps.kg = maps.k;
+    maps.vg = maps.v;
+  }
+  if (!ok) return VI_ERR_CUDA;
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  VI_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 64 && !attr_set[dev]) {
+    VI_CUDA_TRY(cudaFuncSetAttribute(dual_attn_bf16_mma,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, FA_SMEM_BYTES));
+    attr_set[dev] = true;
+  }
+  const int nblk = (N + FA_CLIPS - 1) / FA_CLIPS;
+  const int64_t grid = (int64_t)P * heads * nblk;
+  if (grid > 0x7fffffff) return VI_ERR_UNSUPPORTED;
+  const float scale_log2 = 1.4426950408889634f / 8.0f;    // log2(e) / sqrt(64)
+  unsigned int* err = device_error_word();
+  if (!err) return VI_ERR_CUDA;
+  dual_attn_bf16_mma<<<(unsigned)grid, 256, FA_SMEM_BYTES, stream>>>(
+      maps, F, N, heads, nblk, n_pre, n_post, n_global, scale_log2, err);
+  VI_CUDA_TRY(cudaGetLastError());
+  return VI_OK;
+}
+
+bool dual_attn_fast_ok(int F, int N, int d, int n_pre, int n_post, int n_global) {
+  return d == 64 && F / N == FA_L && n_pre <= FA_HALO && n_post <= FA_HALO &&
+         n_global <= FA_NG;
+}
+
+template int dual_attn_generic_launch<float>(const float*, const float*, const float*, float*,
+                                             int, int, int, int, int, int, int, int,
+                                             cudaStream_t);
+template int dual_attn_generic_launch<bf16>(const bf16*, const bf16*, const bf16*, bf16*, int,
+                                            int, int, int, int, int, int, int, cudaStream_t);
+
+}  // namespace vi

@@ -1,0 +1,234 @@
+// extern "C" entry points of libvi: host-side argument checks, then dispatch
+// to the kernels.  Nothing is launched unless every check passes.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <math.h>
+#include <mutex>
+
+#include "ptx.cuh"
+#include "vi_internal.cuh"
+
+namespace vi {
+
+static __device__ unsigned int g_device_error = 0u;
+
+unsigned int* device_error_word() {
+  static void* cached[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (!cached[dev] && cudaGetSymbolAddress(&cached[dev], g_device_error) != cudaSuccess)
+    cached[dev] = nullptr;
+  return static_cast<unsigned int*>(cached[dev]);
+}
+
+// Kernel launchers (defined next to their kernels).
+template <typename T>
+int dual_attn_generic_launch(const T*, const T*, const T*, T*, int, int, int, int, int, int, int,
+                             int, cudaStream_t);
+int dual_attn_bf16_fast(const bf16*, const bf16*, const bf16*, bf16*, int, int, int, int, int,
+                        int, int, cudaStream_t);
+bool dual_attn_fast_ok(int F, int N, int d, int n_pre, int n_post, int n_global);
+template <typename T>
+int temporal_conv_generic_launch(const T*, const T*, const T*, T*, int, int, int, int,
+                                 cudaStream_t);
+int temporal_conv_bf16_tc(const bf16*, const bf16*, const bf16*, bf16*, int, int, int, int,
+                          cudaStream_t);
+bool temporal_conv_tc_ok(int F, int P, int C, int k);
+template <typename T>
+int groupnorm_global(const T*, const T*, const T*, T*, int64_t, int, int, float, cudaStream_t);
+
+int sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev >= 0 && dev < 64 && cached[dev] > 0) return cached[dev];
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    n = 148;
+  if (dev >= 0 && dev < 64) cached[dev] = n;
+  return n;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
+static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+bool encode_tmap(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                 const uint64_t* strides_bytes, const uint32_t* box, CUtensorMapSwizzle swz,
+                 CUtensorMapDataType dt) {
+  auto fn = get_encode();
+  if (!fn) return false;
+  cuuint64_t d[5], s[4];
+  cuuint32_t bx[5], es[5];
+  for (int i = 0; i < rank; ++i) {
+    d[i] = dims[i];
+    bx[i] = box[i];
+    es[i] = 1;
+    if (i + 1 < rank) s[i] = strides_bytes[i];
+  }
+  const CUresult r = fn(map, dt, (cuuint32_t)rank, const_cast<void*>(base), d, s, bx, es,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace vi
+
+using namespace vi;
+
+namespace {
+
+inline cudaStream_t as_stream(vi_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// Sizes shared by all three calls.
+int check_clips(int F, int N, int P, int C) {
+  if (F <= 0 || N <= 0 || P <= 0 || C <= 0) return VI_ERR_INVALID_ARG;
+  if (F % N != 0) return VI_ERR_INVALID_ARG;
+  // Element offsets are 64-bit; cap the tensor at 2^40 elements.
+  if ((double)P * (double)F * (double)C > 1.099511627776e12) return VI_ERR_UNSUPPORTED;
+  return VI_OK;
+}
+
+template <typename T>
+int attn_entry(const void* q, const void* k, const void* v, void* out, int F, int N, int P,
+               int heads, int d, int n_pre, int n_post, int n_global, vi_stream_t stream) {
+  if (!q || !k || !v || !out) return VI_ERR_INVALID_ARG;
+  if (heads <= 0 || d <= 0) return VI_ERR_INVALID_ARG;
+  if ((int64_t)heads * d > 0x7fffffff) return VI_ERR_INVALID_ARG;
+  const int C = heads * d;
+  int st = check_clips(F, N, P, C);
+  if (st != VI_OK) return st;
+  const int L = F / N;
+  if (n_pre < 0 || n_post < 0 || n_global < 0 || n_global > F) return VI_ERR_INVALID_ARG;
+  if (N > 1 && (n_pre > L || n_post > L)) return VI_ERR_INVALID_ARG;
+  if (d != 64) return VI_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return VI_ERR_ALIGNMENT;
+  if ((C * sizeof(T)) % 16 != 0) return VI_ERR_ALIGNMENT;
+  const size_t bytes = (size_t)P * F * C * sizeof(T);
+  if (overlaps(out, bytes, q, bytes) || overlaps(out, bytes, k, bytes) ||
+      overlaps(out, bytes, v, bytes))
+    return VI_ERR_INVALID_ARG;
+  const T* qq = static_cast<const T*>(q);
+  const T* kk = static_cast<const T*>(k);
+  const T* vv = static_cast<const T*>(v);
+  T* oo = static_cast<T*>(out);
+  if constexpr (sizeof(T) == 2) {
+    if (dual_attn_fast_ok(F, N, d, n_pre, n_post, n_global))
+      return dual_attn_bf16_fast(qq, kk, vv, oo, F, N, P, heads, n_pre, n_post, n_global,
+                                 as_stream(stream));
+  }
+  return dual_attn_generic_launch<T>(qq, kk, vv, oo, F, N, P, heads, d, n_pre, n_post, n_global,
+                                     as_stream(stream));
+}
+
+template <typename T>
+int conv_entry(const void* x, const void* w, const void* b, void* y, int F, int N, int P, int C,
+               int k, vi_stream_t stream) {
+  if (!x || !w || !b || !y) return VI_ERR_INVALID_ARG;
+  int st = check_clips(F, N, P, C);
+  if (st != VI_OK) return st;
+  if (k <= 0 || k % 2 == 0 || k / 2 > F / N) return VI_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w) || !aligned16(b) || !aligned16(y)) return VI_ERR_ALIGNMENT;
+  if ((C * sizeof(T)) % 16 != 0) return VI_ERR_ALIGNMENT;
+  const size_t bytes = (size_t)P * F * C * sizeof(T);
+  const size_t wbytes = (size_t)C * C * k * sizeof(T), bbytes = (size_t)C * sizeof(T);
+  if (overlaps(y, bytes, x, bytes) || overlaps(y, bytes, w, wbytes) || overlaps(y, bytes, b, bbytes))
+    return VI_ERR_INVALID_ARG;
+  const T* xx = static_cast<const T*>(x);
+  const T* ww = static_cast<const T*>(w);
+  const T* bb = static_cast<const T*>(b);
+  T* yy = static_cast<T*>(y);
+  if constexpr (sizeof(T) == 2) {
+    if (temporal_conv_tc_ok(F, P, C, k))
+      return temporal_conv_bf16_tc(xx, ww, bb, yy, F, P, C, k, as_stream(stream));
+  }
+  return temporal_conv_generic_launch<T>(xx, ww, bb, yy, F, P, C, k, as_stream(stream));
+}
+
+template <typename T>
+int gn_entry(const void* x, const void* gamma, const void* beta, void* y, int F, int N, int P,
+             int C, int groups, float eps, vi_stream_t stream) {
+  if (!x || !gamma || !beta || !y) return VI_ERR_INVALID_ARG;
+  int st = check_clips(F, N, P, C);
+  if (st != VI_OK) return st;
+  if (groups <= 0 || C % groups != 0) return VI_ERR_INVALID_ARG;
+  if (!(eps >= 0.f) || !isfinite(eps)) return VI_ERR_INVALID_ARG;
+  if (groups > 1024) return VI_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(gamma) || !aligned16(beta) || !aligned16(y))
+    return VI_ERR_ALIGNMENT;
+  if ((C * sizeof(T)) % 16 != 0) return VI_ERR_ALIGNMENT;
+  const size_t bytes = (size_t)P * F * C * sizeof(T);
+  if (y != x && overlaps(y, bytes, x, bytes)) return VI_ERR_INVALID_ARG;
+  if (overlaps(y, bytes, gamma, C * sizeof(T)) || overlaps(y, bytes, beta, C * sizeof(T)))
+    return VI_ERR_INVALID_ARG;
+  return groupnorm_global<T>(static_cast<const T*>(x), static_cast<const T*>(gamma),
+                             static_cast<const T*>(beta), static_cast<T*>(y), (int64_t)P * F, C,
+                             groups, eps, as_stream(stream));
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* vi_status_string(int status) {
+  switch (status) {
+    case VI_OK: return "VI_OK";
+    case VI_ERR_INVALID_ARG: return "VI_ERR_INVALID_ARG";
+    case VI_ERR_ALIGNMENT: return "VI_ERR_ALIGNMENT";
+    case VI_ERR_UNSUPPORTED: return "VI_ERR_UNSUPPORTED";
+    case VI_ERR_CUDA: return "VI_ERR_CUDA";
+    case VI_ERR_DEVICE_TIMEOUT: return "VI_ERR_DEVICE_TIMEOUT";
+    default: return "VI_ERR_UNKNOWN";
+  }
+}
+
+int vi_version(void) { return 100; }
+
+int vi_take_device_errors(void) {
+  if (!device_error_word()) return VI_ERR_CUDA;
+  if (cudaDeviceSynchronize() != cudaSuccess) return VI_ERR_CUDA;
+  unsigned int word = 0u, zero = 0u;
+  if (cudaMemcpyFromSymbol(&word, g_device_error, sizeof(word)) != cudaSuccess) return VI_ERR_CUDA;
+  if (word != 0u && cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)) != cudaSuccess)
+    return VI_ERR_CUDA;
+  return word ? VI_ERR_DEVICE_TIMEOUT : VI_OK;
+}
+
+int vi_dual_attn(const void* q, const void* k, const void* v, void* out, int F, int N, int P,
+                 int heads, int d, int n_pre, int n_post, int n_global, vi_stream_t stream) {
+  return attn_entry<bf16>(q, k, v, out, F, N, P, heads, d, n_pre, n_post, n_global, stream);
+}
+int vi_dual_attn_f32(const void* q, const void* k, const void* v, void* out, int F, int N, int P,
+                     int heads, int d, int n_pre, int n_post, int n_global, vi_stream_t stream) {
+  return attn_entry<float>(q, k, v, out, F, N, P, heads, d, n_pre, n_post, n_global, stream);
+}
+int vi_temporal_conv(const void* x, const void* w, const void* b, void* y, int F, int N, int P,
+                     int C, int k, vi_stream_t stream) {
+  return conv_entry<bf16>(x, w, b, y, F, N, P, C, k, stream);
+}
+int vi_temporal_conv_f32(const void* x, const void* w, const void* b, void* y, int F, int N,
+                         int P, int C, int k, vi_stream_t stream) {
+  return conv_entry<float>(x, w, b, y, F, N, P, C, k, stream);
+}
+int vi_groupnorm_global(const void* x, const void* gamma, const void* beta, void* y, int F, int N,
+                        int P, int C, int groups, float eps, vi_stream_t stream) {
+  return gn_entry<bf16>(x, gamma, beta, y, F, N, P, C, groups, eps, stream);
+}
+int vi_groupnorm_global_f32(const void* x, const void* gamma, const void* beta, void* y, int F,
+                            int N, int P, int C, int groups, float eps, vi_stream_t stream) {
+  return gn_entry<float>(x, gamma, beta, y, F, N, P, C, groups, eps, stream);
+}
+
+}  // extern "C"

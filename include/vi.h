@@ -1,0 +1,148 @@
+/*
+ * vi.h -- C ABI of libvi, the B200 (sm_100a) kernels for the clip-parallel
+ * temporal modules of a video-diffusion U-Net (Video-Infinity).
+ *
+ * Source of every operation: "Video-Infinity: Distributed Long Video
+ * Generation" (write-up on news.43zhubao.com), the paragraphs on clip
+ * parallelism and on the three temporal modules: dual-domain attention, the
+ * temporal convolution, and GroupNorm.  The pages distribute the N clips of a
+ * video over N GPUs and synchronise context between them; here all N clips
+ * live on one GPU and each call partitions them inside one kernel grid.
+ *
+ * Common conventions
+ * ------------------
+ * Layout.  Every activation (q, k, v, out, x, y) is a dense row-major array
+ *   [P positions][F frames][C channels], C innermost, with C = heads * d for
+ *   attention.  P = H'*W' is the latent's spatial size.  Frames of one
+ *   position are contiguous, so a clip and its neighbours are adjacent.
+ * Clips.  F frames are cut into N clips of L = F / N frames; F % N == 0.
+ * Types.  The un-suffixed entry points take bf16 tensors (IEEE bfloat16, bit
+ *   patterns in uint16 storage) and accumulate in fp32; the _f32 entry points
+ *   take fp32 tensors and compute in fp32 on CUDA cores (no TF32).  Small
+ *   parameter vectors (conv weight and bias, GroupNorm gamma and beta) have
+ *   the same type as the activations.
+ * Pointers.  Every array pointer is a DEVICE pointer on the current CUDA
+ *   device, 16-byte aligned, owned by the caller before and after the call.
+ *   The library keeps no pointer after the call returns.
+ * Streams.  `stream` is a cudaStream_t (NULL = the legacy default stream).
+ *   Calls enqueue work on it and return without synchronising; the outputs
+ *   are ready when the stream reaches that point.  Scratch memory the library
+ *   needs is taken from the stream-ordered allocator on that stream and given
+ *   back on it (cudaMallocAsync / cudaFreeAsync).  Calls on different streams
+ *   may run concurrently; calls on one stream run in order.
+ * Errors.  Every argument is checked on the host before anything is launched;
+ *   a failed check returns a negative vi_status and enqueues nothing.
+ *   VI_ERR_CUDA reports a CUDA error seen while launching.  A fault that
+ *   happens on the device later surfaces, as usual in CUDA, at the caller's
+ *   next synchronisation.
+ */
+#ifndef VI_H_
+#define VI_H_
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;                 /* == cudaStream_t's pointee */
+typedef struct CUstream_st* vi_stream_t;
+
+typedef enum {
+  VI_OK = 0,
+  VI_ERR_INVALID_ARG = -1,  /* null pointer, non-positive size, F % N != 0, ... */
+  VI_ERR_ALIGNMENT = -2,    /* pointer not 16-byte aligned, or C * sizeof(T) % 16 != 0 */
+  VI_ERR_UNSUPPORTED = -3,  /* valid request outside what the library implements */
+  VI_ERR_CUDA = -4,         /* a CUDA runtime/driver call failed while enqueuing */
+  VI_ERR_DEVICE_TIMEOUT = -5  /* a kernel's bounded wait ran out (see vi_take_device_errors) */
+} vi_status;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* vi_status_string(int status);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int vi_version(void);
+
+/*
+ * Kernels that wait on an asynchronous copy or tensor-core operation bound
+ * that wait (2 s of device time); when it runs out they record the fact in a
+ * device-side error word and return early instead of hanging the GPU.  This
+ * call synchronises the current device, reads and clears that word, and
+ * returns VI_OK if no wait ran out since the last call, VI_ERR_DEVICE_TIMEOUT
+ * otherwise (or VI_ERR_CUDA if the synchronisation itself failed).
+ */
+int vi_take_device_errors(void);
+
+/*
+ * Dual-domain temporal attention (attention-module paragraph of the source).
+ *
+ * For every position p, head h and clip i (frames [s, e), s = i*L, e = s+L),
+ * each query frame f in [s, e) attends over the clip's key/value frame list
+ *   own clip      s .. e-1
+ *   C_pre         s-n_pre .. s-1          only if i > 0     (end of clip i-1)
+ *   C_post        e .. e+n_post-1         only if i < N-1   (start of clip i+1)
+ *   C_global      j * floor(F/n_global)   for j < n_global  (same for all clips)
+ * concatenated without de-duplication (a frame listed twice counts twice):
+ *   out[p,f,h,:] = sum_j softmax_j(q[p,f,h,:].k[p,j,h,:] / sqrt(d)) v[p,j,h,:]
+ * Absent context at the video ends is left out of the softmax (not zero keys).
+ *
+ * q, k, v, out : [P][F][heads*d] (bf16, or fp32 for _f32); out must not
+ *                overlap q, k or v.
+ * Requirements : all sizes > 0 except the context sizes (>= 0); F % N == 0;
+ *                d == 64; if N > 1 then n_pre <= L and n_post <= L;
+ *                n_global <= F.  Otherwise VI_ERR_INVALID_ARG, or
+ *                VI_ERR_UNSUPPORTED for d != 64.
+ * Scratch      : none.
+ */
+int vi_dual_attn(const void* q, const void* k, const void* v, void* out, int F, int N, int P,
+                 int heads, int d, int n_pre, int n_post, int n_global, vi_stream_t stream);
+int vi_dual_attn_f32(const void* q, const void* k, const void* v, void* out, int F, int N, int P,
+                     int heads, int d, int n_pre, int n_post, int n_global, vi_stream_t stream);
+
+/*
+ * Temporal convolution with neighbour padding (conv-module paragraph).
+ *
+ * Each clip is extended by n = k/2 frames on each side, taken from the end of
+ * the previous clip and the start of the next one, with zeros at the two ends
+ * of the video; a valid cross-correlation over the extended clip gives
+ *   y[p,f,co] = b[co] + sum_{t<k} sum_ci w[co,ci,t] * x[p, f+t-n, ci]
+ * with x = 0 outside [0, F).  Because the neighbours' frames are exactly the
+ * frames the unpartitioned sequence has there, the result equals the
+ * zero-padded Conv1d of the whole video, and does not depend on N.
+ *
+ * x, y : [P][F][C];  w : [C_out=C][C_in=C][k] (PyTorch Conv1d order);  b : [C].
+ * Requirements : sizes > 0; F % N == 0; k odd; k/2 <= L; y must not overlap
+ *                x, w or b.  Otherwise VI_ERR_INVALID_ARG.
+ * Scratch      : the bf16 path repacks w into a stream-ordered scratch buffer
+ *                of k*C*C*2 bytes, freed on the stream after the kernel.
+ */
+int vi_temporal_conv(const void* x, const void* w, const void* b, void* y, int F, int N, int P,
+                     int C, int k, vi_stream_t stream);
+int vi_temporal_conv_f32(const void* x, const void* w, const void* b, void* y, int F, int N,
+                         int P, int C, int k, vi_stream_t stream);
+
+/*
+ * GroupNorm with global statistics (GroupNorm-module paragraph).
+ *
+ * Group g holds the C/groups contiguous channels [g*C/G, (g+1)*C/G).  Its mean
+ * mu_g is aggregated over every clip (all frames, all positions); the spread
+ * about that global mean is then aggregated over every clip into the global
+ * variance var_g (biased: divided by the element count).  Each element is
+ *   y = (x - mu_g) / sqrt(var_g + eps) * gamma[c] + beta[c]
+ * which equals GroupNorm (batch 1) of the unpartitioned latent for any N.
+ *
+ * x, y : [P][F][C] (y may equal x: in place);  gamma, beta : [C].
+ * Requirements : sizes > 0; F % N == 0; C % groups == 0; eps >= 0 and finite.
+ *                y may alias x exactly but must not partly overlap it.
+ * Scratch      : (24 * groups * blocks + 8*C + 64) bytes of stream-ordered
+ *                scratch for per-block partial sums and the per-channel
+ *                coefficients, freed on the stream after the last kernel.
+ */
+int vi_groupnorm_global(const void* x, const void* gamma, const void* beta, void* y, int F, int N,
+                        int P, int C, int groups, float eps, vi_stream_t stream);
+int vi_groupnorm_global_f32(const void* x, const void* gamma, const void* beta, void* y, int F,
+                            int N, int P, int C, int groups, float eps, vi_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VI_H_ */

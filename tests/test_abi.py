@@ -1,0 +1,120 @@
+"""The C ABI without a GPU: libvi.so loads, exports every function include/vi.h
+declares, and rejects bad arguments on the host before anything is launched.
+
+Only invalid calls are made here; each one must return its error code from
+the host-side checks, so no CUDA work is enqueued (there is no device)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import clip_temporal_modules_b200 as vi
+from clip_temporal_modules_b200 import _binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "vi.h")
+
+OK, INVALID, ALIGN, UNSUP = 0, -1, -2, -3
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(vi_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from clip_temporal_modules_b200 import build
+    build.build()
+    return vi.lib()
+
+
+def test_every_declared_function_is_exported(L):
+    names = declared_functions()
+    assert {"vi_dual_attn", "vi_temporal_conv", "vi_groupnorm_global"} <= set(names)
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings_and_version(L):
+    assert L.vi_status_string(0) == b"VI_OK"
+    assert L.vi_status_string(-2) == b"VI_ERR_ALIGNMENT"
+    assert L.vi_status_string(-5) == b"VI_ERR_DEVICE_TIMEOUT"
+    assert L.vi_status_string(7) == b"VI_ERR_UNKNOWN"
+    assert L.vi_version() >= 100
+
+
+A = 1 << 20          # fake 16-byte-aligned "device" addresses, never dereferenced
+B = 1 << 30
+Cp = 1 << 31
+D = 1 << 32
+
+
+def attn(L, q=A, k=B, v=Cp, o=D, F=64, N=4, P=2, heads=2, d=64, pre=8, post=8, glob=16,
+         f32=False):
+    fn = L.vi_dual_attn_f32 if f32 else L.vi_dual_attn
+    return fn(q, k, v, o, F, N, P, heads, d, pre, post, glob, None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(q=0), INVALID), (dict(o=0), INVALID),
+    (dict(F=0), INVALID), (dict(N=0), INVALID), (dict(P=-1), INVALID), (dict(heads=0), INVALID),
+    (dict(F=63), INVALID),                      # F % N != 0
+    (dict(pre=17), INVALID),                    # C_pre longer than a clip (L = 16)
+    (dict(post=-1), INVALID), (dict(glob=65), INVALID),
+    (dict(d=32), UNSUP),
+    (dict(q=A + 8), ALIGN), (dict(o=D + 2), ALIGN),
+    (dict(o=A + 64), INVALID),                  # out overlaps q
+])
+def test_attention_rejects(L, kw, expect):
+    assert attn(L, **kw) == expect
+
+
+def test_attention_rejects_f32_too(L):
+    assert attn(L, F=10, N=4, f32=True) == INVALID
+    assert attn(L, v=Cp + 4, f32=True) == ALIGN
+
+
+def conv(L, x=A, w=B, b=Cp, y=D, F=64, N=4, P=2, C=64, k=3, f32=False):
+    fn = L.vi_temporal_conv_f32 if f32 else L.vi_temporal_conv
+    return fn(x, w, b, y, F, N, P, C, k, None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(x=0), INVALID), (dict(b=0), INVALID), (dict(F=62), INVALID), (dict(k=2), INVALID),
+    (dict(k=0), INVALID), (dict(k=35, F=64, N=4), INVALID),   # halo wider than a clip
+    (dict(C=0), INVALID), (dict(C=12), ALIGN),                # 12 bf16 = 24 bytes per row
+    (dict(w=B + 4), ALIGN), (dict(y=A), INVALID),             # y aliases x
+    (dict(y=B - 64), INVALID),                                # y runs into w
+])
+def test_conv_rejects(L, kw, expect):
+    assert conv(L, **kw) == expect
+
+
+def test_conv_f32_row_alignment(L):
+    assert conv(L, C=6, f32=True) == ALIGN      # 24 bytes per row
+    assert conv(L, F=7, N=7, k=3, C=8, f32=True, x=0) == INVALID
+
+
+def gn(L, x=A, g=B, bt=Cp, y=D, F=64, N=4, P=2, C=64, groups=8, eps=1e-5, f32=False):
+    fn = L.vi_groupnorm_global_f32 if f32 else L.vi_groupnorm_global
+    return fn(x, g, bt, y, F, N, P, C, groups, eps, None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(x=0), INVALID), (dict(groups=0), INVALID), (dict(groups=7), INVALID),
+    (dict(eps=-1.0), INVALID), (dict(eps=float("nan")), INVALID), (dict(eps=float("inf")), INVALID),
+    (dict(F=65), INVALID), (dict(groups=2048, C=4096), UNSUP),
+    (dict(g=B + 8), ALIGN), (dict(C=4, groups=4), ALIGN),
+    (dict(y=A + 16), INVALID),                  # partial overlap with x
+])
+def test_groupnorm_rejects(L, kw, expect):
+    assert gn(L, **kw) == expect
+
+
+def test_binding_signatures_cover_header():
+    for n in declared_functions():
+        if n != "vi_status_string":
+            assert n in _binding.SIGNATURES, n

@@ -1,0 +1,83 @@
+"""GPU parity of dual-domain attention against the fp64 oracle.
+
+Source: "Video-Infinity: Distributed Long Video Generation" (news.43zhubao.com
+write-up), attention-module paragraph.  Small cases are compared element by
+element and span several CTA tiles, ragged tails and every branch of the key
+list (absent ends, short context, no global frames, one clip); the five
+workloads run at full size and are compared on sampled positions."""
+import numpy as np
+import pytest
+import torch
+
+import clip_temporal_modules_b200 as vi
+import oracle
+import synth
+from parity import assert_close, from_device, sample_positions, to_device
+
+pytestmark = pytest.mark.gpu
+
+
+def run_case(w: synth.Workload, positions=None):
+    q, k, v = (synth.make(w, t) for t in ("q", "k", "v"))
+    dq, dk, dv = (to_device(a, w.dtype) for a in (q, k, v))
+    out = vi.dual_attn(dq, dk, dv, N=w.N, heads=w.heads, n_pre=w.n_pre, n_post=w.n_post,
+                       n_global=w.n_global)
+    torch.cuda.synchronize()
+    vi.take_device_errors()
+    got = from_device(out)
+    ref = oracle.dual_attn(q, k, v, w.F, w.N, w.heads, w.d, w.n_pre, w.n_post, w.n_global,
+                           positions=positions)
+    if positions is not None:
+        got = got[positions]
+    return assert_close(got, ref, w.dtype, "attn", w.name)
+
+
+def W(name, dtype, F, N, P, heads, **kw):
+    return synth.Workload(name, dtype, F=F, N=N, P=P, C=heads * 64, heads=heads, d=64, **kw)
+
+
+SMALL = [
+    synth.WORKLOADS[0],                                        # tiny fp32 (generic path)
+    W("bf16_1blk_ragged", "bf16", 48, 3, 5, 2),                # fast path, 3 of 8 clips
+    W("bf16_2blk_ragged", "bf16", 160, 10, 3, 3),              # 8 + 2 clips, stride 10
+    W("bf16_short_ctx", "bf16", 64, 4, 4, 2, n_pre=3, n_post=5, n_global=7),
+    W("bf16_no_global", "bf16", 64, 4, 3, 1, n_global=0),
+    W("bf16_one_clip", "bf16", 16, 1, 6, 2, n_global=4),
+    W("bf16_no_context", "bf16", 48, 3, 2, 1, n_pre=0, n_post=0, n_global=0),
+    W("bf16_L8_generic", "bf16", 32, 4, 4, 2),                 # L = 8: generic path
+    W("bf16_L32_generic", "bf16", 64, 2, 3, 1, n_pre=16, n_post=12, n_global=20),
+    W("f32_generic", "f32", 48, 3, 3, 2),
+    W("f32_L16_short", "f32", 64, 4, 2, 1, n_pre=2, n_post=0, n_global=5),
+]
+
+
+@pytest.mark.parametrize("w", SMALL, ids=lambda w: w.name)
+def test_small_elementwise(cuda_device, w):
+    run_case(w)
+
+
+@pytest.mark.parametrize("w", synth.WORKLOADS[1:], ids=lambda w: w.name)
+def test_full_size_sampled_positions(cuda_device, w):
+    run_case(w, positions=sample_positions(w.P))
+
+
+def test_fp32_tiny_full_workload_all_positions(cuda_device):
+    run_case(synth.WORKLOADS[0])
+
+
+def test_runs_on_given_stream_and_leaves_neighbours_untouched(cuda_device):
+    w = W("bf16_stream", "bf16", 64, 4, 3, 2)
+    q, k, v = (to_device(synth.make(w, t), w.dtype) for t in ("q", "k", "v"))
+    n = q.numel()
+    buf = torch.full((n + 64,), 7.0, dtype=torch.bfloat16, device="cuda")
+    out = buf[32:32 + n].view_as(q)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        vi.dual_attn(q, k, v, out, N=w.N, heads=w.heads, stream=s)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    assert torch.all(buf[:32] == 7.0) and torch.all(buf[32 + n:] == 7.0)
+    ref = vi.dual_attn(q, k, v, N=w.N, heads=w.heads)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref)
