@@ -1,0 +1,482 @@
+#!/usr/bin/env python
+"""Throughput of the clip-parallel temporal modules (Video-Infinity) on B200.
+
+One step = one pass of the whole hot path over one latent video: dual-domain
+attention (q, k, v -> out), the clip-padded temporal conv (x -> y) and the
+global-statistics GroupNorm (x' -> z), each through the C ABI of libvi.
+Inputs are seeded synthetic tensors of the workload's shape (the pages'
+512x320 video at a /8 latent, F = 1024 frames in 64 clips by default), already
+resident in HBM when the timed region starts; every tensor (1.68 GB) is larger
+than L2, so no flush is needed between steps.
+
+Metric: temporal-module tokens/s, tokens = F * P (= F * H'W') per step, for
+the whole job (all ranks).  With --gpus N every rank runs its own video
+(weak scaling; the path has no exchange between independent videos).
+
+Printed (rank 0, one JSON line): value, ms_per_step, a per-kernel breakdown,
+the roofline of the dominant kernel (algorithmic bytes or flops over its
+CUDA-event time, against MEASURED_PEAKS.json), the oracle timed on the host
+cores as cpu_baseline, an end-to-end figure through host buffers (e2e), the
+SM clocks sampled during the timed region, and the number of libvi kernel
+launches in the timed region.
+
+--impl reference times the fp64 CPU oracle itself on a bounded sample of the
+same workload (the only reference this method has: the pages ship no code).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+DEFAULT_WORKLOAD = "bf16_F1024_P2560_C320"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "sm_max_mhz": 1965.0}
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="target CPU time of the oracle sample")
+    return ap.parse_args(argv)
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(backend: str):
+    import torch.distributed as dist
+    world, rank, _ = dist_env()
+    if world > 1 and not dist.is_initialized():
+        from datetime import timedelta
+        dist.init_process_group(backend, timeout=timedelta(seconds=120))
+    return world, rank
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ---------------------------------------------------------------------------
+# accounting
+
+
+def kernel_work(w):
+    """Algorithmic bytes (attention, GroupNorm) and flops (conv) per step.
+
+    attention: read q, k, v and write out once: 4 S bytes (halo and global
+               frames are re-reads that must come from L2, not HBM).
+    GroupNorm: one read for the statistics, one read and one write to
+               normalise: 3 S bytes.
+    conv:      2 * k * C^2 flops per token (a C x kC contraction); bytes
+               2 S + weights.
+    """
+    S = w.P * w.F * w.C * w.elem_bytes
+    return {
+        "dual_attn": {"bytes": 4 * S},
+        "temporal_conv": {"flops": 2 * w.k * w.C * w.C * w.tokens,
+                          "bytes": 2 * S + w.C * w.C * w.k * w.elem_bytes},
+        "groupnorm_global": {"bytes": 3 * S},
+    }
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def __init__(self, index: int, period_s: float = 0.02):
+        self.index, self.period = index, period_s
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        self.ok = False
+
+    def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            return self
+        self._thread = threading.Thread(target=self._run, daemon=True)
+        self._thread.start()
+        return self
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for b, name in self.REASONS.items():
+                    if bits & b and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread:
+            self._thread.join(timeout=1.0)
+        return False
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unsampled"],
+                    "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# inputs
+
+
+def host_inputs(w, pinned: bool):
+    """Seeded synthetic inputs of workload w as torch CPU tensors (bf16 or fp32)."""
+    import torch
+
+    import synth
+    out = {}
+    for name in ("q", "k", "v", "conv_x", "conv_w", "conv_b", "gn_x", "gn_gamma", "gn_beta"):
+        a = synth.make(w, name)
+        t = torch.from_numpy(a)
+        if w.dtype == "bf16":
+            t = t.view(torch.bfloat16)
+        out[name] = t.pin_memory() if pinned else t
+    return out
+
+
+# ---------------------------------------------------------------------------
+# our arm
+
+
+def run_ours(args):
+    import torch
+
+    import clip_temporal_modules_b200 as vi
+    import synth
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    init_dist("nccl")
+    w = synth.BY_NAME[args.workload]
+    stream = torch.cuda.current_stream()
+
+    host = host_inputs(w, pinned=True)
+    d = {k: v.to(dev, non_blocking=True) for k, v in host.items()}
+    out = torch.empty_like(d["q"])
+    y = torch.empty_like(d["conv_x"])
+    z = torch.empty_like(d["gn_x"])
+    torch.cuda.synchronize()
+
+    names = ("dual_attn", "temporal_conv", "groupnorm_global")
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        vi.dual_attn(d["q"], d["k"], d["v"], out, N=w.N, heads=w.heads, n_pre=w.n_pre,
+                     n_post=w.n_post, n_global=w.n_global)
+        if ev is not None:
+            ev[1].record(stream)
+        vi.temporal_conv(d["conv_x"], d["conv_w"], d["conv_b"], y, N=w.N)
+        if ev is not None:
+            ev[2].record(stream)
+        vi.groupnorm_global(d["gn_x"], d["gn_gamma"], d["gn_beta"], z, N=w.N, groups=w.groups,
+                            eps=w.eps)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    vi.take_device_errors()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(dev)
+    torch.cuda.synchronize()
+    launches0 = vi.launch_count()
+    with ClockSampler(dev.index) as clocks:
+        t0.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        t1.record(stream)
+        torch.cuda.synchronize()
+    launches = vi.launch_count() - launches0
+    barrier(dev)
+    elapsed_ms = t0.elapsed_time(t1)
+    elapsed_ms = max_over_ranks(elapsed_ms, dev)
+    vi.take_device_errors()
+
+    per_kernel = {n: statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs)
+                  for j, n in enumerate(names)}
+    ms_per_step = elapsed_ms / args.steps
+    tokens = w.tokens * world * args.steps
+    value = tokens / (elapsed_ms / 1e3)
+
+    peaks, peak_src = load_peaks()
+    work = kernel_work(w)
+    long_step = True     # kernels are timed inside a multi-kernel step
+    tensor_peak = peaks.get("bf16_tflops_sustained" if long_step else "bf16_tflops")
+    kernels = {}
+    for n in names:
+        ms = per_kernel[n]
+        if "flops" in work[n]:
+            ach = work[n]["flops"] / (ms / 1e3) / 1e12
+            kernels[n] = {"ms": round(ms, 4), "achieved": round(ach, 1), "unit": "TFLOP/s",
+                          "frac": round(ach / tensor_peak, 4), "bound": "tensor",
+                          "tokens_per_s": w.tokens / (ms / 1e3)}
+        else:
+            ach = work[n]["bytes"] / (ms / 1e3) / 1e9
+            kernels[n] = {"ms": round(ms, 4), "achieved": round(ach, 1), "unit": "GB/s",
+                          "frac": round(ach / peaks["hbm_gbs"], 4), "bound": "hbm",
+                          "tokens_per_s": w.tokens / (ms / 1e3)}
+    dom = max(names, key=lambda n: per_kernel[n])
+    kd = kernels[dom]
+    traffic = load_traffic(dom, w)
+    roofline = {"kernel": dom, "bound": kd["bound"], "achieved": kd["achieved"],
+                "peak": tensor_peak if kd["bound"] == "tensor" else peaks["hbm_gbs"],
+                "unit": kd["unit"], "frac": kd["frac"], "traffic": traffic,
+                "peak_source": f"{peak_src} ({'bf16_tflops_sustained' if kd['bound'] == 'tensor' else 'hbm_gbs'})"}
+
+    result = {
+        "metric": "temporal-module tokens/s (F*H'W') at F=1024",
+        "value": round(value, 1),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": w.dtype,
+        "data": "synthetic (seeded SplitMix64 + Box-Muller, N(0,1) q/k/v/x, BASELINE distributions)",
+        "config": {"workload": w.name, "F": w.F, "N_clips": w.N, "P": w.P, "C": w.C,
+                   "heads": w.heads, "d": w.d, "n_pre": w.n_pre, "n_post": w.n_post,
+                   "n_global": w.n_global, "k": w.k, "groups": w.groups,
+                   "tokens_per_step_per_gpu": w.tokens,
+                   "parallelism": f"replica x{world} (one video per GPU)",
+                   "l2": "no flush: every tensor (%.2f GB) exceeds L2" % (w.act_bytes / 1e9)},
+        "kernels": kernels,
+        "roofline": roofline,
+        "gpu_launches": int(launches),
+        "clocks": clocks.summary(),
+    }
+
+    if not args.no_e2e:
+        result["e2e"] = run_e2e(args, w, host, dev, stream)
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    cleanup()
+
+
+def run_e2e(args, w, host, dev, stream):
+    """Same step through host buffers: H2D of every input, 3 kernels, D2H of every output."""
+    import torch
+
+    import clip_temporal_modules_b200 as vi
+    world, _, _ = dist_env()
+    res = {k: torch.empty_like(host["q"]).pin_memory() for k in ("out", "y", "z")}
+    d = {}
+
+    def e2e_step():
+        for k_, v_ in host.items():
+            d[k_] = v_.to(dev, non_blocking=True)
+        o = vi.dual_attn(d["q"], d["k"], d["v"], N=w.N, heads=w.heads, n_pre=w.n_pre,
+                         n_post=w.n_post, n_global=w.n_global)
+        yy = vi.temporal_conv(d["conv_x"], d["conv_w"], d["conv_b"], N=w.N)
+        zz = vi.groupnorm_global(d["gn_x"], d["gn_gamma"], d["gn_beta"], N=w.N, groups=w.groups,
+                                 eps=w.eps)
+        res["out"].copy_(o, non_blocking=True)
+        res["y"].copy_(yy, non_blocking=True)
+        res["z"].copy_(zz, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier(dev)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(a.elapsed_time(b), dev)
+    barrier(dev)
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = sum(t.numel() * t.element_size() for t in res.values())
+    return {"value": round(w.tokens * world * args.e2e_steps / (ms / 1e3), 1), "unit": "tokens/s",
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "steps": args.e2e_steps, "ms_per_step": round(ms / args.e2e_steps, 3),
+            "path": "pinned host -> cudaMemcpyAsync -> libvi C ABI x3 -> pinned host"}
+
+
+def load_traffic(kernel, w):
+    """DRAM bytes per launch from the committed ncu summary of this kernel, if current."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as fh:
+        d = json.load(fh)
+    e = d.get(kernel, {}).get(w.name)
+    return None if e is None else e.get("bytes_per_launch")
+
+
+# ---------------------------------------------------------------------------
+# the oracle on the host cores
+
+
+def oracle_sample(w, positions: int):
+    """One bounded sample of the workload: `positions` whole positions (all F frames,
+    all C channels) through the three modules of the oracle.  GroupNorm takes its
+    statistics over the sample (the same work per token as over the full tensor)."""
+    import synth
+    sub = w.with_(P=positions)
+    return {name: synth.make(sub, name) for name in
+            ("q", "k", "v", "conv_x", "conv_w", "conv_b", "gn_x", "gn_gamma", "gn_beta")}, sub
+
+
+def oracle_step(inp, sub):
+    import oracle
+    oracle.dual_attn(inp["q"], inp["k"], inp["v"], sub.F, sub.N, sub.heads, sub.d, sub.n_pre,
+                     sub.n_post, sub.n_global)
+    oracle.temporal_conv(inp["conv_x"], inp["conv_w"], inp["conv_b"], sub.F, sub.N, sub.k)
+    oracle.groupnorm_global(inp["gn_x"], inp["gn_gamma"], inp["gn_beta"], sub.F, sub.N,
+                            sub.groups, sub.eps)
+
+
+def calibrate_positions(w, seconds: float) -> int:
+    inp, sub = oracle_sample(w, 1)
+    t = time.perf_counter()
+    oracle_step(inp, sub)
+    per_pos = max(time.perf_counter() - t, 1e-3)
+    return max(1, min(w.P, int(seconds / per_pos)))
+
+
+def cpu_baseline(w, seconds: float):
+    import oracle
+    npos = calibrate_positions(w, seconds)
+    inp, sub = oracle_sample(w, npos)
+    t = time.perf_counter()
+    oracle_step(inp, sub)
+    dt = time.perf_counter() - t
+    return {"value": round(sub.tokens / dt, 1), "unit": "tokens/s", "cores": oracle.max_threads(),
+            "kind": "oracle", "seconds": round(dt, 2),
+            "sample": f"{npos} of {w.P} positions x all {w.F} frames x {w.C} channels of "
+                      f"{w.name}, all three modules (GroupNorm statistics over the sample)"}
+
+
+def run_reference(args):
+    """The oracle, as it stands, on the host cores: each step is a bounded sample."""
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    import oracle
+    import synth
+    w = synth.BY_NAME[args.workload]
+    budget = 120.0 / max(1, args.steps + args.warmup)        # whole run in ~2 minutes
+    npos = calibrate_positions(w, min(budget, args.cpu_seconds))
+    inp, sub = oracle_sample(w, npos)
+    for _ in range(args.warmup):
+        oracle_step(inp, sub)
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(inp, sub)
+    dt = time.perf_counter() - t
+    value = sub.tokens * args.steps / dt
+    cpu = {"value": round(value, 1), "unit": "tokens/s", "cores": oracle.max_threads(),
+           "kind": "oracle",
+           "sample": f"{npos} of {w.P} positions x all {w.F} frames x {w.C} channels of {w.name}"}
+    print(json.dumps({
+        "impl": "reference", "metric": "temporal-module tokens/s (F*H'W') at F=1024",
+        "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded)", "config": {"workload": w.name, "sample_positions": npos},
+        "cpu_baseline": cpu,
+        "e2e": {"value": round(value, 1), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def cleanup():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.destroy_process_group()
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

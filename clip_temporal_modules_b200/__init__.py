@@ -12,8 +12,8 @@ kernel grid:
 
 Python here only marshals arguments; see _binding.py.
 """
-from ._binding import (LIB_PATH, ViError, dual_attn, groupnorm_global, lib,  # noqa: F401
-                       take_device_errors, temporal_conv)
+from ._binding import (LIB_PATH, ViError, dual_attn, groupnorm_global,  # noqa: F401
+                       launch_count, lib, take_device_errors, temporal_conv)
 
-__all__ = ["dual_attn", "temporal_conv", "groupnorm_global", "take_device_errors", "lib",
+__all__ = ["dual_attn", "temporal_conv", "groupnorm_global", "take_device_errors", "launch_count", "lib",
            "ViError", "LIB_PATH"]

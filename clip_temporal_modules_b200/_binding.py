@@ -52,6 +52,8 @@ def lib() -> ctypes.CDLL:
             fn = getattr(L, name)
             fn.argtypes = args
             fn.restype = ctypes.c_int
+        L.vi_launch_count.argtypes = []
+        L.vi_launch_count.restype = ctypes.c_ulonglong
         L.vi_status_string.argtypes = [ctypes.c_int]
         L.vi_status_string.restype = ctypes.c_char_p
         _lib = L
@@ -128,6 +130,11 @@ def groupnorm_global(x, gamma, beta, out=None, *, N: int, groups: int, eps: floa
                                       out.data_ptr(), F, N, P, C, groups, float(eps),
                                       _stream_ptr(stream)))
     return out
+
+
+def launch_count() -> int:
+    """Kernels libvi has launched in this process so far."""
+    return int(lib().vi_launch_count())
 
 
 def take_device_errors() -> None:

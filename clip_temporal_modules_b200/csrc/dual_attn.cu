@@ -116,7 +116,7 @@ int dual_attn_generic_launch(const T* q, const T* k, const T* v, T* out, int F, 
                                                                   n_pre, n_post, n_global, scale);
   else
     return VI_ERR_UNSUPPORTED;
-  VI_CUDA_TRY(cudaGetLastError());
+  VI_LAUNCHED();
   return VI_OK;
 }
 
@@ -330,7 +330,7 @@ int dual_attn_bf16_fast(const bf16* q, const bf16* k, const bf16* v, bf16* out, 
   if (!err) return VI_ERR_CUDA;
   dual_attn_bf16_mma<<<(unsigned)grid, 256, FA_SMEM_BYTES, stream>>>(
       maps, F, N, heads, nblk, n_pre, n_post, n_global, scale_log2, err);
-  VI_CUDA_TRY(cudaGetLastError());
+  VI_LAUNCHED();
   return VI_OK;
 }
 

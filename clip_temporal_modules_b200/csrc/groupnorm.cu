@@ -16,22 +16,23 @@
 //   last block (atomic ticket) merges them in fp64:
 //     mu_g = K_g + S1/n,  var_g = S2/n - (S1/n)^2,
 //   which is algebraically the pages' "global mean, then spread about it", and
-//   turns them into per-channel coefficients a_c = gamma_c / sqrt(var_g+eps),
-//   b_c = beta_c - mu_g a_c.
-// Pass 2 (gn_apply_*): one read of x and one write of y = x a_c + b_c.
+//   turns them into per-channel coefficients m_c = mu_g (rounded to fp32),
+//   a_c = gamma_c / sqrt(var_g+eps) and beta_c.
+// Pass 2 (gn_apply_*): one read of x and one write of y = (x - m_c) a_c + beta_c
+//   (subtracting first keeps a constant group exactly at beta).
 // HBM traffic: 3 x |x|, the minimum for a two-pass normalisation of a tensor
 // far larger than L2.
+#include "ptx.cuh"
 #include "vi_internal.cuh"
 
 namespace vi {
 
-constexpr int GN_THREADS_TARGET = 320;
 constexpr int GN_MAX_GROUPS = 1024;
 constexpr int GN_FOLD = 32;            // fp32 run length before folding into fp64
 
 struct GnScratch {
   double* partials;        // [nparts][groups][3]: n, S1, S2
-  float* coef;             // [C][2]: a_c, b_c
+  float* coef;             // [C][4]: m_c, a_c, beta_c, 0
   unsigned int* ticket;    // blocks finished (reset to 0 by the last block)
   double* stats;           // [groups][2]: mu_g, var_g (kept for inspection)
 };
@@ -70,8 +71,10 @@ __device__ void gn_finalize(const GnScratch& s, int nparts, int groups, int C, i
     const double var = fmax(red[g][2] / nn - m1 * m1, 0.0);
     const double mu = (double)to_f32(x[(size_t)g * cg]) + m1;
     const double a = (double)to_f32(gamma[c]) / sqrt(var + (double)eps);
-    s.coef[2 * c] = (float)a;
-    s.coef[2 * c + 1] = (float)((double)to_f32(beta[c]) - mu * a);
+    s.coef[4 * c] = (float)mu;
+    s.coef[4 * c + 1] = (float)a;
+    s.coef[4 * c + 2] = to_f32(beta[c]);
+    s.coef[4 * c + 3] = 0.f;
     if (c == g * cg) {
       s.stats[2 * g] = mu;
       s.stats[2 * g + 1] = var;
@@ -98,74 +101,117 @@ __device__ __forceinline__ void gn_block_done(const GnScratch& s, int nblocks, i
   }
 }
 
-// Vector path: blockDim = VPR * RB threads; thread (rr, j) owns channel vector
-// j (channels [j*V, j*V+V)) of rows rr, rr+RB, ... of its block's share.  The
-// vector spans at most two groups (checked on the host).
+// Vector path.  Persistent, one CTA per SM.  The tensor is cut into chunks of
+// R_c whole rows (<= 32 KB); a producer warp streams chunks into a ring of
+// GN_STAGES shared-memory stages with 1-D TMA bulk copies (up to 192 KB in
+// flight per SM), and VPR x RB consumer threads read them back as 16-byte
+// vectors.  Consumer thread (rr, j) always owns channel vector j (channels
+// [jV, jV+V)) of rows rr, rr+RB, ... of a chunk, so it only ever touches the
+// one or two groups that vector spans (checked on the host).
+constexpr int GN_STAGES = 6;
+constexpr int GN_CHUNK_MAX = 32768;
+
+struct GnRing {
+  int64_t rows;        // P * F
+  int C;               // channels
+  int rowbytes;        // C * sizeof(T)
+  int rc;              // rows per chunk
+  int64_t nchunks;
+  int stage_bytes;     // rc * rowbytes (16B multiple)
+  int VPR, RB;         // consumer layout
+};
+
+__device__ __forceinline__ uint32_t ring_stage(uint32_t base, const GnRing& g, int s) {
+  return base + (uint32_t)s * g.stage_bytes;
+}
+
 template <typename T>
-__global__ void __launch_bounds__(1024) gn_stats_vec(const T* __restrict__ x, int64_t rows, int C,
-                                                     int cg, int groups, int RB, GnScratch s,
-                                                     const T* __restrict__ gamma,
-                                                     const T* __restrict__ beta, float eps) {
+__global__ void __launch_bounds__(1024, 1) gn_stats_ring(const T* __restrict__ x, GnRing rg,
+                                                         int cg, int groups, GnScratch s,
+                                                         const T* __restrict__ gamma,
+                                                         const T* __restrict__ beta, float eps,
+                                                         unsigned int* err_word) {
   constexpr int V = VecOf<T>::n;
+  extern __shared__ __align__(128) uint8_t smem[];
   __shared__ double acc[GN_MAX_GROUPS][3];
-  const int VPR = C / V;
+  const uint32_t base = smem_u32(smem);
+  const uint32_t bars = base + GN_STAGES * rg.stage_bytes;     // full[S], empty[S]
+  const int ncw = (blockDim.x >> 5) - 1;                        // consumer warps
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int g = threadIdx.x; g < groups; g += blockDim.x) acc[g][0] = acc[g][1] = acc[g][2] = 0.0;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < GN_STAGES; ++i) {
+      mbar_init(bars + 8 * i, 1);
+      mbar_init(bars + 8 * (GN_STAGES + i), ncw);
+    }
+    fence_barrier_init();
+  }
   __syncthreads();
 
-  const int j = threadIdx.x % VPR, rr = threadIdx.x / VPR;
-  if (rr < RB) {
+  if (warp == ncw) {                                            // producer warp
+    if (lane == 0) {
+      int kl = 0;
+      for (int64_t c = blockIdx.x; c < rg.nchunks; c += gridDim.x, ++kl) {
+        const int st = kl % GN_STAGES, use = kl / GN_STAGES;
+        if (use > 0 && !mbar_wait_bounded(bars + 8 * (GN_STAGES + st), (use - 1) & 1, err_word,
+                                          VI_DEV_ERR_TMA_TIMEOUT))
+          break;
+        const int64_t r0 = c * rg.rc;
+        const int nr = (int)min((int64_t)rg.rc, rg.rows - r0);
+        const uint32_t bytes = (uint32_t)nr * rg.rowbytes;
+        mbar_arrive_expect_tx(bars + 8 * st, bytes);
+        bulk_load(ring_stage(base, rg, st), x + r0 * rg.C, bytes, bars + 8 * st);
+      }
+    }
+  } else {
+    const int t = threadIdx.x;
+    const bool active = t < rg.VPR * rg.RB;
+    const int j = t % rg.VPR, rr = t / rg.VPR;
     const int c0 = j * V;
     const int glo = c0 / cg;
     const int split = min(V, (glo + 1) * cg - c0);      // elements [0, split) are in glo
     const bool has_hi = split < V;
-    const float klo = to_f32(x[(size_t)glo * cg]);
-    const float khi = has_hi ? to_f32(x[(size_t)(glo + 1) * cg]) : 0.f;
+    const float klo = active ? to_f32(x[(size_t)glo * cg]) : 0.f;
+    const float khi = active && has_hi ? to_f32(x[(size_t)(glo + 1) * cg]) : 0.f;
     double d1lo = 0, d2lo = 0, d1hi = 0, d2hi = 0;
     int64_t nrows = 0;
-    const int64_t step = (int64_t)gridDim.x * RB;
-    int64_t r = (int64_t)blockIdx.x * RB + rr;
-    while (r < rows) {
-      float a1lo = 0.f, a2lo = 0.f, a1hi = 0.f, a2hi = 0.f;
-      // A run of up to GN_FOLD rows, 4 loads in flight per thread.
-      for (int it = 0; it < GN_FOLD && r < rows; it += 4) {
-        uint4 u[4];
-        int cnt = 0;
+    int kl = 0;
+    for (int64_t c = blockIdx.x; c < rg.nchunks; c += gridDim.x, ++kl) {
+      const int st = kl % GN_STAGES, use = kl / GN_STAGES;
+      if (!mbar_wait_bounded(bars + 8 * st, use & 1, err_word, VI_DEV_ERR_TMA_TIMEOUT)) break;
+      const int nr = (int)min((int64_t)rg.rc, rg.rows - c * rg.rc);
+      if (active) {
+        float a1lo = 0.f, a2lo = 0.f, a1hi = 0.f, a2hi = 0.f;
+        const uint32_t p0 = ring_stage(base, rg, st) + j * 16;
+        for (int r = rr; r < nr; r += rg.RB) {
+          float f[V];
+          unpack(lds128(p0 + r * rg.rowbytes), f);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          if (r + q * step < rows) {
-            u[q] = *reinterpret_cast<const uint4*>(x + (r + q * step) * C + c0);
-            ++cnt;
-          }
-        }
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          if (q < cnt) {
-            float f[V];
-            unpack(u[q], f);
-#pragma unroll
-            for (int e = 0; e < V; ++e) {
-              if (e < split) {
-                const float dv = f[e] - klo;
-                a1lo += dv; a2lo = fmaf(dv, dv, a2lo);
-              } else {
-                const float dv = f[e] - khi;
-                a1hi += dv; a2hi = fmaf(dv, dv, a2hi);
-              }
+          for (int e = 0; e < V; ++e) {
+            if (e < split) {
+              const float dv = f[e] - klo;
+              a1lo += dv; a2lo = fmaf(dv, dv, a2lo);
+            } else {
+              const float dv = f[e] - khi;
+              a1hi += dv; a2hi = fmaf(dv, dv, a2hi);
             }
           }
+          ++nrows;
         }
-        nrows += cnt;
-        r += (int64_t)cnt * step;
+        d1lo += a1lo; d2lo += a2lo; d1hi += a1hi; d2hi += a2hi;
       }
-      d1lo += a1lo; d2lo += a2lo; d1hi += a1hi; d2hi += a2hi;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bars + 8 * (GN_STAGES + st));
     }
-    atomicAdd(&acc[glo][0], (double)(nrows * split));
-    atomicAdd(&acc[glo][1], d1lo);
-    atomicAdd(&acc[glo][2], d2lo);
-    if (has_hi) {
-      atomicAdd(&acc[glo + 1][0], (double)(nrows * (V - split)));
-      atomicAdd(&acc[glo + 1][1], d1hi);
-      atomicAdd(&acc[glo + 1][2], d2hi);
+    if (active) {
+      atomicAdd(&acc[glo][0], (double)(nrows * split));
+      atomicAdd(&acc[glo][1], d1lo);
+      atomicAdd(&acc[glo][2], d2lo);
+      if (has_hi) {
+        atomicAdd(&acc[glo + 1][0], (double)(nrows * (V - split)));
+        atomicAdd(&acc[glo + 1][1], d1hi);
+        atomicAdd(&acc[glo + 1][2], d2hi);
+      }
     }
   }
   __syncthreads();
@@ -174,41 +220,97 @@ __global__ void __launch_bounds__(1024) gn_stats_vec(const T* __restrict__ x, in
     p[0] = acc[g][0]; p[1] = acc[g][1]; p[2] = acc[g][2];
   }
   __syncthreads();
-  gn_block_done<T>(s, gridDim.x, gridDim.x, groups, C, cg, x, gamma, beta, eps, acc);
+  gn_block_done<T>(s, gridDim.x, gridDim.x, groups, rg.C, cg, x, gamma, beta, eps, acc);
 }
 
+// y = (x - m_c) a_c + beta_c through the same ring: consumers rewrite each
+// stage in place and the producer bulk-stores it back before reusing it.
+// Chunks are visited last-first: the end of x, read last by the statistics
+// pass, is the part most likely to still sit in L2.
 template <typename T>
-__global__ void __launch_bounds__(1024) gn_apply_vec(const T* __restrict__ x, T* __restrict__ y,
-                                                     int64_t rows, int C, int RB,
-                                                     const float* __restrict__ coef) {
+__global__ void __launch_bounds__(1024, 1) gn_apply_ring(const T* __restrict__ x,
+                                                         T* __restrict__ y, GnRing rg,
+                                                         const float* __restrict__ coef,
+                                                         unsigned int* err_word) {
   constexpr int V = VecOf<T>::n;
-  const int VPR = C / V;
-  const int j = threadIdx.x % VPR, rr = threadIdx.x / VPR;
-  if (rr >= RB) return;
-  const int c0 = j * V;
-  float a[V], b[V];
-#pragma unroll
-  for (int e = 0; e < V; ++e) {
-    a[e] = coef[2 * (c0 + e)];
-    b[e] = coef[2 * (c0 + e) + 1];
+  extern __shared__ __align__(128) uint8_t smem[];
+  const uint32_t base = smem_u32(smem);
+  const uint32_t bars = base + GN_STAGES * rg.stage_bytes;     // full[S], done[S]
+  const int ncw = (blockDim.x >> 5) - 1;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < GN_STAGES; ++i) {
+      mbar_init(bars + 8 * i, 1);
+      mbar_init(bars + 8 * (GN_STAGES + i), ncw);
+    }
+    fence_barrier_init();
   }
-  // Rows are visited last-first: the end of x, read last by the statistics
-  // pass, is the part most likely to still sit in L2.
-  const int64_t step = (int64_t)gridDim.x * RB;
-  for (int64_t r = (int64_t)blockIdx.x * RB + rr; r < rows; r += 4 * step) {
-    uint4 u[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-      if (r + q * step < rows) u[q] = ld_stream(x + (rows - 1 - (r + q * step)) * C + c0);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      if (r + q * step < rows) {
-        float f[V];
-        unpack(u[q], f);
-#pragma unroll
-        for (int e = 0; e < V; ++e) f[e] = fmaf(f[e], a[e], b[e]);
-        st_stream(y + (rows - 1 - (r + q * step)) * C + c0, pack(f));
+  __syncthreads();
+  auto chunk_of = [&](int kl) { return rg.nchunks - 1 - (blockIdx.x + (int64_t)kl * gridDim.x); };
+
+  if (warp == ncw) {
+    if (lane == 0) {
+      const int nloc = (int)((rg.nchunks - blockIdx.x + gridDim.x - 1) / gridDim.x);
+      bool ok = true;
+      auto store_back = [&](int kl) {        // stage of local chunk kl -> y
+        const int st = kl % GN_STAGES;
+        if (!mbar_wait_bounded(bars + 8 * (GN_STAGES + st), (kl / GN_STAGES) & 1, err_word,
+                               VI_DEV_ERR_TMA_TIMEOUT))
+          return false;
+        const int64_t r0 = chunk_of(kl) * rg.rc;
+        const int nr = (int)min((int64_t)rg.rc, rg.rows - r0);
+        bulk_store(y + r0 * rg.C, ring_stage(base, rg, st), (uint32_t)nr * rg.rowbytes);
+        bulk_commit();
+        return true;
+      };
+      for (int kl = 0; kl < nloc && ok; ++kl) {
+        const int st = kl % GN_STAGES;
+        if (kl >= GN_STAGES) {
+          ok = store_back(kl - GN_STAGES);
+          bulk_wait_read_all();
+          if (!ok) break;
+        }
+        const int64_t r0 = chunk_of(kl) * rg.rc;
+        const int nr = (int)min((int64_t)rg.rc, rg.rows - r0);
+        const uint32_t bytes = (uint32_t)nr * rg.rowbytes;
+        mbar_arrive_expect_tx(bars + 8 * st, bytes);
+        bulk_load(ring_stage(base, rg, st), x + r0 * rg.C, bytes, bars + 8 * st);
       }
+      for (int kl = max(0, nloc - GN_STAGES); kl < nloc && ok; ++kl) ok = store_back(kl);
+      bulk_wait_all();
+    }
+  } else {
+    const int t = threadIdx.x;
+    const bool active = t < rg.VPR * rg.RB;
+    const int j = t % rg.VPR, rr = t / rg.VPR;
+    const int c0 = j * V;
+    float m[V], a[V], b[V];
+#pragma unroll
+    for (int e = 0; e < V; ++e) {
+      m[e] = active ? coef[4 * (c0 + e)] : 0.f;
+      a[e] = active ? coef[4 * (c0 + e) + 1] : 0.f;
+      b[e] = active ? coef[4 * (c0 + e) + 2] : 0.f;
+    }
+    int kl = 0;
+    for (int64_t c = blockIdx.x; c < rg.nchunks; c += gridDim.x, ++kl) {
+      const int st = kl % GN_STAGES;
+      if (!mbar_wait_bounded(bars + 8 * st, (kl / GN_STAGES) & 1, err_word,
+                             VI_DEV_ERR_TMA_TIMEOUT))
+        break;
+      const int nr = (int)min((int64_t)rg.rc, rg.rows - chunk_of(kl) * rg.rc);
+      if (active) {
+        const uint32_t p0 = ring_stage(base, rg, st) + j * 16;
+        for (int r = rr; r < nr; r += rg.RB) {
+          float f[V];
+          unpack(lds128(p0 + r * rg.rowbytes), f);
+#pragma unroll
+          for (int e = 0; e < V; ++e) f[e] = fmaf(f[e] - m[e], a[e], b[e]);
+          sts128(p0 + r * rg.rowbytes, pack(f));
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bars + 8 * (GN_STAGES + st));
     }
   }
 }
@@ -261,7 +363,7 @@ __global__ void __launch_bounds__(256) gn_apply_scalar(const T* __restrict__ x, 
   for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n;
        e += (int64_t)gridDim.x * blockDim.x) {
     const int c = (int)(e % C);
-    y[e] = from_f32<T>(fmaf(to_f32(x[e]), coef[2 * c], coef[2 * c + 1]));
+    y[e] = from_f32<T>(fmaf(to_f32(x[e]) - coef[4 * c], coef[4 * c + 1], coef[4 * c + 2]));
   }
 }
 
@@ -269,11 +371,12 @@ __global__ void __launch_bounds__(256) gn_apply_scalar(const T* __restrict__ x, 
 // Host side.
 
 struct GnPlan {
-  bool vec;
-  int RB, threads, blocks;     // vector path
+  bool ring;
+  GnRing rg;
+  int threads, blocks;         // ring path
+  size_t smem;                 // ring path dynamic shared memory
   int parts;                   // scalar path: row slices per group
   int nparts;                  // partial records per group
-  size_t scratch_bytes;
 };
 
 template <typename T>
@@ -282,20 +385,26 @@ static GnPlan gn_plan(int64_t rows, int C, int groups) {
   GnPlan pl{};
   const int cg = C / groups;
   const int VPR = C / V;
-  bool span_ok = VPR <= 1024;
-  for (int c0 = 0; span_ok && c0 < C; c0 += V)
-    if ((c0 + V - 1) / cg - c0 / cg > 1) span_ok = false;
-  pl.vec = span_ok;
-  if (pl.vec) {
-    pl.RB = GN_THREADS_TARGET / VPR > 0 ? GN_THREADS_TARGET / VPR : 1;
-    pl.threads = VPR * pl.RB;
-    int per_sm = 0;
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gn_stats_vec<T>, pl.threads, 0);
-    if (per_sm < 1) per_sm = 1;
-    const int64_t want = (rows + pl.RB - 1) / pl.RB;
-    int64_t blocks = (int64_t)sm_count() * per_sm;
-    if (blocks > want) blocks = want;
-    pl.blocks = (int)(blocks > 0 ? blocks : 1);
+  const int rowbytes = C * (int)sizeof(T);
+  bool ok = VPR <= 512 && rowbytes <= GN_CHUNK_MAX;
+  for (int c0 = 0; ok && c0 < C; c0 += V)
+    if ((c0 + V - 1) / cg - c0 / cg > 1) ok = false;
+  pl.ring = ok;
+  if (pl.ring) {
+    GnRing& g = pl.rg;
+    g.rows = rows;
+    g.C = C;
+    g.rowbytes = rowbytes;
+    g.VPR = VPR;
+    g.RB = 256 / VPR > 0 ? 256 / VPR : 1;
+    g.rc = GN_CHUNK_MAX / rowbytes;
+    g.stage_bytes = g.rc * rowbytes;
+    g.nchunks = (rows + g.rc - 1) / g.rc;
+    pl.threads = ((VPR * g.RB + 31) / 32) * 32 + 32;
+    pl.smem = (size_t)GN_STAGES * g.stage_bytes + 16 * GN_STAGES;
+    int64_t blocks = sm_count();
+    if (blocks > g.nchunks) blocks = g.nchunks;
+    pl.blocks = (int)blocks;
     pl.nparts = pl.blocks;
   } else {
     const int64_t per_group = (int64_t)(sm_count()) * 8 / groups + 1;
@@ -304,12 +413,10 @@ static GnPlan gn_plan(int64_t rows, int C, int groups) {
     if (pl.parts < 1) pl.parts = 1;
     pl.nparts = pl.parts;
   }
-  pl.scratch_bytes = 256 + sizeof(double) * 3 * (size_t)groups * pl.nparts +
-                     sizeof(float) * 2 * (size_t)C + sizeof(double) * 2 * (size_t)groups;
   return pl;
 }
 
-// Carve the scratch block: ticket | stats | coef | partials (each 16B aligned).
+// Carve the scratch block: ticket | stats | coef | partials (each 64B aligned).
 static GnScratch gn_carve(void* base, int groups, int C) {
   GnScratch s;
   char* p = static_cast<char*>(base);
@@ -318,7 +425,7 @@ static GnScratch gn_carve(void* base, int groups, int C) {
   s.stats = reinterpret_cast<double*>(p);
   p += ((sizeof(double) * 2 * groups + 63) / 64) * 64;
   s.coef = reinterpret_cast<float*>(p);
-  p += ((sizeof(float) * 2 * (size_t)C + 63) / 64) * 64;
+  p += ((sizeof(float) * 4 * (size_t)C + 63) / 64) * 64;
   s.partials = reinterpret_cast<double*>(p);
   return s;
 }
@@ -327,38 +434,38 @@ template <typename T>
 static size_t gn_scratch_bytes(int64_t rows, int C, int groups) {
   const GnPlan pl = gn_plan<T>(rows, C, groups);
   return 64 + ((sizeof(double) * 2 * groups + 63) / 64) * 64 +
-         ((sizeof(float) * 2 * (size_t)C + 63) / 64) * 64 +
+         ((sizeof(float) * 4 * (size_t)C + 63) / 64) * 64 +
          sizeof(double) * 3 * (size_t)groups * pl.nparts;
 }
 
-// Enqueue both passes using caller-provided scratch (ticket must read 0).
+// Enqueue both passes using caller-provided scratch (its ticket must read 0).
 template <typename T>
 static int gn_launch(const T* x, const T* gamma, const T* beta, T* y, int64_t rows, int C,
                      int groups, float eps, void* scratch, cudaStream_t stream) {
   const GnPlan pl = gn_plan<T>(rows, C, groups);
   const GnScratch s = gn_carve(scratch, groups, C);
   const int cg = C / groups;
-  if (pl.vec) {
-    gn_stats_vec<T><<<pl.blocks, pl.threads, 0, stream>>>(x, rows, C, cg, groups, pl.RB, s, gamma,
-                                                         beta, eps);
-    VI_CUDA_TRY(cudaGetLastError());
-    int per_sm = 0;
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gn_apply_vec<T>, pl.threads, 0);
-    if (per_sm < 1) per_sm = 1;
-    int64_t blocks = (int64_t)sm_count() * per_sm;
-    const int64_t want = (rows + pl.RB - 1) / pl.RB;
-    if (blocks > want) blocks = want;
-    gn_apply_vec<T><<<(int)blocks, pl.threads, 0, stream>>>(x, y, rows, C, pl.RB, s.coef);
-    VI_CUDA_TRY(cudaGetLastError());
+  if (pl.ring) {
+    unsigned int* err = device_error_word();
+    if (!err) return VI_ERR_CUDA;
+    VI_CUDA_TRY(cudaFuncSetAttribute(gn_stats_ring<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)pl.smem));
+    VI_CUDA_TRY(cudaFuncSetAttribute(gn_apply_ring<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)pl.smem));
+    gn_stats_ring<T><<<pl.blocks, pl.threads, pl.smem, stream>>>(x, pl.rg, cg, groups, s, gamma,
+                                                                 beta, eps, err);
+    VI_LAUNCHED();
+    gn_apply_ring<T><<<pl.blocks, pl.threads, pl.smem, stream>>>(x, y, pl.rg, s.coef, err);
+    VI_LAUNCHED();
   } else {
     gn_stats_scalar<T><<<dim3(groups, pl.parts), 256, 0, stream>>>(x, rows, C, cg, groups, s,
                                                                   gamma, beta, eps);
-    VI_CUDA_TRY(cudaGetLastError());
+    VI_LAUNCHED();
     const int64_t n = rows * C;
     int64_t blocks = (n + 255) / 256;
     if (blocks > (int64_t)sm_count() * 16) blocks = (int64_t)sm_count() * 16;
     gn_apply_scalar<T><<<(int)blocks, 256, 0, stream>>>(x, y, n, C, s.coef);
-    VI_CUDA_TRY(cudaGetLastError());
+    VI_LAUNCHED();
   }
   return VI_OK;
 }

@@ -85,7 +85,7 @@ int temporal_conv_generic_launch(const T* x, const T* w, const T* b, T* y, int F
       (int64_t)P * ((F + CG_TF - 1) / CG_TF) * ((C + CG_TCO - 1) / CG_TCO);
   if (blocks > 0x7fffffff) return VI_ERR_UNSUPPORTED;
   temporal_conv_generic<T><<<(unsigned)blocks, 256, 0, stream>>>(x, w, b, y, F, P, C, k);
-  VI_CUDA_TRY(cudaGetLastError());
+  VI_LAUNCHED();
   return VI_OK;
 }
 

@@ -3,6 +3,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <math.h>
+#include <atomic>
 #include <mutex>
 
 #include "ptx.cuh"
@@ -36,6 +37,9 @@ int temporal_conv_bf16_tc(const bf16*, const bf16*, const bf16*, bf16*, int, int
 bool temporal_conv_tc_ok(int F, int P, int C, int k);
 template <typename T>
 int groupnorm_global(const T*, const T*, const T*, T*, int64_t, int, int, float, cudaStream_t);
+
+static std::atomic<unsigned long long> g_launches{0};
+void note_launch(int n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
 
 int sm_count() {
   static int cached[64] = {0};
@@ -195,6 +199,8 @@ const char* vi_status_string(int status) {
 }
 
 int vi_version(void) { return 100; }
+
+unsigned long long vi_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 int vi_take_device_errors(void) {
   if (!device_error_word()) return VI_ERR_CUDA;

@@ -68,6 +68,17 @@ inline bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
 
 int sm_count();   // multiprocessors of the current device (cached per device)
 
+// Count one kernel launch (backs vi_launch_count).
+void note_launch(int n = 1);
+
+// Check the launch just made and count it.
+#define VI_LAUNCHED()                                          \
+  do {                                                         \
+    cudaError_t _e = cudaGetLastError();                       \
+    if (_e != cudaSuccess) return VI_ERR_CUDA;                 \
+    ::vi::note_launch();                                       \
+  } while (0)
+
 #define VI_CUDA_TRY(expr)                       \
   do {                                          \
     cudaError_t _e = (expr);                    \

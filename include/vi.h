@@ -72,6 +72,13 @@ int vi_version(void);
 int vi_take_device_errors(void);
 
 /*
+ * Number of CUDA kernels this library has launched in the calling process
+ * since it was loaded (all devices and streams; a diagnostic for profiling
+ * and benchmarks, not an ordering primitive).
+ */
+unsigned long long vi_launch_count(void);
+
+/*
  * Dual-domain temporal attention (attention-module paragraph of the source).
  *
  * For every position p, head h and clip i (frames [s, e), s = i*L, e = s+L),
@@ -132,7 +139,7 @@ int vi_temporal_conv_f32(const void* x, const void* w, const void* b, void* y, i
  * x, y : [P][F][C] (y may equal x: in place);  gamma, beta : [C].
  * Requirements : sizes > 0; F % N == 0; C % groups == 0; eps >= 0 and finite.
  *                y may alias x exactly but must not partly overlap it.
- * Scratch      : (24 * groups * blocks + 8*C + 64) bytes of stream-ordered
+ * Scratch      : (24 * groups * blocks + 16*C + 16*groups + 64) bytes of stream-ordered
  *                scratch for per-block partial sums and the per-channel
  *                coefficients, freed on the stream after the last kernel.
  */

@@ -44,6 +44,7 @@ def test_status_strings_and_version(L):
     assert L.vi_status_string(-5) == b"VI_ERR_DEVICE_TIMEOUT"
     assert L.vi_status_string(7) == b"VI_ERR_UNKNOWN"
     assert L.vi_version() >= 100
+    assert vi.launch_count() == 0         # nothing launched without a device
 
 
 A = 1 << 20          # fake 16-byte-aligned "device" addresses, never dereferenced
@@ -116,5 +117,5 @@ def test_groupnorm_rejects(L, kw, expect):
 
 def test_binding_signatures_cover_header():
     for n in declared_functions():
-        if n != "vi_status_string":
+        if n not in ("vi_status_string", "vi_launch_count"):
             assert n in _binding.SIGNATURES, n
