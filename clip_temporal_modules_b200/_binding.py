@@ -27,6 +27,7 @@ SIGNATURES = {
     "vi_temporal_conv_f32": [_vp, _vp, _vp, _vp] + [_i] * 5 + [_vp],
     "vi_groupnorm_global": [_vp, _vp, _vp, _vp] + [_i] * 5 + [_f, _vp],
     "vi_groupnorm_global_f32": [_vp, _vp, _vp, _vp] + [_i] * 5 + [_f, _vp],
+    "vi_groupnorm_global_noalloc": [_vp, _vp, _vp, _vp] + [_i] * 5 + [_f, _vp],
     "vi_version": [],
     "vi_take_device_errors": [],
 }

@@ -22,6 +22,10 @@
 //   (subtracting first keeps a constant group exactly at beta).
 // HBM traffic: 3 x |x|, the minimum for a two-pass normalisation of a tensor
 // far larger than L2.
+#include <math.h>
+
+#include <mutex>
+
 #include "ptx.cuh"
 #include "vi_internal.cuh"
 
@@ -490,3 +494,74 @@ template int groupnorm_global<bf16>(const bf16*, const bf16*, const bf16*, bf16*
                                     int, float, cudaStream_t);
 
 }  // namespace vi
+
+// ---------------------------------------------------------------------------
+// Allocation-free entry point.
+//
+// Some callers cannot allocate device memory while they run: a plugin inside
+// an inference engine that owns all device memory and forbids allocation in
+// its execution step, or a service whose memory footprint is fixed when it
+// starts.  vi_groupnorm_global takes its scratch from cudaMallocAsync, so
+// those callers cannot use it.  vi_groupnorm_global_noalloc runs the same two
+// kernels with its scratch in the file-scope array below instead; the caller
+// still provides every input and output.
+//
+// The array is a module global: every GPU that loads libvi holds it until the
+// process exits, and every call shares it (see include/vi.h).
+
+namespace vi {
+
+constexpr size_t GN_STATIC_SCRATCH_BYTES = size_t(1) << 20;      // 1 MiB
+static __device__ __align__(256) unsigned char g_gn_static_scratch[GN_STATIC_SCRATCH_BYTES];
+
+// Device address of g_gn_static_scratch on the current device.  In host code
+// the array's name is only a host-side stand-in, so the address is looked up
+// once per device, with that device current, and cached.
+static void* gn_static_scratch() {
+  static std::mutex mu;
+  static void* cached[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!cached[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_gn_static_scratch) != cudaSuccess) return nullptr;
+    cached[dev] = p;
+  }
+  return cached[dev];
+}
+
+}  // namespace vi
+
+extern "C" int vi_groupnorm_global_noalloc(const void* x, const void* gamma, const void* beta,
+                                           void* y, int F, int N, int P, int C, int groups,
+                                           float eps, vi_stream_t stream) {
+  using namespace vi;
+  using T = bf16;
+  // The argument checks of vi_groupnorm_global.
+  if (!x || !gamma || !beta || !y) return VI_ERR_INVALID_ARG;
+  if (F <= 0 || N <= 0 || P <= 0 || C <= 0 || F % N != 0) return VI_ERR_INVALID_ARG;
+  if ((double)P * (double)F * (double)C > 1.099511627776e12) return VI_ERR_UNSUPPORTED;
+  if (groups <= 0 || C % groups != 0) return VI_ERR_INVALID_ARG;
+  if (!(eps >= 0.f) || !isfinite(eps)) return VI_ERR_INVALID_ARG;
+  if (groups > GN_MAX_GROUPS) return VI_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(gamma) || !aligned16(beta) || !aligned16(y))
+    return VI_ERR_ALIGNMENT;
+  if ((C * sizeof(T)) % 16 != 0) return VI_ERR_ALIGNMENT;
+  const size_t bytes = (size_t)P * F * C * sizeof(T);
+  if (y != x && overlaps(y, bytes, x, bytes)) return VI_ERR_INVALID_ARG;
+  if (overlaps(y, bytes, gamma, C * sizeof(T)) || overlaps(y, bytes, beta, C * sizeof(T)))
+    return VI_ERR_INVALID_ARG;
+  // Scratch from the static array, never from an allocator.
+  const int64_t rows = (int64_t)P * F;
+  if (gn_scratch_bytes<T>(rows, C, groups) > GN_STATIC_SCRATCH_BYTES) return VI_ERR_UNSUPPORTED;
+  void* scratch = gn_static_scratch();
+  if (!scratch) return VI_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // The array keeps the previous call's contents: the completion ticket must
+  // start at zero (the rest is fully rewritten before it is read).
+  VI_CUDA_TRY(cudaMemsetAsync(scratch, 0, 64, s));
+  return gn_launch<T>(static_cast<const T*>(x), static_cast<const T*>(gamma),
+                      static_cast<const T*>(beta), static_cast<T*>(y), rows, C, groups, eps,
+                      scratch, s);
+}

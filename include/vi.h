@@ -148,6 +148,39 @@ int vi_groupnorm_global(const void* x, const void* gamma, const void* beta, void
 int vi_groupnorm_global_f32(const void* x, const void* gamma, const void* beta, void* y, int F,
                             int N, int P, int C, int groups, float eps, vi_stream_t stream);
 
+/*
+ * GroupNorm with global statistics that allocates nothing (bf16 only).
+ *
+ * The source paper has no counterpart to this entry point.  It is for callers
+ * that cannot allocate device memory while they run -- for example a plugin
+ * inside an inference engine that owns all device memory and forbids
+ * allocation in its execution step, or a service whose memory footprint is
+ * fixed when it starts -- and therefore cannot use vi_groupnorm_global, which
+ * takes its scratch from cudaMallocAsync.  The caller still provides every
+ * input and output.
+ *
+ * Arguments, layout, result and argument checks: as vi_groupnorm_global.
+ * Scratch      : a 1 MiB array inside libvi (a static __device__ array that
+ *                every GPU which loads the library holds until the process
+ *                exits).  A call whose scratch need is larger returns
+ *                VI_ERR_UNSUPPORTED before launching anything.  The need is
+ *                about 64 + 16*groups + 16*C + 24*groups*B bytes, B being the
+ *                number of streaming blocks (at most the SM count); on a
+ *                148-SM B200 that admits, e.g., 32 groups with C up to ~58000
+ *                or 256 groups with C up to ~8000.
+ * First call   : the first call on each device looks up the array's device
+ *                address with that device current (cudaGetSymbolAddress) and
+ *                caches it; make that first call before any stream capture.
+ * Sharing      : every call uses the same array.  Each call clears the part
+ *                that must start at zero and rewrites the rest, but calls
+ *                whose work overlaps on the GPU (different streams, or several
+ *                host threads) race on it and give wrong results: serialise
+ *                them, e.g. on one stream.
+ */
+int vi_groupnorm_global_noalloc(const void* x, const void* gamma, const void* beta, void* y,
+                                int F, int N, int P, int C, int groups, float eps,
+                                vi_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
