@@ -175,8 +175,15 @@ __global__ void __launch_bounds__(1024, 1) gn_stats_ring(const T* __restrict__ x
     const int glo = c0 / cg;
     const int split = min(V, (glo + 1) * cg - c0);      // elements [0, split) are in glo
     const bool has_hi = split < V;
-    const float klo = active ? to_f32(x[(size_t)glo * cg]) : 0.f;
-    const float khi = active && has_hi ? to_f32(x[(size_t)(glo + 1) * cg]) : 0.f;
+    // Per-element shift (the group's first value) and per-element running sums:
+    // V independent dependency chains per thread, no per-element branching.
+    float kk[V];
+    {
+      const float klo = active ? to_f32(x[(size_t)glo * cg]) : 0.f;
+      const float khi = active && has_hi ? to_f32(x[(size_t)(glo + 1) * cg]) : 0.f;
+#pragma unroll
+      for (int e = 0; e < V; ++e) kk[e] = e < split ? klo : khi;
+    }
     double d1lo = 0, d2lo = 0, d1hi = 0, d2hi = 0;
     int64_t nrows = 0;
     int kl = 0;
@@ -185,22 +192,39 @@ __global__ void __launch_bounds__(1024, 1) gn_stats_ring(const T* __restrict__ x
       if (!mbar_wait_bounded(bars + 8 * st, use & 1, err_word, VI_DEV_ERR_TMA_TIMEOUT)) break;
       const int nr = (int)min((int64_t)rg.rc, rg.rows - c * rg.rc);
       if (active) {
-        float a1lo = 0.f, a2lo = 0.f, a1hi = 0.f, a2hi = 0.f;
+        float s1[V], s2[V];
+#pragma unroll
+        for (int e = 0; e < V; ++e) s1[e] = s2[e] = 0.f;
         const uint32_t p0 = ring_stage(base, rg, st) + j * 16;
-        for (int r = rr; r < nr; r += rg.RB) {
+        int r = rr;
+        for (; r + rg.RB < nr; r += 2 * rg.RB) {        // two rows per step
+          float f[V], g[V];
+          unpack(lds128(p0 + r * rg.rowbytes), f);
+          unpack(lds128(p0 + (r + rg.RB) * rg.rowbytes), g);
+#pragma unroll
+          for (int e = 0; e < V; ++e) {
+            const float a = f[e] - kk[e], b = g[e] - kk[e];
+            s1[e] += a + b;
+            s2[e] = fmaf(a, a, fmaf(b, b, s2[e]));
+          }
+          nrows += 2;
+        }
+        if (r < nr) {
           float f[V];
           unpack(lds128(p0 + r * rg.rowbytes), f);
 #pragma unroll
           for (int e = 0; e < V; ++e) {
-            if (e < split) {
-              const float dv = f[e] - klo;
-              a1lo += dv; a2lo = fmaf(dv, dv, a2lo);
-            } else {
-              const float dv = f[e] - khi;
-              a1hi += dv; a2hi = fmaf(dv, dv, a2hi);
-            }
+            const float a = f[e] - kk[e];
+            s1[e] += a;
+            s2[e] = fmaf(a, a, s2[e]);
           }
           ++nrows;
+        }
+        float a1lo = 0.f, a2lo = 0.f, a1hi = 0.f, a2hi = 0.f;
+#pragma unroll
+        for (int e = 0; e < V; ++e) {
+          if (e < split) { a1lo += s1[e]; a2lo += s2[e]; }
+          else { a1hi += s1[e]; a2hi += s2[e]; }
         }
         d1lo += a1lo; d2lo += a2lo; d1hi += a1hi; d2hi += a2hi;
       }
@@ -390,7 +414,7 @@ static GnPlan gn_plan(int64_t rows, int C, int groups) {
   const int cg = C / groups;
   const int VPR = C / V;
   const int rowbytes = C * (int)sizeof(T);
-  bool ok = VPR <= 512 && rowbytes <= GN_CHUNK_MAX;
+  bool ok = VPR <= 960 && rowbytes <= GN_CHUNK_MAX;
   for (int c0 = 0; ok && c0 < C; c0 += V)
     if ((c0 + V - 1) / cg - c0 / cg > 1) ok = false;
   pl.ring = ok;
@@ -400,7 +424,7 @@ static GnPlan gn_plan(int64_t rows, int C, int groups) {
     g.C = C;
     g.rowbytes = rowbytes;
     g.VPR = VPR;
-    g.RB = 256 / VPR > 0 ? 256 / VPR : 1;
+    g.RB = 480 / VPR > 0 ? 480 / VPR : 1;
     g.rc = GN_CHUNK_MAX / rowbytes;
     g.stage_bytes = g.rc * rowbytes;
     g.nchunks = (rows + g.rc - 1) / g.rc;

@@ -10,24 +10,35 @@
 //   Y_p[f, co] = b[co] + sum_t sum_ci X_p[f + t - k/2, ci] W_t[co, ci]
 // of M = F frames, N = C output channels and K = k * C.
 //
-// Job = (position p, 128-frame block, slab of NJ output channels).  Per job
-// the CTA runs C/64 K-blocks; each K-block stages, with TMA, the x rows
-// [f0 - k/2, f0 + 128 + k/2) x 64 channels ONCE (a_rows = 127 + k rows) in the
-// no-swizzle K-major layout (rows 16 bytes apart inside each 8-channel
-// column, columns a_col >= 16*a_rows bytes apart, a multiple of 128), so the
-// k taps read the same shared tile through descriptors whose start differs by
-// 16 bytes per tap: the tap shift costs no extra load.  The
-// frame coordinate -1 (and F) reads as zero from TMA's out-of-bounds fill,
-// which is exactly the zero padding at the two ends of the video.  The
-// k weight slabs (NJ x 64 each) come from a repacked copy of w by 1-D bulk
-// copies.  One thread issues tcgen05.mma (M = 128, N = NJ, K = 16) into one
-// of two TMEM accumulators; four epilogue warps drain the other one (TMEM ->
-// registers, + bias, -> bf16 -> global), so the epilogue overlaps the next
-// job's MMAs.
+// Tile = (position p, block of 128 frames).  Job = (tile, or a pair of tiles
+// on a CTA pair, x slab of NJ output channels).  Per job the CTA runs C/64
+// K-blocks; each K-block stages, with one TMA load, the x rows
+// [f0 - k/2, f0 + 128 + k/2) x 64 channels ONCE (a_rows = 127 + k rows of 128
+// bytes, 128-byte swizzle), so the k taps read the same shared tile through
+// descriptors whose start differs by one 128-byte row per tap: the tap shift
+// costs no extra load.  The frame coordinate -1 (and F) reads as zero from
+// TMA's out-of-bounds fill, which is exactly the zero padding at the two ends
+// of the video.  The weights are repacked once per call so that every
+// (slab, K-block, tap) tile is a contiguous NJ x 64 block in the no-swizzle
+// K-major layout, fetched by a 2-D TMA box of 128-byte rows.
+//
+// PAIR = true (built, not dispatched: see TC_USE_PAIR): a cluster of two
+// CTAs on two SMs runs tcgen05.mma.cta_group::2 with M = 256: each CTA holds
+// its own 128-frame tile of x and HALF of every weight tile, and its own 128
+// accumulator rows in TMEM.  Per SM this halves the weight bytes streamed
+// from L2 per flop, which is what limits the one-SM form.  The even CTA's
+// single thread issues the MMAs; both CTAs' TMA loads complete on the even
+// CTA's barriers, commits are multicast to both CTAs, and the odd CTA's
+// epilogue arrives remotely on the even CTA's accumulator-empty barrier.
+//
+// One of two TMEM accumulators (NJ columns each) is drained by four epilogue
+// warps (TMEM -> registers, + bias, -> bf16 -> global) while the MMAs of the
+// next job fill the other.  Every CTA walks the K-blocks of a job starting at
+// its own offset, so the CTAs do not all stream the same weight tile at once.
 //
 // Warp roles (192 threads, one CTA per SM, persistent over jobs):
 //   warp 0      TMA producer (one elected thread)
-//   warp 1      TMEM allocator + MMA issuer (one elected thread)
+//   warp 1      TMEM allocator + MMA issuer (one thread, even CTA of a pair)
 //   warps 2..5  epilogue; warp w reads TMEM lanes 32*(w%4) .. +31
 #include <mutex>
 
@@ -36,52 +47,66 @@
 
 namespace vi {
 
-constexpr int TC_M = 128;        // frames per job = UMMA M = TMEM lanes
-constexpr int TC_KB = 64;        // input channels per K-block (8 columns of 8)
+constexpr int TC_M = 128;        // frames per tile = TMEM lanes per CTA
+constexpr int TC_KB = 64;        // input channels per K-block
 constexpr int TC_SA = 3;         // A (x) stages
-constexpr int TC_SB_MAX = 8;     // B (w) stages at most
+constexpr int TC_SB_MAX = 12;    // B (w) stages at most
 constexpr int TC_THREADS = 192;
 constexpr int TC_TMEM_COLS = 512;
 constexpr int TC_SMEM_LIMIT = 232448;   // 227 KB opt-in per CTA
 
+// Bounded wait; cluster-scope acquire when the barrier is signalled from the
+// other CTA of a pair (remote arrivals, multicast commits).
+template <bool PAIR>
+__device__ __forceinline__ bool tc_wait(uint32_t bar, uint32_t parity, unsigned int* err,
+                                        unsigned int code) {
+  if constexpr (PAIR) return mbar_wait_bounded_cluster(bar, parity, err, code);
+  else return mbar_wait_bounded(bar, parity, err, code);
+}
+
 struct TcPlan {
   int F, P, C, k;
   int NJ;                // output channels per job (UMMA N), multiple of 32
+  int H;                 // CTAs per MMA (1, or 2 for a pair); each holds NJ/H weight rows
   int n_slabs;           // C / NJ
   int n_fblk;            // ceil(F / 128)
-  long long n_jobs;      // P * n_fblk * n_slabs
+  long long n_tiles;     // P * n_fblk
+  long long n_jobs;      // ceil(n_tiles / H) * n_slabs
   int n_cb;              // C / 64
   int a_rows;            // 127 + k
-  int a_col;             // bytes between 8-channel columns of an A stage (128-aligned)
-  int a_stage;           // bytes per A stage, 1024-aligned
-  int b_stage;           // bytes per B stage = NJ * 64 * 2
+  int a_stage;           // bytes per A stage (a_rows x 128 B), 1024-aligned
+  int b_rows;            // weight rows per CTA per stage = NJ / H
+  int b_stage;           // bytes per B stage = b_rows * 128
   int sb;                // B stages
   int smem;              // dynamic shared memory bytes
 };
 
 struct TcArgs {
-  const bf16* wpk;       // packed weights [slab][cb][t][8 columns][NJ][8]
   const bf16* bias;
   bf16* y;
   unsigned int* err;
 };
 
-static bool tc_plan(int F, int P, int C, int k, TcPlan& pl) {
+static bool tc_plan(int F, int P, int C, int k, bool pair, TcPlan& pl) {
   if (k < 1 || k % 2 == 0 || 127 + k > 256 || C % TC_KB != 0) return false;
   int nj = 0;
   for (int cand = 256; cand >= 32; cand -= 32)
     if (C % cand == 0) { nj = cand; break; }
   if (nj == 0) return false;
+  const int H = pair ? 2 : 1;
+  if ((nj / H) % 8 != 0) return false;
   pl.F = F; pl.P = P; pl.C = C; pl.k = k;
   pl.NJ = nj;
+  pl.H = H;
   pl.n_slabs = C / nj;
   pl.n_fblk = (F + TC_M - 1) / TC_M;
-  pl.n_jobs = (long long)P * pl.n_fblk * pl.n_slabs;
+  pl.n_tiles = (long long)P * pl.n_fblk;
+  pl.n_jobs = ((pl.n_tiles + H - 1) / H) * pl.n_slabs;
   pl.n_cb = C / TC_KB;
   pl.a_rows = 127 + k;
-  pl.a_col = ((pl.a_rows * 16 + 127) / 128) * 128;     // TMA destinations are 128B-aligned
-  pl.a_stage = ((8 * pl.a_col + 1023) / 1024) * 1024;
-  pl.b_stage = nj * TC_KB * 2;
+  pl.a_stage = ((pl.a_rows * 128 + 1023) / 1024) * 1024;
+  pl.b_rows = nj / H;
+  pl.b_stage = pl.b_rows * 128;
   const int fixed = 1024 /* align slack */ + TC_SA * pl.a_stage + 4 * C /* bias */ + 512 /* bars */;
   int sb = (TC_SMEM_LIMIT - fixed) / pl.b_stage;
   if (sb > TC_SB_MAX) sb = TC_SB_MAX;
@@ -91,8 +116,10 @@ static bool tc_plan(int F, int P, int C, int k, TcPlan& pl) {
   return pl.smem <= TC_SMEM_LIMIT;
 }
 
+template <bool PAIR>
 __global__ void __launch_bounds__(TC_THREADS, 1)
-    temporal_conv_tc_kernel(const __grid_constant__ CUtensorMap tmx, const TcPlan pl,
+    temporal_conv_tc_kernel(const __grid_constant__ CUtensorMap tmx,
+                            const __grid_constant__ CUtensorMap tmw, const TcPlan pl,
                             const TcArgs args) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
@@ -108,127 +135,171 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   float* bias_s = reinterpret_cast<float*>(smem_raw + (sBias - smem_u32(smem_raw)));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const long long cluster_id = PAIR ? blockIdx.x / 2 : blockIdx.x;
+  const long long n_clusters = PAIR ? gridDim.x / 2 : gridDim.x;
+  // In a pair, the full barriers and the accumulator-empty barrier that count
+  // both CTAs live in the even CTA; these are their cluster addresses.
+  const uint32_t lead_a_full = PAIR ? mapa_shared(a_full, 0) : a_full;
+  const uint32_t lead_b_full = PAIR ? mapa_shared(b_full, 0) : b_full;
+  const uint32_t lead_acc_empty = PAIR ? mapa_shared(acc_empty, 0) : acc_empty;
+
   if (threadIdx.x == 0) {
-    for (int i = 0; i < TC_SA; ++i) { mbar_init(a_full + 8 * i, 1); mbar_init(a_empty + 8 * i, 1); }
-    for (int i = 0; i < pl.sb; ++i) { mbar_init(b_full + 8 * i, 1); mbar_init(b_empty + 8 * i, 1); }
-    for (int i = 0; i < 2; ++i) { mbar_init(acc_full + 8 * i, 1); mbar_init(acc_empty + 8 * i, 4); }
+    for (int i = 0; i < TC_SA; ++i) { mbar_init(a_full + 8 * i, PAIR ? 2 : 1); mbar_init(a_empty + 8 * i, 1); }
+    for (int i = 0; i < pl.sb; ++i) { mbar_init(b_full + 8 * i, PAIR ? 2 : 1); mbar_init(b_empty + 8 * i, 1); }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(acc_full + 8 * i, 1);
+      mbar_init(acc_empty + 8 * i, PAIR ? 8 : 4);
+    }
     mbar_init(drain, 1);
     fence_barrier_init();
   }
   for (int c = threadIdx.x; c < pl.C; c += blockDim.x) bias_s[c] = to_f32(args.bias[c]);
   if (warp == 1) {
-    tmem_alloc(tmem_slot, TC_TMEM_COLS);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(tmem_slot, TC_TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, TC_TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) cluster_sync();      // barriers of both CTAs initialised
   tc_fence_after();
   uint32_t tmem_base;
   asm volatile("ld.shared.u32 %0, [%1];" : "=r"(tmem_base) : "r"(tmem_slot));
 
   const int halo = pl.k / 2;
+  const int cb_rot = (int)(cluster_id % pl.n_cb);
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      long long a_it = 0, b_it = 0;
+      // Ring positions as (stage, phase) counters: no division in the loop.
+      int sa = 0, pa = 0, sbi = 0, pb = 0;
+      bool a_used = false, b_used = false;         // first pass over a ring needs no wait
       bool ok = true;
-      for (long long job = blockIdx.x; job < pl.n_jobs && ok; job += gridDim.x) {
+      for (long long job = cluster_id; job < pl.n_jobs && ok; job += n_clusters) {
         const int slab = (int)(job % pl.n_slabs);
-        const long long rest = job / pl.n_slabs;
-        const int fb = (int)(rest % pl.n_fblk);
-        const int p = (int)(rest / pl.n_fblk);
+        const long long tile = (job / pl.n_slabs) * pl.H + rank;
+        const int fb = (int)(tile % pl.n_fblk);
+        const int p = (int)(tile / pl.n_fblk);     // == P past the last tile: reads as zeros
         const int f0 = fb * TC_M;
-        for (int cb = 0; cb < pl.n_cb && ok; ++cb) {
-          const int sa = (int)(a_it % TC_SA);
-          const long long ua = a_it / TC_SA;
-          if (ua > 0 && !mbar_wait_bounded(a_empty + 8 * sa, (uint32_t)((ua - 1) & 1), args.err,
-                                           VI_DEV_ERR_TMA_TIMEOUT)) { ok = false; break; }
+        int wrow = (slab * pl.n_cb * pl.k * pl.H + (int)rank) * pl.b_rows;   // row of (slab, cb 0, t 0)
+        const int wrow_cb = pl.k * pl.H * pl.b_rows, wrow_t = pl.H * pl.b_rows;
+        for (int ib = 0; ib < pl.n_cb && ok; ++ib) {
+          const int cb = (ib + cb_rot) % pl.n_cb;
+          if (a_used && !tc_wait<PAIR>(a_empty + 8 * sa, (uint32_t)(pa ^ 1), args.err,
+                                       VI_DEV_ERR_TMA_TIMEOUT)) { ok = false; break; }
           const uint32_t dst = sA + sa * pl.a_stage;
-          mbar_arrive_expect_tx(a_full + 8 * sa, (uint32_t)pl.a_rows * 128u);
-          // 8 columns of 8 channels; column c lands at dst + c * a_col.
-#pragma unroll 1
-          for (int c = 0; c < 8; ++c)
-            tma_load_3d(dst + c * pl.a_col, &tmx, cb * TC_KB + c * 8, f0 - halo, p,
-                        a_full + 8 * sa);
-          ++a_it;
+          if constexpr (PAIR) {
+            mbar_arrive_expect_tx_cluster(lead_a_full + 8 * sa, (uint32_t)pl.a_rows * 128u);
+            tma_load_3d_pair(dst, &tmx, cb * TC_KB, f0 - halo, p, lead_a_full + 8 * sa);
+          } else {
+            mbar_arrive_expect_tx(a_full + 8 * sa, (uint32_t)pl.a_rows * 128u);
+            tma_load_3d(dst, &tmx, cb * TC_KB, f0 - halo, p, a_full + 8 * sa);
+          }
+          if (++sa == TC_SA) { sa = 0; pa ^= 1; a_used = true; }
           for (int t = 0; t < pl.k; ++t) {
-            const int s = (int)(b_it % pl.sb);
-            const long long ub = b_it / pl.sb;
-            if (ub > 0 && !mbar_wait_bounded(b_empty + 8 * s, (uint32_t)((ub - 1) & 1), args.err,
-                                             VI_DEV_ERR_TMA_TIMEOUT)) { ok = false; break; }
-            mbar_arrive_expect_tx(b_full + 8 * s, (uint32_t)pl.b_stage);
-            const bf16* src = args.wpk + ((size_t)(slab * pl.n_cb + cb) * pl.k + t) *
-                                             (size_t)(pl.NJ * TC_KB);
-            bulk_load(sB + s * pl.b_stage, src, (uint32_t)pl.b_stage, b_full + 8 * s);
-            ++b_it;
+            if (b_used && !tc_wait<PAIR>(b_empty + 8 * sbi, (uint32_t)(pb ^ 1), args.err,
+                                         VI_DEV_ERR_TMA_TIMEOUT)) { ok = false; break; }
+            // Row of this CTA's weight block in the packed [..][128 B] view.
+            const int row = wrow + cb * wrow_cb + t * wrow_t;
+            if constexpr (PAIR) {
+              mbar_arrive_expect_tx_cluster(lead_b_full + 8 * sbi, (uint32_t)pl.b_stage);
+              tma_load_2d_pair(sB + sbi * pl.b_stage, &tmw, 0, row, lead_b_full + 8 * sbi);
+            } else {
+              mbar_arrive_expect_tx(b_full + 8 * sbi, (uint32_t)pl.b_stage);
+              tma_load_2d(sB + sbi * pl.b_stage, &tmw, 0, row, b_full + 8 * sbi);
+            }
+            if (++sbi == pl.sb) { sbi = 0; pb ^= 1; b_used = true; }
           }
         }
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc = umma_idesc_bf16_f32(TC_M, pl.NJ);
-      const uint32_t lbo_a = (uint32_t)pl.a_col, lbo_b = (uint32_t)pl.NJ * 16u;
-      long long a_it = 0, b_it = 0, j_it = 0;
+    if (lane == 0 && rank == 0) {
+      const uint32_t idesc = umma_idesc_bf16_f32(TC_M * pl.H, pl.NJ);
+      const uint32_t lbo_b = (uint32_t)pl.b_rows * 16u;
+      // Descriptors of stage 0; stage s adds s * stage_bytes / 16 to the start field.
+      const uint64_t ad_base = umma_desc_kmajor_sw128(sA, 1024u);
+      const uint64_t bd_base = umma_desc_kmajor_noswizzle(sB, lbo_b, 128u);
+      const uint32_t a_st16 = (uint32_t)pl.a_stage >> 4, b_st16 = (uint32_t)pl.b_stage >> 4;
+      const uint32_t bk16 = (2u * lbo_b) >> 4;     // one K step of 16 in w
+      int sa = 0, pa = 0, sbi = 0, pb = 0, buf = 0, pacc = 0;
+      bool acc_used = false;
       bool ok = true;
-      for (long long job = blockIdx.x; job < pl.n_jobs && ok; job += gridDim.x, ++j_it) {
-        const int buf = (int)(j_it & 1);
-        const long long use = j_it >> 1;
-        if (use > 0 && !mbar_wait_bounded(acc_empty + 8 * buf, (uint32_t)((use - 1) & 1), args.err,
-                                          VI_DEV_ERR_MMA_TIMEOUT)) { ok = false; break; }
+      for (long long job = cluster_id; job < pl.n_jobs && ok; job += n_clusters) {
+        if (acc_used && !tc_wait<PAIR>(acc_empty + 8 * buf, (uint32_t)(pacc ^ 1), args.err,
+                                       VI_DEV_ERR_MMA_TIMEOUT)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(buf * pl.NJ);
-        for (int cb = 0; cb < pl.n_cb && ok; ++cb) {
-          const int sa = (int)(a_it % TC_SA);
-          if (!mbar_wait_bounded(a_full + 8 * sa, (uint32_t)((a_it / TC_SA) & 1), args.err,
-                                 VI_DEV_ERR_TMA_TIMEOUT)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t a_base = sA + sa * pl.a_stage;
-          for (int t = 0; t < pl.k; ++t) {
-            const int s = (int)(b_it % pl.sb);
-            if (!mbar_wait_bounded(b_full + 8 * s, (uint32_t)((b_it / pl.sb) & 1), args.err,
-                                   VI_DEV_ERR_TMA_TIMEOUT)) { ok = false; break; }
-            tc_fence_after();
-            const uint32_t b_base = sB + s * pl.b_stage;
-#pragma unroll
-            for (int ks = 0; ks < TC_KB / 16; ++ks) {
-              const uint64_t ad =
-                  umma_desc_kmajor_noswizzle(a_base + 16u * t + 2u * ks * lbo_a, lbo_a, 128u);
-              const uint64_t bd =
-                  umma_desc_kmajor_noswizzle(b_base + 2u * ks * lbo_b, lbo_b, 128u);
-              umma_bf16(d_tmem, ad, bd, idesc, (cb | t | ks) != 0 ? 1u : 0u);
-            }
-            umma_commit(b_empty + 8 * s);       // frees the w stage when these MMAs finish
-            ++b_it;
+        uint32_t acc = 0u;
+        for (int ib = 0; ib < pl.n_cb && ok; ++ib) {
+          if (!tc_wait<PAIR>(a_full + 8 * sa, (uint32_t)pa, args.err, VI_DEV_ERR_TMA_TIMEOUT)) {
+            ok = false;
+            break;
           }
-          umma_commit(a_empty + 8 * sa);        // frees the x stage
-          ++a_it;
+          tc_fence_after();
+          const uint64_t ad_stage = ad_base + (uint64_t)(sa * a_st16);
+          for (int t = 0; t < pl.k; ++t) {
+            if (!tc_wait<PAIR>(b_full + 8 * sbi, (uint32_t)pb, args.err, VI_DEV_ERR_TMA_TIMEOUT)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            // Tap t: the x tile shifted down by t rows of 128 B (8 units of 16 B).
+            const uint64_t ad = ad_stage + (uint64_t)(8u * t);
+            const uint64_t bd = bd_base + (uint64_t)(sbi * b_st16);
+            // K steps of 16: +32 B inside the swizzled x rows, +2 columns of 8 in w.
+            if constexpr (PAIR) {
+              umma_bf16_pair(d_tmem, ad, bd, idesc, acc);
+              umma_bf16_pair(d_tmem, ad + 2u, bd + bk16, idesc, 1u);
+              umma_bf16_pair(d_tmem, ad + 4u, bd + 2u * bk16, idesc, 1u);
+              umma_bf16_pair(d_tmem, ad + 6u, bd + 3u * bk16, idesc, 1u);
+              umma_commit_pair_mc(b_empty + 8 * sbi, 0x3);
+            } else {
+              umma_bf16(d_tmem, ad, bd, idesc, acc);
+              umma_bf16(d_tmem, ad + 2u, bd + bk16, idesc, 1u);
+              umma_bf16(d_tmem, ad + 4u, bd + 2u * bk16, idesc, 1u);
+              umma_bf16(d_tmem, ad + 6u, bd + 3u * bk16, idesc, 1u);
+              umma_commit(b_empty + 8 * sbi);       // frees the w stage when these MMAs finish
+            }
+            acc = 1u;
+            if (++sbi == pl.sb) { sbi = 0; pb ^= 1; }
+          }
+          if constexpr (PAIR) umma_commit_pair_mc(a_empty + 8 * sa, 0x3);
+          else umma_commit(a_empty + 8 * sa);         // frees the x stage
+          if (++sa == TC_SA) { sa = 0; pa ^= 1; }
         }
-        umma_commit(acc_full + 8 * buf);        // accumulator ready for the epilogue
+        if constexpr (PAIR) umma_commit_pair_mc(acc_full + 8 * buf, 0x3);
+        else umma_commit(acc_full + 8 * buf);         // accumulator ready for the epilogue
+        if (++buf == 2) { buf = 0; pacc ^= 1; acc_used = true; }
       }
-      // Wait for every MMA this thread issued before TMEM can be released.
-      umma_commit(drain);
-      mbar_wait_bounded(drain, 0, args.err, VI_DEV_ERR_MMA_TIMEOUT);
+      // Every MMA this thread issued must finish before TMEM is released.
+      if constexpr (PAIR) umma_commit_pair_mc(drain, 0x3);
+      else umma_commit(drain);
+      tc_wait<PAIR>(drain, 0, args.err, VI_DEV_ERR_MMA_TIMEOUT);
     }
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;                      // TMEM lane quadrant of this warp
-    const int m = 32 * q + lane;                 // frame within the job
-    long long j_it = 0;
-    for (long long job = blockIdx.x; job < pl.n_jobs; job += gridDim.x, ++j_it) {
-      const int buf = (int)(j_it & 1);
-      if (!mbar_wait_bounded(acc_full + 8 * buf, (uint32_t)((j_it >> 1) & 1), args.err,
-                             VI_DEV_ERR_MMA_TIMEOUT))
+    const int m = 32 * q + lane;                 // frame within the tile
+    int buf = 0, pacc = 0;
+    for (long long job = cluster_id; job < pl.n_jobs; job += n_clusters) {
+      if (!tc_wait<PAIR>(acc_full + 8 * buf, (uint32_t)pacc, args.err, VI_DEV_ERR_MMA_TIMEOUT))
         break;
       tc_fence_after();
       const int slab = (int)(job % pl.n_slabs);
-      const long long rest = job / pl.n_slabs;
-      const int fb = (int)(rest % pl.n_fblk);
-      const long long p = rest / pl.n_fblk;
+      const long long tile = (job / pl.n_slabs) * pl.H + rank;
+      const int fb = (int)(tile % pl.n_fblk);
+      const long long p = tile / pl.n_fblk;
       const int f = fb * TC_M + m;
-      const bool valid = f < pl.F;
-      bf16* out = args.y + ((size_t)p * pl.F + (valid ? f : 0)) * pl.C + (size_t)slab * pl.NJ;
+      const bool valid = tile < pl.n_tiles && f < pl.F;
+      bf16* out = args.y + ((size_t)(valid ? p : 0) * pl.F + (valid ? f : 0)) * pl.C +
+                  (size_t)slab * pl.NJ;
       const float* bs = bias_s + slab * pl.NJ;
       for (int c0 = 0; c0 < pl.NJ; c0 += 32) {
         uint32_t r[32];
@@ -242,38 +313,47 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                                __uint_as_float(r[2 * i + 1]) + bs[c0 + 2 * i + 1]);
           uint4* o = reinterpret_cast<uint4*>(out + c0);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) o[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          for (int i = 0; i < 4; ++i)
+            o[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
         }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(acc_empty + 8 * buf);
+      if (lane == 0) {
+        if constexpr (PAIR) mbar_arrive_cluster(lead_acc_empty + 8 * buf);
+        else mbar_arrive(acc_empty + 8 * buf);
+      }
+      if (++buf == 2) { buf = 0; pacc ^= 1; }
     }
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) cluster_sync();        // the pair is done with each other's memory
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, TC_TMEM_COLS);
+    if constexpr (PAIR) tmem_dealloc_pair(tmem_base, TC_TMEM_COLS);
+    else tmem_dealloc(tmem_base, TC_TMEM_COLS);
   }
 }
 
-// w [C_out][C_in][k] -> [slab][cb][t][8 columns][NJ][8]: for each (slab, K-block,
-// tap) an NJ x 64 K-major tile in the no-swizzle layout, contiguous.
+// w [C_out][C_in][k] -> [slab][cb][t][h][8 columns][NJ/H][8]: for each (slab,
+// K-block, tap, CTA of the pair) an NJ/H x 64 K-major block in the no-swizzle
+// layout, contiguous.
 __global__ void temporal_conv_pack_w(const bf16* __restrict__ w, bf16* __restrict__ wpk, int C,
-                                     int k, int NJ) {
+                                     int k, int NJ, int H) {
   const long long total = (long long)C * C * k;
-  const int n_cb = C / TC_KB;
+  const int n_cb = C / TC_KB, R = NJ / H;
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
        i += (long long)gridDim.x * blockDim.x) {
     const int e = (int)(i & 7);
     long long r = i >> 3;
-    const int n = (int)(r % NJ); r /= NJ;
+    const int n = (int)(r % R); r /= R;
     const int col = (int)(r % 8); r /= 8;
+    const int h = (int)(r % H); r /= H;
     const int t = (int)(r % k); r /= k;
     const int cb = (int)(r % n_cb);
     const int slab = (int)(r / n_cb);
-    const int co = slab * NJ + n, ci = cb * TC_KB + col * 8 + e;
+    const int co = slab * NJ + h * R + n, ci = cb * TC_KB + col * 8 + e;
     wpk[i] = w[((size_t)co * C + ci) * k + t];
   }
 }
@@ -282,26 +362,18 @@ bool encode_tmap(CUtensorMap* map, const void* base, int rank, const uint64_t* d
                  const uint64_t* strides_bytes, const uint32_t* box, CUtensorMapSwizzle swz,
                  CUtensorMapDataType dt);
 
+// The CTA-pair form is correct but, measured on B200, slower than the
+// one-SM form at every workload here, so the dispatcher takes the one-SM form.
+constexpr bool TC_USE_PAIR = false;
+
 bool temporal_conv_tc_ok(int F, int P, int C, int k) {
   TcPlan pl;
-  return F > 0 && P > 0 && tc_plan(F, P, C, k, pl);
+  return F > 0 && P > 0 && tc_plan(F, P, C, k, TC_USE_PAIR, pl);
 }
 
-int temporal_conv_bf16_tc(const bf16* x, const bf16* w, const bf16* b, bf16* y, int F, int P,
-                          int C, int k, cudaStream_t stream) {
-  TcPlan pl;
-  if (!tc_plan(F, P, C, k, pl)) return VI_ERR_UNSUPPORTED;
-  unsigned int* err = device_error_word();
-  if (!err) return VI_ERR_CUDA;
-  // x as [P][F][C]: box of 8 channels x a_rows frames x 1 position, no swizzle.
-  CUtensorMap tmx;
-  const uint64_t dims[3] = {(uint64_t)C, (uint64_t)F, (uint64_t)P};
-  const uint64_t strides[2] = {(uint64_t)C * 2, (uint64_t)F * C * 2};
-  const uint32_t box[3] = {8, (uint32_t)pl.a_rows, 1};
-  if (!encode_tmap(&tmx, x, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE,
-                   CU_TENSOR_MAP_DATA_TYPE_BFLOAT16))
-    return VI_ERR_CUDA;
-
+template <bool PAIR>
+static int tc_launch(const CUtensorMap& tmx, const CUtensorMap& tmw, const TcPlan& pl,
+                     const TcArgs& a, cudaStream_t stream) {
   static std::mutex mu;
   static bool attr_done[64] = {false};
   int dev = 0;
@@ -309,29 +381,85 @@ int temporal_conv_bf16_tc(const bf16* x, const bf16* w, const bf16* b, bf16* y, 
   {
     std::lock_guard<std::mutex> lock(mu);
     if (dev < 64 && !attr_done[dev]) {
-      VI_CUDA_TRY(cudaFuncSetAttribute(temporal_conv_tc_kernel,
+      VI_CUDA_TRY(cudaFuncSetAttribute(temporal_conv_tc_kernel<PAIR>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        TC_SMEM_LIMIT));
       attr_done[dev] = true;
     }
+  }
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.blockDim = dim3(TC_THREADS);
+  cfg.dynamicSmemBytes = (size_t)pl.smem;
+  cfg.stream = stream;
+  long long grid;
+  if constexpr (PAIR) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cfg.gridDim = dim3(2 * sm_count());
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, temporal_conv_tc_kernel<PAIR>, &cfg) !=
+            cudaSuccess ||
+        clusters < 1)
+      clusters = sm_count() / 2;
+    grid = clusters;
+    if (grid > pl.n_jobs) grid = pl.n_jobs;
+    grid *= 2;
+  } else {
+    grid = sm_count();
+    if (grid > pl.n_jobs) grid = pl.n_jobs;
+  }
+  cfg.gridDim = dim3((unsigned)grid);
+  VI_CUDA_TRY(cudaLaunchKernelEx(&cfg, temporal_conv_tc_kernel<PAIR>, tmx, tmw, pl, a));
+  note_launch();
+  return VI_OK;
+}
+
+int temporal_conv_bf16_tc(const bf16* x, const bf16* w, const bf16* b, bf16* y, int F, int P,
+                          int C, int k, cudaStream_t stream) {
+  TcPlan pl;
+  const bool pair = TC_USE_PAIR && tc_plan(F, P, C, k, true, pl);
+  if (!pair && !tc_plan(F, P, C, k, false, pl)) return VI_ERR_UNSUPPORTED;
+  unsigned int* err = device_error_word();
+  if (!err) return VI_ERR_CUDA;
+  // x as [P][F][C]: box of 64 channels x a_rows frames x 1 position, 128B swizzle.
+  CUtensorMap tmx, tmw;
+  {
+    const uint64_t dims[3] = {(uint64_t)C, (uint64_t)F, (uint64_t)P};
+    const uint64_t strides[2] = {(uint64_t)C * 2, (uint64_t)F * C * 2};
+    const uint32_t box[3] = {(uint32_t)TC_KB, (uint32_t)pl.a_rows, 1};
+    if (!encode_tmap(&tmx, x, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_DATA_TYPE_BFLOAT16))
+      return VI_ERR_CUDA;
   }
   const size_t wbytes = (size_t)C * C * k * sizeof(bf16);
   void* wpk = nullptr;
   VI_CUDA_TRY(cudaMallocAsync(&wpk, wbytes, stream));
   int st = VI_OK;
   {
+    // Packed weights viewed as rows of 128 bytes; one box = one CTA's block.
+    const uint64_t dims[2] = {64, (uint64_t)C * C * k / 64};
+    const uint64_t strides[1] = {128};
+    const uint32_t box[2] = {64, (uint32_t)pl.b_rows};
+    if (!encode_tmap(&tmw, wpk, 2, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE,
+                     CU_TENSOR_MAP_DATA_TYPE_BFLOAT16))
+      st = VI_ERR_CUDA;
+  }
+  if (st == VI_OK) {
     const long long total = (long long)C * C * k;
     int blocks = (int)((total + 255) / 256);
     if (blocks > 4 * sm_count()) blocks = 4 * sm_count();
-    temporal_conv_pack_w<<<blocks, 256, 0, stream>>>(w, static_cast<bf16*>(wpk), C, k, pl.NJ);
+    temporal_conv_pack_w<<<blocks, 256, 0, stream>>>(w, static_cast<bf16*>(wpk), C, k, pl.NJ,
+                                                     pl.H);
     if (cudaGetLastError() != cudaSuccess) st = VI_ERR_CUDA; else note_launch();
   }
   if (st == VI_OK) {
-    TcArgs a{static_cast<const bf16*>(wpk), b, y, err};
-    long long grid = sm_count();
-    if (grid > pl.n_jobs) grid = pl.n_jobs;
-    temporal_conv_tc_kernel<<<(unsigned)grid, TC_THREADS, pl.smem, stream>>>(tmx, pl, a);
-    if (cudaGetLastError() != cudaSuccess) st = VI_ERR_CUDA; else note_launch();
+    TcArgs a{b, y, err};
+    st = pair ? tc_launch<true>(tmx, tmw, pl, a, stream) : tc_launch<false>(tmx, tmw, pl, a, stream);
   }
   if (cudaFreeAsync(wpk, stream) != cudaSuccess && st == VI_OK) st = VI_ERR_CUDA;
   return st;
