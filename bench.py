@@ -377,14 +377,27 @@ def run_e2e(args, w, host, dev, stream):
 
 
 def load_traffic(kernel, w):
-    """DRAM bytes per launch from the committed ncu summary of this kernel, if current."""
+    """DRAM bytes per launch from the committed ncu summary of this kernel.
+
+    None when there is no capture for this workload, or when the kernel's
+    source has changed since the counters were taken (the summary records a
+    hash of the source file it was measured with)."""
+    import hashlib
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as fh:
         d = json.load(fh)
     e = d.get(kernel, {}).get(w.name)
-    return None if e is None else e.get("bytes_per_launch")
+    if e is None:
+        return None
+    src = os.path.join(ROOT, "clip_temporal_modules_b200", e["source"])
+    if not os.path.exists(src):
+        return None
+    with open(src, "rb") as fh:
+        if hashlib.sha256(fh.read()).hexdigest()[:16] != e.get("source_sha256_16"):
+            return None
+    return e.get("bytes_per_launch")
 
 
 # ---------------------------------------------------------------------------
