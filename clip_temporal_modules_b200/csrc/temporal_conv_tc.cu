@@ -49,8 +49,9 @@ namespace vi {
 
 constexpr int TC_M = 128;        // frames per tile = TMEM lanes per CTA
 constexpr int TC_KB = 64;        // input channels per K-block
-constexpr int TC_SA = 3;         // A (x) stages
-constexpr int TC_SB_MAX = 12;    // B (w) stages at most
+constexpr int TC_SA = 2;         // A (x) stages
+constexpr int TC_SB_MAX = 8;     // B (w) stages at most
+constexpr int TC_NJ_MAX = 160;   // a B stage holds all k taps of one K-block
 constexpr int TC_THREADS = 192;
 constexpr int TC_TMEM_COLS = 512;
 constexpr int TC_SMEM_LIMIT = 232448;   // 227 KB opt-in per CTA
@@ -75,8 +76,9 @@ struct TcPlan {
   int n_cb;              // C / 64
   int a_rows;            // 127 + k
   int a_stage;           // bytes per A stage (a_rows x 128 B), 1024-aligned
-  int b_rows;            // weight rows per CTA per stage = NJ / H
-  int b_stage;           // bytes per B stage = b_rows * 128
+  int b_rows;            // weight rows per CTA per tap = NJ / H
+  int b_tap;             // bytes of one tap's block = b_rows * 128
+  int b_stage;           // bytes per B stage = k * b_tap (one K-block, all taps)
   int sb;                // B stages
   int smem;              // dynamic shared memory bytes
 };
@@ -89,31 +91,36 @@ struct TcArgs {
 
 static bool tc_plan(int F, int P, int C, int k, bool pair, TcPlan& pl) {
   if (k < 1 || k % 2 == 0 || 127 + k > 256 || C % TC_KB != 0) return false;
-  int nj = 0;
-  for (int cand = 256; cand >= 32; cand -= 32)
-    if (C % cand == 0) { nj = cand; break; }
-  if (nj == 0) return false;
   const int H = pair ? 2 : 1;
-  if ((nj / H) % 8 != 0) return false;
-  pl.F = F; pl.P = P; pl.C = C; pl.k = k;
-  pl.NJ = nj;
-  pl.H = H;
-  pl.n_slabs = C / nj;
-  pl.n_fblk = (F + TC_M - 1) / TC_M;
-  pl.n_tiles = (long long)P * pl.n_fblk;
-  pl.n_jobs = ((pl.n_tiles + H - 1) / H) * pl.n_slabs;
-  pl.n_cb = C / TC_KB;
-  pl.a_rows = 127 + k;
-  pl.a_stage = ((pl.a_rows * 128 + 1023) / 1024) * 1024;
-  pl.b_rows = nj / H;
-  pl.b_stage = pl.b_rows * 128;
-  const int fixed = 1024 /* align slack */ + TC_SA * pl.a_stage + 4 * C /* bias */ + 512 /* bars */;
-  int sb = (TC_SMEM_LIMIT - fixed) / pl.b_stage;
-  if (sb > TC_SB_MAX) sb = TC_SB_MAX;
-  if (sb < 2) return false;
-  pl.sb = sb;
-  pl.smem = fixed + sb * pl.b_stage;
-  return pl.smem <= TC_SMEM_LIMIT;
+  const int a_rows = 127 + k;
+  const int a_stage = ((a_rows * 128 + 1023) / 1024) * 1024;
+  const int fixed = 1024 /* align slack */ + TC_SA * a_stage + 4 * C /* bias */ + 512 /* bars */;
+  // Widest slab (<= 160 output channels, a multiple of 32 dividing C) whose
+  // all-tap weight stage still leaves room for two stages.
+  for (int nj = TC_NJ_MAX; nj >= 32; nj -= 32) {
+    if (C % nj != 0 || (nj / H) % 8 != 0) continue;
+    const int b_stage = k * (nj / H) * 128;
+    int sb = (TC_SMEM_LIMIT - fixed) / b_stage;
+    if (sb > TC_SB_MAX) sb = TC_SB_MAX;
+    if (sb < 2) continue;
+    pl.F = F; pl.P = P; pl.C = C; pl.k = k;
+    pl.NJ = nj;
+    pl.H = H;
+    pl.n_slabs = C / nj;
+    pl.n_fblk = (F + TC_M - 1) / TC_M;
+    pl.n_tiles = (long long)P * pl.n_fblk;
+    pl.n_jobs = ((pl.n_tiles + H - 1) / H) * pl.n_slabs;
+    pl.n_cb = C / TC_KB;
+    pl.a_rows = a_rows;
+    pl.a_stage = a_stage;
+    pl.b_rows = nj / H;
+    pl.b_tap = pl.b_rows * 128;
+    pl.b_stage = b_stage;
+    pl.sb = sb;
+    pl.smem = fixed + sb * b_stage;
+    return pl.smem <= TC_SMEM_LIMIT;
+  }
+  return false;
 }
 
 template <bool PAIR>
@@ -201,20 +208,19 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             tma_load_3d(dst, &tmx, cb * TC_KB, f0 - halo, p, a_full + 8 * sa);
           }
           if (++sa == TC_SA) { sa = 0; pa ^= 1; a_used = true; }
+          // One B stage = this CTA's weight blocks of every tap of K-block cb.
+          if (b_used && !tc_wait<PAIR>(b_empty + 8 * sbi, (uint32_t)(pb ^ 1), args.err,
+                                       VI_DEV_ERR_TMA_TIMEOUT)) { ok = false; break; }
+          if constexpr (PAIR) mbar_arrive_expect_tx_cluster(lead_b_full + 8 * sbi, (uint32_t)pl.b_stage);
+          else mbar_arrive_expect_tx(b_full + 8 * sbi, (uint32_t)pl.b_stage);
           for (int t = 0; t < pl.k; ++t) {
-            if (b_used && !tc_wait<PAIR>(b_empty + 8 * sbi, (uint32_t)(pb ^ 1), args.err,
-                                         VI_DEV_ERR_TMA_TIMEOUT)) { ok = false; break; }
             // Row of this CTA's weight block in the packed [..][128 B] view.
             const int row = wrow + cb * wrow_cb + t * wrow_t;
-            if constexpr (PAIR) {
-              mbar_arrive_expect_tx_cluster(lead_b_full + 8 * sbi, (uint32_t)pl.b_stage);
-              tma_load_2d_pair(sB + sbi * pl.b_stage, &tmw, 0, row, lead_b_full + 8 * sbi);
-            } else {
-              mbar_arrive_expect_tx(b_full + 8 * sbi, (uint32_t)pl.b_stage);
-              tma_load_2d(sB + sbi * pl.b_stage, &tmw, 0, row, b_full + 8 * sbi);
-            }
-            if (++sbi == pl.sb) { sbi = 0; pb ^= 1; b_used = true; }
+            const uint32_t dstb = sB + sbi * pl.b_stage + t * pl.b_tap;
+            if constexpr (PAIR) tma_load_2d_pair(dstb, &tmw, 0, row, lead_b_full + 8 * sbi);
+            else tma_load_2d(dstb, &tmw, 0, row, b_full + 8 * sbi);
           }
+          if (++sbi == pl.sb) { sbi = 0; pb ^= 1; b_used = true; }
         }
       }
     }
@@ -227,6 +233,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       const uint64_t ad_base = umma_desc_kmajor_sw128(sA, 1024u);
       const uint64_t bd_base = umma_desc_kmajor_noswizzle(sB, lbo_b, 128u);
       const uint32_t a_st16 = (uint32_t)pl.a_stage >> 4, b_st16 = (uint32_t)pl.b_stage >> 4;
+      const uint32_t bt16 = (uint32_t)pl.b_tap >> 4;  // one tap's block in w
       const uint32_t bk16 = (2u * lbo_b) >> 4;     // one K step of 16 in w
       int sa = 0, pa = 0, sbi = 0, pb = 0, buf = 0, pacc = 0;
       bool acc_used = false;
@@ -238,40 +245,42 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         const uint32_t d_tmem = tmem_base + (uint32_t)(buf * pl.NJ);
         uint32_t acc = 0u;
         for (int ib = 0; ib < pl.n_cb && ok; ++ib) {
-          if (!tc_wait<PAIR>(a_full + 8 * sa, (uint32_t)pa, args.err, VI_DEV_ERR_TMA_TIMEOUT)) {
+          if (!tc_wait<PAIR>(a_full + 8 * sa, (uint32_t)pa, args.err, VI_DEV_ERR_TMA_TIMEOUT) ||
+              !tc_wait<PAIR>(b_full + 8 * sbi, (uint32_t)pb, args.err, VI_DEV_ERR_TMA_TIMEOUT)) {
             ok = false;
             break;
           }
           tc_fence_after();
+          // k taps x 4 K steps = 4k MMAs back to back (12 for k = 3): enough
+          // tensor work queued to hide the wait/commit of the next K-block.
           const uint64_t ad_stage = ad_base + (uint64_t)(sa * a_st16);
+          const uint64_t bd_stage = bd_base + (uint64_t)(sbi * b_st16);
           for (int t = 0; t < pl.k; ++t) {
-            if (!tc_wait<PAIR>(b_full + 8 * sbi, (uint32_t)pb, args.err, VI_DEV_ERR_TMA_TIMEOUT)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
             // Tap t: the x tile shifted down by t rows of 128 B (8 units of 16 B).
             const uint64_t ad = ad_stage + (uint64_t)(8u * t);
-            const uint64_t bd = bd_base + (uint64_t)(sbi * b_st16);
+            const uint64_t bd = bd_stage + (uint64_t)(t * bt16);
             // K steps of 16: +32 B inside the swizzled x rows, +2 columns of 8 in w.
             if constexpr (PAIR) {
               umma_bf16_pair(d_tmem, ad, bd, idesc, acc);
               umma_bf16_pair(d_tmem, ad + 2u, bd + bk16, idesc, 1u);
               umma_bf16_pair(d_tmem, ad + 4u, bd + 2u * bk16, idesc, 1u);
               umma_bf16_pair(d_tmem, ad + 6u, bd + 3u * bk16, idesc, 1u);
-              umma_commit_pair_mc(b_empty + 8 * sbi, 0x3);
             } else {
               umma_bf16(d_tmem, ad, bd, idesc, acc);
               umma_bf16(d_tmem, ad + 2u, bd + bk16, idesc, 1u);
               umma_bf16(d_tmem, ad + 4u, bd + 2u * bk16, idesc, 1u);
               umma_bf16(d_tmem, ad + 6u, bd + 3u * bk16, idesc, 1u);
-              umma_commit(b_empty + 8 * sbi);       // frees the w stage when these MMAs finish
             }
             acc = 1u;
-            if (++sbi == pl.sb) { sbi = 0; pb ^= 1; }
           }
-          if constexpr (PAIR) umma_commit_pair_mc(a_empty + 8 * sa, 0x3);
-          else umma_commit(a_empty + 8 * sa);         // frees the x stage
+          if constexpr (PAIR) {
+            umma_commit_pair_mc(b_empty + 8 * sbi, 0x3);
+            umma_commit_pair_mc(a_empty + 8 * sa, 0x3);
+          } else {
+            umma_commit(b_empty + 8 * sbi);       // frees the w stage when these MMAs finish
+            umma_commit(a_empty + 8 * sa);        // frees the x stage
+          }
+          if (++sbi == pl.sb) { sbi = 0; pb ^= 1; }
           if (++sa == TC_SA) { sa = 0; pa ^= 1; }
         }
         if constexpr (PAIR) umma_commit_pair_mc(acc_full + 8 * buf, 0x3);
