@@ -503,12 +503,12 @@ int groupnorm_global(const T* x, const T* gamma, const T* beta, T* y, int64_t ro
                      int groups, float eps, cudaStream_t stream) {
   const size_t bytes = gn_scratch_bytes<T>(rows, C, groups);
   void* scratch = nullptr;
-  VI_CUDA_TRY(cudaMallocAsync(&scratch, bytes, stream));
+  VI_CUDA_TRY(scratch_alloc(&scratch, bytes, stream));
   cudaError_t e = cudaMemsetAsync(scratch, 0, 64, stream);
   int st = (e == cudaSuccess) ? gn_launch<T>(x, gamma, beta, y, rows, C, groups, eps, scratch,
                                              stream)
                               : VI_ERR_CUDA;
-  if (cudaFreeAsync(scratch, stream) != cudaSuccess && st == VI_OK) st = VI_ERR_CUDA;
+  if (scratch_free(scratch, stream) != cudaSuccess && st == VI_OK) st = VI_ERR_CUDA;
   return st;
 }
 
@@ -525,7 +525,7 @@ template int groupnorm_global<bf16>(const bf16*, const bf16*, const bf16*, bf16*
 // Some callers cannot allocate device memory while they run: a plugin inside
 // an inference engine that owns all device memory and forbids allocation in
 // its execution step, or a service whose memory footprint is fixed when it
-// starts.  vi_groupnorm_global takes its scratch from cudaMallocAsync, so
+// starts.  vi_groupnorm_global takes its scratch from a stream-ordered pool, so
 // those callers cannot use it.  vi_groupnorm_global_noalloc runs the same two
 // kernels with its scratch in the file-scope array below instead; the caller
 // still provides every input and output.

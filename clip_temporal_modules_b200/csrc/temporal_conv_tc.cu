@@ -447,7 +447,7 @@ int temporal_conv_bf16_tc(const bf16* x, const bf16* w, const bf16* b, bf16* y, 
   }
   const size_t wbytes = (size_t)C * C * k * sizeof(bf16);
   void* wpk = nullptr;
-  VI_CUDA_TRY(cudaMallocAsync(&wpk, wbytes, stream));
+  VI_CUDA_TRY(scratch_alloc(&wpk, wbytes, stream));
   int st = VI_OK;
   {
     // Packed weights viewed as rows of 128 bytes; one box = one CTA's block.
@@ -470,7 +470,7 @@ int temporal_conv_bf16_tc(const bf16* x, const bf16* w, const bf16* b, bf16* y, 
     TcArgs a{b, y, err};
     st = pair ? tc_launch<true>(tmx, tmw, pl, a, stream) : tc_launch<false>(tmx, tmw, pl, a, stream);
   }
-  if (cudaFreeAsync(wpk, stream) != cudaSuccess && st == VI_OK) st = VI_ERR_CUDA;
+  if (scratch_free(wpk, stream) != cudaSuccess && st == VI_OK) st = VI_ERR_CUDA;
   return st;
 }
 

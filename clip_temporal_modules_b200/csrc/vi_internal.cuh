@@ -68,6 +68,12 @@ inline bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
 
 int sm_count();   // multiprocessors of the current device (cached per device)
 
+// Stream-ordered scratch from the library's own memory pool on the current
+// device (created on first use; it keeps freed memory mapped for reuse, so a
+// call after a synchronisation does not pay to map pages again).
+cudaError_t scratch_alloc(void** p, size_t bytes, cudaStream_t stream);
+cudaError_t scratch_free(void* p, cudaStream_t stream);
+
 // Count one kernel launch (backs vi_launch_count).
 void note_launch(int n = 1);
 

@@ -27,9 +27,11 @@
  * Streams.  `stream` is a cudaStream_t (NULL = the legacy default stream).
  *   Calls enqueue work on it and return without synchronising; the outputs
  *   are ready when the stream reaches that point.  Scratch memory the library
- *   needs is taken from the stream-ordered allocator on that stream and given
- *   back on it (cudaMallocAsync / cudaFreeAsync).  Calls on different streams
- *   may run concurrently; calls on one stream run in order.
+ *   needs is taken, in stream order on that stream, from a memory pool the
+ *   library creates for each device on first use (cudaMallocFromPoolAsync /
+ *   cudaFreeAsync); the pool keeps up to 64 MiB of freed memory mapped so
+ *   later calls reuse it.  Calls on different streams may run concurrently;
+ *   calls on one stream run in order.
  * Errors.  Every argument is checked on the host before anything is launched;
  *   a failed check returns a negative vi_status and enqueues nothing.
  *   VI_ERR_CUDA reports a CUDA error seen while launching.  A fault that
@@ -119,7 +121,8 @@ int vi_dual_attn_f32(const void* q, const void* k, const void* v, void* out, int
  * Requirements : sizes > 0; F % N == 0; k odd; k/2 <= L; y must not overlap
  *                x, w or b.  Otherwise VI_ERR_INVALID_ARG.
  * Scratch      : the bf16 path repacks w into a stream-ordered scratch buffer
- *                of k*C*C*2 bytes, freed on the stream after the kernel.
+ *                of k*C*C*2 bytes (library pool), freed on the stream after
+ *                the kernel.
  */
 int vi_temporal_conv(const void* x, const void* w, const void* b, void* y, int F, int N, int P,
                      int C, int k, vi_stream_t stream);
@@ -140,8 +143,9 @@ int vi_temporal_conv_f32(const void* x, const void* w, const void* b, void* y, i
  * Requirements : sizes > 0; F % N == 0; C % groups == 0; eps >= 0 and finite.
  *                y may alias x exactly but must not partly overlap it.
  * Scratch      : (24 * groups * blocks + 16*C + 16*groups + 64) bytes of stream-ordered
- *                scratch for per-block partial sums and the per-channel
- *                coefficients, freed on the stream after the last kernel.
+ *                scratch (library pool) for per-block partial sums and the
+ *                per-channel coefficients, freed on the stream after the last
+ *                kernel.
  */
 int vi_groupnorm_global(const void* x, const void* gamma, const void* beta, void* y, int F, int N,
                         int P, int C, int groups, float eps, vi_stream_t stream);
@@ -156,7 +160,7 @@ int vi_groupnorm_global_f32(const void* x, const void* gamma, const void* beta, 
  * inside an inference engine that owns all device memory and forbids
  * allocation in its execution step, or a service whose memory footprint is
  * fixed when it starts -- and therefore cannot use vi_groupnorm_global, which
- * takes its scratch from cudaMallocAsync.  The caller still provides every
+ * takes its scratch from a stream-ordered allocator.  The caller still provides every
  * input and output.
  *
  * Arguments, layout, result and argument checks: as vi_groupnorm_global.
