@@ -325,6 +325,9 @@ def run_ours(args):
         "clocks": clocks.summary(),
     }
 
+    result["attn_ablations"] = attn_ablations(w, d, out, stream)
+    result["groupnorm_conv_fused"] = fused_gn_conv(w, d, y, z, stream)
+
     if not args.no_e2e:
         result["e2e"] = run_e2e(args, w, host, dev, stream)
 
@@ -334,6 +337,63 @@ def run_ours(args):
     if rank == 0:
         print(json.dumps(result), flush=True)
     cleanup()
+
+
+def attn_ablations(w, d, out, stream, reps=10):
+    """Dual attention under the write-up's ablation settings (timed after the
+    headline region): no global context, no local context, no exchange."""
+    import torch
+
+    import clip_temporal_modules_b200 as vi
+    S = w.P * w.F * w.C * w.elem_bytes
+    res = {}
+    for name, (a, b_, g) in {"full_8_8_16": (w.n_pre, w.n_post, w.n_global),
+                             "local_only_8_8_0": (8, 8, 0), "global_only_0_0_16": (0, 0, 16),
+                             "no_sync_0_0_0": (0, 0, 0)}.items():
+        for _ in range(2):
+            vi.dual_attn(d["q"], d["k"], d["v"], out, N=w.N, heads=w.heads, n_pre=a, n_post=b_,
+                         n_global=g)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            vi.dual_attn(d["q"], d["k"], d["v"], out, N=w.N, heads=w.heads, n_pre=a, n_post=b_,
+                         n_global=g)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / reps
+        res[name] = {"ms": round(ms, 4), "GB/s": round(4 * S / (ms / 1e3) / 1e9, 1)}
+    return res
+
+
+def fused_gn_conv(w, d, y, z, stream, reps=10):
+    """GroupNorm -> conv of one tensor: the fused call against the two calls
+    (timed after the headline region)."""
+    import torch
+
+    import clip_temporal_modules_b200 as vi
+
+    def two():
+        vi.groupnorm_global(d["gn_x"], d["gn_gamma"], d["gn_beta"], z, N=w.N, groups=w.groups,
+                            eps=w.eps)
+        vi.temporal_conv(z, d["conv_w"], d["conv_b"], y, N=w.N)
+
+    def fused():
+        vi.groupnorm_conv(d["gn_x"], d["gn_gamma"], d["gn_beta"], d["conv_w"], d["conv_b"], y,
+                          N=w.N, groups=w.groups, eps=w.eps)
+
+    res = {}
+    for name, fn in (("two_calls", two), ("fused", fused)):
+        for _ in range(2):
+            fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / reps
+        res[name] = {"ms": round(ms, 4), "tokens_per_s": round(w.tokens / (ms / 1e3), 1)}
+    return res
 
 
 def run_e2e(args, w, host, dev, stream):

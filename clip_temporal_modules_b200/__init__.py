@@ -9,11 +9,14 @@ kernel grid:
                     context + uniformly sampled global frames)
   temporal_conv     temporal conv1d with neighbour padding, zeros at the ends
   groupnorm_global  GroupNorm with statistics aggregated over every clip
+  groupnorm_conv    GroupNorm followed by the conv, fused (no normalised
+                    tensor in memory)
 
 Python here only marshals arguments; see _binding.py.
 """
-from ._binding import (LIB_PATH, ViError, dual_attn, groupnorm_global,  # noqa: F401
-                       launch_count, lib, take_device_errors, temporal_conv)
+from ._binding import (LIB_PATH, ViError, dual_attn, groupnorm_conv,  # noqa: F401
+                       groupnorm_global, launch_count, lib, take_device_errors,
+                       temporal_conv)
 
-__all__ = ["dual_attn", "temporal_conv", "groupnorm_global", "take_device_errors", "launch_count", "lib",
+__all__ = ["dual_attn", "temporal_conv", "groupnorm_global", "groupnorm_conv", "take_device_errors", "launch_count", "lib",
            "ViError", "LIB_PATH"]

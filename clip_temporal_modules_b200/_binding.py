@@ -28,6 +28,7 @@ SIGNATURES = {
     "vi_groupnorm_global": [_vp, _vp, _vp, _vp] + [_i] * 5 + [_f, _vp],
     "vi_groupnorm_global_f32": [_vp, _vp, _vp, _vp] + [_i] * 5 + [_f, _vp],
     "vi_groupnorm_global_noalloc": [_vp, _vp, _vp, _vp] + [_i] * 5 + [_f, _vp],
+    "vi_groupnorm_conv": [_vp] * 6 + [_i] * 5 + [_f, _i, _vp],
     "vi_version": [],
     "vi_take_device_errors": [],
 }
@@ -130,6 +131,20 @@ def groupnorm_global(x, gamma, beta, out=None, *, N: int, groups: int, eps: floa
     _check(name, getattr(lib(), name)(x.data_ptr(), gamma.data_ptr(), beta.data_ptr(),
                                       out.data_ptr(), F, N, P, C, groups, float(eps),
                                       _stream_ptr(stream)))
+    return out
+
+
+def groupnorm_conv(x, gamma, beta, w, b, out=None, *, N: int, groups: int, eps: float = 1e-5,
+                   stream=None):
+    """Fused GroupNorm (global statistics) -> temporal conv; bf16 CUDA tensors."""
+    import torch
+    if out is None:
+        out = torch.empty_like(x)
+    _dev(x, gamma, beta, w, b, out)
+    P, F, C = x.shape
+    _check("vi_groupnorm_conv", lib().vi_groupnorm_conv(
+        x.data_ptr(), gamma.data_ptr(), beta.data_ptr(), w.data_ptr(), b.data_ptr(),
+        out.data_ptr(), F, N, P, C, groups, float(eps), w.shape[2], _stream_ptr(stream)))
     return out
 
 

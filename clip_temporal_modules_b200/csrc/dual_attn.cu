@@ -194,10 +194,15 @@ __global__ void __launch_bounds__(256) dual_attn_bf16_mma(const __grid_constant_
     for (int ks = 0; ks < 4; ++ks)
       ldsm_x4(sw128(sQ, warp * 16 + (lane & 15), 2 * ks + (lane >> 4)), qa[ks][0], qa[ks][1],
               qa[ks][2], qa[ks][3]);
+    // Without global frames their K/V tiles are not loaded: the MMAs that
+    // would read them are skipped (their scores are masked below anyway, but
+    // stale shared memory must not reach the P.V product as 0 * NaN).
+    const bool has_global = n_global > 0;
     float s[6][4];
 #pragma unroll
     for (int nt = 0; nt < 6; ++nt) {
       s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+      if (nt >= 4 && !has_global) continue;
       const uint32_t region = nt < 4 ? sKW : sKG;
       const int row = nt < 4 ? warp * 16 + nt * 8 + (lane & 7) : (nt - 4) * 8 + (lane & 7);
 #pragma unroll
@@ -254,6 +259,7 @@ __global__ void __launch_bounds__(256) dual_attn_bf16_mma(const __grid_constant_
     for (int nd = 0; nd < 8; ++nd) o[nd][0] = o[nd][1] = o[nd][2] = o[nd][3] = 0.f;
 #pragma unroll
     for (int ks = 0; ks < 3; ++ks) {
+      if (ks == 2 && !has_global) continue;
       const uint32_t region = ks < 2 ? sVW : sVG;
       const int row = (ks < 2 ? warp * 16 + ks * 16 : 0) + (lane & 15);
 #pragma unroll

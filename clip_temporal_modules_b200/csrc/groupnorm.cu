@@ -498,6 +498,40 @@ static int gn_launch(const T* x, const T* gamma, const T* beta, T* y, int64_t ro
   return VI_OK;
 }
 
+// Statistics pass alone (for a consumer that applies the normalisation
+// itself, such as the fused GroupNorm -> conv): fills the per-channel
+// coefficients in `scratch` (whose ticket must read 0) and returns their
+// address, [C][4] floats (m_c, a_c, beta_c, 0).
+template <typename T>
+int gn_stats_launch(const T* x, const T* gamma, const T* beta, int64_t rows, int C, int groups,
+                    float eps, void* scratch, cudaStream_t stream, const float** coef) {
+  const GnPlan pl = gn_plan<T>(rows, C, groups);
+  const GnScratch s = gn_carve(scratch, groups, C);
+  const int cg = C / groups;
+  if (pl.ring) {
+    unsigned int* err = device_error_word();
+    if (!err) return VI_ERR_CUDA;
+    VI_CUDA_TRY(cudaFuncSetAttribute(gn_stats_ring<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)pl.smem));
+    gn_stats_ring<T><<<pl.blocks, pl.threads, pl.smem, stream>>>(x, pl.rg, cg, groups, s, gamma,
+                                                                 beta, eps, err);
+    VI_LAUNCHED();
+  } else {
+    gn_stats_scalar<T><<<dim3(groups, pl.parts), 256, 0, stream>>>(x, rows, C, cg, groups, s,
+                                                                  gamma, beta, eps);
+    VI_LAUNCHED();
+  }
+  *coef = s.coef;
+  return VI_OK;
+}
+
+size_t gn_scratch_size_bf16(int64_t rows, int C, int groups) {
+  return gn_scratch_bytes<bf16>(rows, C, groups);
+}
+
+template int gn_stats_launch<bf16>(const bf16*, const bf16*, const bf16*, int64_t, int, int, float,
+                                   void*, cudaStream_t, const float**);
+
 template <typename T>
 int groupnorm_global(const T* x, const T* gamma, const T* beta, T* y, int64_t rows, int C,
                      int groups, float eps, cudaStream_t stream) {

@@ -49,10 +49,10 @@ namespace vi {
 
 constexpr int TC_M = 128;        // frames per tile = TMEM lanes per CTA
 constexpr int TC_KB = 64;        // input channels per K-block
-constexpr int TC_SA = 2;         // A (x) stages
+constexpr int TC_SA_MAX = 6;     // A (x) stages at most
 constexpr int TC_SB_MAX = 8;     // B (w) stages at most
 constexpr int TC_NJ_MAX = 160;   // a B stage holds all k taps of one K-block
-constexpr int TC_THREADS = 192;
+constexpr int TC_THREADS = 192;          // + 128 transform threads with NORM
 constexpr int TC_TMEM_COLS = 512;
 constexpr int TC_SMEM_LIMIT = 232448;   // 227 KB opt-in per CTA
 
@@ -79,29 +79,47 @@ struct TcPlan {
   int b_rows;            // weight rows per CTA per tap = NJ / H
   int b_tap;             // bytes of one tap's block = b_rows * 128
   int b_stage;           // bytes per B stage = k * b_tap (one K-block, all taps)
+  int sa;                // A stages
   int sb;                // B stages
   int smem;              // dynamic shared memory bytes
 };
 
 struct TcArgs {
+  const float* coef;     // NORM: per-channel (m_c, a_c, beta_c, 0) of the GroupNorm
   const bf16* bias;
   bf16* y;
   unsigned int* err;
 };
 
-static bool tc_plan(int F, int P, int C, int k, bool pair, TcPlan& pl) {
+// Ring depths (measured on B200 at F = 1024): with C <= 640 three x stages
+// and two weight stages beat two and three (1.48 vs 1.53 ms at C = 320); at
+// C = 1280 two x stages and as many weight stages as fit are best.  With the
+// GroupNorm transform, three x stages.  sb_pref / sa_pref override (0 = default).
+static int g_tc_sb_pref = 0, g_tc_sa_pref = 0;
+
+static bool tc_plan(int F, int P, int C, int k, bool pair, TcPlan& pl, bool norm = false) {
   if (k < 1 || k % 2 == 0 || 127 + k > 256 || C % TC_KB != 0) return false;
   const int H = pair ? 2 : 1;
   const int a_rows = 127 + k;
   const int a_stage = ((a_rows * 128 + 1023) / 1024) * 1024;
-  const int fixed = 1024 /* align slack */ + TC_SA * a_stage + 4 * C /* bias */ + 512 /* bars */;
+  const int fixed = 1024 /* align slack */ + 4 * C + 64 /* bias, padded */ + 512 /* bars */ +
+                    (norm ? 16 * C : 0) /* GroupNorm coefficients */;
   // Widest slab (<= 160 output channels, a multiple of 32 dividing C) whose
-  // all-tap weight stage still leaves room for two stages.
+  // all-tap weight stages leave room for at least two of each ring.
   for (int nj = TC_NJ_MAX; nj >= 32; nj -= 32) {
     if (C % nj != 0 || (nj / H) % 8 != 0) continue;
     const int b_stage = k * (nj / H) * 128;
-    int sb = (TC_SMEM_LIMIT - fixed) / b_stage;
-    if (sb > TC_SB_MAX) sb = TC_SB_MAX;
+    const bool few_k = C <= 640 || norm;
+    int sa = g_tc_sa_pref > 0 ? g_tc_sa_pref : (few_k ? 3 : 2);
+    if (sa > TC_SA_MAX) sa = TC_SA_MAX;
+    int sb = g_tc_sb_pref > 0 ? g_tc_sb_pref : (few_k ? 2 : TC_SB_MAX);
+    const int sb_fit = (TC_SMEM_LIMIT - fixed - sa * a_stage) / b_stage;
+    if (sb > sb_fit) sb = sb_fit;
+    if (sb < 2) {            // not enough room: fall back to the minimum x ring
+      sa = 2;
+      sb = (TC_SMEM_LIMIT - fixed - sa * a_stage) / b_stage;
+      if (sb > TC_SB_MAX) sb = TC_SB_MAX;
+    }
     if (sb < 2) continue;
     pl.F = F; pl.P = P; pl.C = C; pl.k = k;
     pl.NJ = nj;
@@ -116,29 +134,32 @@ static bool tc_plan(int F, int P, int C, int k, bool pair, TcPlan& pl) {
     pl.b_rows = nj / H;
     pl.b_tap = pl.b_rows * 128;
     pl.b_stage = b_stage;
+    pl.sa = sa;
     pl.sb = sb;
-    pl.smem = fixed + sb * b_stage;
+    pl.smem = fixed + sa * a_stage + sb * b_stage;
     return pl.smem <= TC_SMEM_LIMIT;
   }
   return false;
 }
 
-template <bool PAIR>
-__global__ void __launch_bounds__(TC_THREADS, 1)
+template <bool PAIR, bool NORM>
+__global__ void __launch_bounds__(TC_THREADS + (NORM ? 128 : 0), 1)
     temporal_conv_tc_kernel(const __grid_constant__ CUtensorMap tmx,
                             const __grid_constant__ CUtensorMap tmw, const TcPlan pl,
                             const TcArgs args) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
   const uint32_t sA = base;
-  const uint32_t sB = sA + TC_SA * pl.a_stage;
+  const uint32_t sB = sA + pl.sa * pl.a_stage;
   const uint32_t sBias = sB + pl.sb * pl.b_stage;
   const uint32_t sBar = sBias + ((4 * pl.C + 63) / 64) * 64;
   // barrier block: a_full[SA] a_empty[SA] b_full[SB] b_empty[SB] acc_full[2] acc_empty[2] drain tmem_slot
-  const uint32_t a_full = sBar, a_empty = a_full + 8 * TC_SA;
-  const uint32_t b_full = a_empty + 8 * TC_SA, b_empty = b_full + 8 * TC_SB_MAX;
+  const uint32_t a_full = sBar, a_empty = a_full + 8 * TC_SA_MAX;
+  const uint32_t b_full = a_empty + 8 * TC_SA_MAX, b_empty = b_full + 8 * TC_SB_MAX;
   const uint32_t acc_full = b_empty + 8 * TC_SB_MAX, acc_empty = acc_full + 16;
   const uint32_t drain = acc_empty + 16, tmem_slot = drain + 8;
+  const uint32_t a_ready = tmem_slot + 8;      // NORM: x stage normalised [SA]
+  const uint32_t sCoef = sBar + 512;           // NORM: float4 per channel
   float* bias_s = reinterpret_cast<float*>(smem_raw + (sBias - smem_u32(smem_raw)));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -152,16 +173,23 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   const uint32_t lead_acc_empty = PAIR ? mapa_shared(acc_empty, 0) : acc_empty;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < TC_SA; ++i) { mbar_init(a_full + 8 * i, PAIR ? 2 : 1); mbar_init(a_empty + 8 * i, 1); }
+    for (int i = 0; i < pl.sa; ++i) { mbar_init(a_full + 8 * i, PAIR ? 2 : 1); mbar_init(a_empty + 8 * i, 1); }
     for (int i = 0; i < pl.sb; ++i) { mbar_init(b_full + 8 * i, PAIR ? 2 : 1); mbar_init(b_empty + 8 * i, 1); }
     for (int i = 0; i < 2; ++i) {
       mbar_init(acc_full + 8 * i, 1);
       mbar_init(acc_empty + 8 * i, PAIR ? 8 : 4);
     }
     mbar_init(drain, 1);
+    if (NORM)
+      for (int i = 0; i < pl.sa; ++i) mbar_init(a_ready + 8 * i, 4);
     fence_barrier_init();
   }
   for (int c = threadIdx.x; c < pl.C; c += blockDim.x) bias_s[c] = to_f32(args.bias[c]);
+  if constexpr (NORM) {
+    float4* coef_s = reinterpret_cast<float4*>(smem_raw + (sCoef - smem_u32(smem_raw)));
+    for (int c = threadIdx.x; c < pl.C; c += blockDim.x)
+      coef_s[c] = reinterpret_cast<const float4*>(args.coef)[c];
+  }
   if (warp == 1) {
     if constexpr (PAIR) {
       tmem_alloc_pair(tmem_slot, TC_TMEM_COLS);
@@ -207,7 +235,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             mbar_arrive_expect_tx(a_full + 8 * sa, (uint32_t)pl.a_rows * 128u);
             tma_load_3d(dst, &tmx, cb * TC_KB, f0 - halo, p, a_full + 8 * sa);
           }
-          if (++sa == TC_SA) { sa = 0; pa ^= 1; a_used = true; }
+          if (++sa == pl.sa) { sa = 0; pa ^= 1; a_used = true; }
           // One B stage = this CTA's weight blocks of every tap of K-block cb.
           if (b_used && !tc_wait<PAIR>(b_empty + 8 * sbi, (uint32_t)(pb ^ 1), args.err,
                                        VI_DEV_ERR_TMA_TIMEOUT)) { ok = false; break; }
@@ -245,7 +273,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         const uint32_t d_tmem = tmem_base + (uint32_t)(buf * pl.NJ);
         uint32_t acc = 0u;
         for (int ib = 0; ib < pl.n_cb && ok; ++ib) {
-          if (!tc_wait<PAIR>(a_full + 8 * sa, (uint32_t)pa, args.err, VI_DEV_ERR_TMA_TIMEOUT) ||
+          if (!tc_wait<PAIR>((NORM ? a_ready : a_full) + 8 * sa, (uint32_t)pa, args.err,
+                             VI_DEV_ERR_TMA_TIMEOUT) ||
               !tc_wait<PAIR>(b_full + 8 * sbi, (uint32_t)pb, args.err, VI_DEV_ERR_TMA_TIMEOUT)) {
             ok = false;
             break;
@@ -281,7 +310,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             umma_commit(a_empty + 8 * sa);        // frees the x stage
           }
           if (++sbi == pl.sb) { sbi = 0; pb ^= 1; }
-          if (++sa == TC_SA) { sa = 0; pa ^= 1; }
+          if (++sa == pl.sa) { sa = 0; pa ^= 1; }
         }
         if constexpr (PAIR) umma_commit_pair_mc(acc_full + 8 * buf, 0x3);
         else umma_commit(acc_full + 8 * buf);         // accumulator ready for the epilogue
@@ -291,6 +320,55 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       if constexpr (PAIR) umma_commit_pair_mc(drain, 0x3);
       else umma_commit(drain);
       tc_wait<PAIR>(drain, 0, args.err, VI_DEV_ERR_MMA_TIMEOUT);
+    }
+  } else if (warp >= 6) {
+    // ------------------------------------------------------------ transform (NORM)
+    // Normalise each landed x stage in place, x -> (x - m_c) a_c + beta_c,
+    // then hand it to the MMA.  Rows outside [0, F) stay zero: the conv pads
+    // the normalised sequence with zeros.  128B swizzle: the 16-byte chunk of
+    // channels [8c, 8c+8) of row r sits at chunk c ^ (r mod 8).
+    if constexpr (NORM) {
+      const float4* coef_s = reinterpret_cast<const float4*>(smem_raw + (sCoef - smem_u32(smem_raw)));
+      uint4* stage0 = reinterpret_cast<uint4*>(smem_raw + (sA - smem_u32(smem_raw)));
+      // Thread tt always handles physical chunk pc of rows r0, r0+16, ...; all
+      // those rows share r mod 8, so the logical chunk (its 8 channels) is fixed.
+      const int tt = threadIdx.x - TC_THREADS;
+      const int pc = tt & 7, r0 = tt >> 3;
+      const int c = pc ^ (r0 & 7);
+      int sa = 0, pa = 0;
+      bool ok = true;
+      for (long long job = cluster_id; job < pl.n_jobs && ok; job += n_clusters) {
+        const long long tile = (job / pl.n_slabs) * pl.H + rank;
+        const int fb = (int)(tile % pl.n_fblk);
+        const int f_first = fb * TC_M - halo;
+        for (int ib = 0; ib < pl.n_cb && ok; ++ib) {
+          const int cb = (ib + cb_rot) % pl.n_cb;
+          float m[8], a[8], bt[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float4 k4 = coef_s[cb * TC_KB + c * 8 + e];
+            m[e] = k4.x; a[e] = k4.y; bt[e] = k4.z;
+          }
+          if (!mbar_wait_bounded(a_full + 8 * sa, (uint32_t)pa, args.err, VI_DEV_ERR_TMA_TIMEOUT)) {
+            ok = false;
+            break;
+          }
+          uint4* st = stage0 + (size_t)sa * (pl.a_stage / 16);
+          for (int r = r0; r < pl.a_rows; r += 16) {
+            const int f = f_first + r;
+            if (f < 0 || f >= pl.F) continue;
+            float v[8];
+            unpack(st[r * 8 + pc], v);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v[e] = fmaf(v[e] - m[e], a[e], bt[e]);
+            st[r * 8 + pc] = pack(v);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(a_ready + 8 * sa);
+          if (++sa == pl.sa) { sa = 0; pa ^= 1; }
+        }
+      }
     }
   } else {
     // ------------------------------------------------------------ epilogue
@@ -380,7 +458,12 @@ bool temporal_conv_tc_ok(int F, int P, int C, int k) {
   return F > 0 && P > 0 && tc_plan(F, P, C, k, TC_USE_PAIR, pl);
 }
 
-template <bool PAIR>
+bool temporal_conv_tc_norm_ok(int F, int P, int C, int k) {
+  TcPlan pl;
+  return F > 0 && P > 0 && tc_plan(F, P, C, k, false, pl, true);
+}
+
+template <bool PAIR, bool NORM>
 static int tc_launch(const CUtensorMap& tmx, const CUtensorMap& tmw, const TcPlan& pl,
                      const TcArgs& a, cudaStream_t stream) {
   static std::mutex mu;
@@ -390,7 +473,7 @@ static int tc_launch(const CUtensorMap& tmx, const CUtensorMap& tmw, const TcPla
   {
     std::lock_guard<std::mutex> lock(mu);
     if (dev < 64 && !attr_done[dev]) {
-      VI_CUDA_TRY(cudaFuncSetAttribute(temporal_conv_tc_kernel<PAIR>,
+      VI_CUDA_TRY(cudaFuncSetAttribute(temporal_conv_tc_kernel<PAIR, NORM>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        TC_SMEM_LIMIT));
       attr_done[dev] = true;
@@ -398,7 +481,7 @@ static int tc_launch(const CUtensorMap& tmx, const CUtensorMap& tmw, const TcPla
   }
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
-  cfg.blockDim = dim3(TC_THREADS);
+  cfg.blockDim = dim3(TC_THREADS + (NORM ? 128 : 0));
   cfg.dynamicSmemBytes = (size_t)pl.smem;
   cfg.stream = stream;
   long long grid;
@@ -411,7 +494,7 @@ static int tc_launch(const CUtensorMap& tmx, const CUtensorMap& tmw, const TcPla
     cfg.numAttrs = 1;
     cfg.gridDim = dim3(2 * sm_count());
     int clusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&clusters, temporal_conv_tc_kernel<PAIR>, &cfg) !=
+    if (cudaOccupancyMaxActiveClusters(&clusters, temporal_conv_tc_kernel<PAIR, NORM>, &cfg) !=
             cudaSuccess ||
         clusters < 1)
       clusters = sm_count() / 2;
@@ -423,16 +506,19 @@ static int tc_launch(const CUtensorMap& tmx, const CUtensorMap& tmw, const TcPla
     if (grid > pl.n_jobs) grid = pl.n_jobs;
   }
   cfg.gridDim = dim3((unsigned)grid);
-  VI_CUDA_TRY(cudaLaunchKernelEx(&cfg, temporal_conv_tc_kernel<PAIR>, tmx, tmw, pl, a));
+  VI_CUDA_TRY(cudaLaunchKernelEx(&cfg, temporal_conv_tc_kernel<PAIR, NORM>, tmx, tmw, pl, a));
   note_launch();
   return VI_OK;
 }
 
+// coef != nullptr: normalise x on the fly with the GroupNorm coefficients
+// (m_c, a_c, beta_c) before the contraction (fused GroupNorm -> conv).
 int temporal_conv_bf16_tc(const bf16* x, const bf16* w, const bf16* b, bf16* y, int F, int P,
-                          int C, int k, cudaStream_t stream) {
+                          int C, int k, cudaStream_t stream, const float* coef) {
   TcPlan pl;
-  const bool pair = TC_USE_PAIR && tc_plan(F, P, C, k, true, pl);
-  if (!pair && !tc_plan(F, P, C, k, false, pl)) return VI_ERR_UNSUPPORTED;
+  const bool norm = coef != nullptr;
+  const bool pair = !norm && TC_USE_PAIR && tc_plan(F, P, C, k, true, pl);
+  if (!pair && !tc_plan(F, P, C, k, false, pl, norm)) return VI_ERR_UNSUPPORTED;
   unsigned int* err = device_error_word();
   if (!err) return VI_ERR_CUDA;
   // x as [P][F][C]: box of 64 channels x a_rows frames x 1 position, 128B swizzle.
@@ -467,8 +553,10 @@ int temporal_conv_bf16_tc(const bf16* x, const bf16* w, const bf16* b, bf16* y, 
     if (cudaGetLastError() != cudaSuccess) st = VI_ERR_CUDA; else note_launch();
   }
   if (st == VI_OK) {
-    TcArgs a{b, y, err};
-    st = pair ? tc_launch<true>(tmx, tmw, pl, a, stream) : tc_launch<false>(tmx, tmw, pl, a, stream);
+    TcArgs a{coef, b, y, err};
+    st = norm ? tc_launch<false, true>(tmx, tmw, pl, a, stream)
+              : pair ? tc_launch<true, false>(tmx, tmw, pl, a, stream)
+                     : tc_launch<false, false>(tmx, tmw, pl, a, stream);
   }
   if (scratch_free(wpk, stream) != cudaSuccess && st == VI_OK) st = VI_ERR_CUDA;
   return st;

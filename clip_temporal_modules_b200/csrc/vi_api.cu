@@ -33,8 +33,13 @@ template <typename T>
 int temporal_conv_generic_launch(const T*, const T*, const T*, T*, int, int, int, int,
                                  cudaStream_t);
 int temporal_conv_bf16_tc(const bf16*, const bf16*, const bf16*, bf16*, int, int, int, int,
-                          cudaStream_t);
+                          cudaStream_t, const float* coef = nullptr);
 bool temporal_conv_tc_ok(int F, int P, int C, int k);
+bool temporal_conv_tc_norm_ok(int F, int P, int C, int k);
+template <typename T>
+int gn_stats_launch(const T*, const T*, const T*, int64_t, int, int, float, void*, cudaStream_t,
+                    const float**);
+size_t gn_scratch_size_bf16(int64_t rows, int C, int groups);
 template <typename T>
 int groupnorm_global(const T*, const T*, const T*, T*, int64_t, int, int, float, cudaStream_t);
 
@@ -210,6 +215,43 @@ int gn_entry(const void* x, const void* gamma, const void* beta, void* y, int F,
                              groups, eps, as_stream(stream));
 }
 
+int gn_conv_entry(const void* x, const void* gamma, const void* beta, const void* w,
+                  const void* b, void* y, int F, int N, int P, int C, int groups, float eps, int k,
+                  vi_stream_t stream) {
+  using T = bf16;
+  if (!x || !gamma || !beta || !w || !b || !y) return VI_ERR_INVALID_ARG;
+  int st = check_clips(F, N, P, C);
+  if (st != VI_OK) return st;
+  if (groups <= 0 || C % groups != 0) return VI_ERR_INVALID_ARG;
+  if (!(eps >= 0.f) || !isfinite(eps)) return VI_ERR_INVALID_ARG;
+  if (k <= 0 || k % 2 == 0 || k / 2 > F / N) return VI_ERR_INVALID_ARG;
+  if (groups > 1024) return VI_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(gamma) || !aligned16(beta) || !aligned16(w) || !aligned16(b) ||
+      !aligned16(y))
+    return VI_ERR_ALIGNMENT;
+  if ((C * sizeof(T)) % 16 != 0) return VI_ERR_ALIGNMENT;
+  const size_t bytes = (size_t)P * F * C * sizeof(T);
+  const size_t wbytes = (size_t)C * C * k * sizeof(T), cbytes = (size_t)C * sizeof(T);
+  if (overlaps(y, bytes, x, bytes) || overlaps(y, bytes, w, wbytes) || overlaps(y, bytes, b, cbytes) ||
+      overlaps(y, bytes, gamma, cbytes) || overlaps(y, bytes, beta, cbytes))
+    return VI_ERR_INVALID_ARG;
+  if (!temporal_conv_tc_norm_ok(F, P, C, k)) return VI_ERR_UNSUPPORTED;
+  cudaStream_t s = as_stream(stream);
+  const int64_t rows = (int64_t)P * F;
+  void* scratch = nullptr;
+  VI_CUDA_TRY(scratch_alloc(&scratch, gn_scratch_size_bf16(rows, C, groups), s));
+  const float* coef = nullptr;
+  st = cudaMemsetAsync(scratch, 0, 64, s) == cudaSuccess ? VI_OK : VI_ERR_CUDA;
+  if (st == VI_OK)
+    st = gn_stats_launch<T>(static_cast<const T*>(x), static_cast<const T*>(gamma),
+                            static_cast<const T*>(beta), rows, C, groups, eps, scratch, s, &coef);
+  if (st == VI_OK)
+    st = temporal_conv_bf16_tc(static_cast<const T*>(x), static_cast<const T*>(w),
+                               static_cast<const T*>(b), static_cast<T*>(y), F, P, C, k, s, coef);
+  if (scratch_free(scratch, s) != cudaSuccess && st == VI_OK) st = VI_ERR_CUDA;
+  return st;
+}
+
 }  // namespace
 
 extern "C" {
@@ -255,6 +297,11 @@ int vi_temporal_conv(const void* x, const void* w, const void* b, void* y, int F
 int vi_temporal_conv_f32(const void* x, const void* w, const void* b, void* y, int F, int N,
                          int P, int C, int k, vi_stream_t stream) {
   return conv_entry<float>(x, w, b, y, F, N, P, C, k, stream);
+}
+int vi_groupnorm_conv(const void* x, const void* gamma, const void* beta, const void* w,
+                      const void* b, void* y, int F, int N, int P, int C, int groups, float eps,
+                      int k, vi_stream_t stream) {
+  return gn_conv_entry(x, gamma, beta, w, b, y, F, N, P, C, groups, eps, k, stream);
 }
 int vi_groupnorm_global(const void* x, const void* gamma, const void* beta, void* y, int F, int N,
                         int P, int C, int groups, float eps, vi_stream_t stream) {

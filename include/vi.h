@@ -153,6 +153,26 @@ int vi_groupnorm_global_f32(const void* x, const void* gamma, const void* beta, 
                             int N, int P, int C, int groups, float eps, vi_stream_t stream);
 
 /*
+ * GroupNorm with global statistics followed by the temporal convolution,
+ * fused (bf16).  The ResNet module of the write-up normalises and then
+ * convolves along frames (GroupNorm-module and conv-module paragraphs);
+ *   y = vi_temporal_conv(vi_groupnorm_global(x; gamma, beta, groups, eps); w, b)
+ * computed without writing the normalised tensor to memory: one statistics
+ * pass over x, then the conv kernel normalises each staged x tile in shared
+ * memory (bf16, round to nearest even) before the tensor-core contraction.
+ * The zero padding at the video ends applies to the NORMALISED sequence.
+ *
+ * x, y : [P][F][C];  gamma, beta, b : [C];  w : [C][C][k].
+ * Requirements : those of vi_groupnorm_global and vi_temporal_conv; y must
+ *                not overlap any input; the fused kernel also needs
+ *                C % 64 == 0 (VI_ERR_UNSUPPORTED otherwise).
+ * Scratch      : GroupNorm statistics and repacked w (library pool).
+ */
+int vi_groupnorm_conv(const void* x, const void* gamma, const void* beta, const void* w,
+                      const void* b, void* y, int F, int N, int P, int C, int groups, float eps,
+                      int k, vi_stream_t stream);
+
+/*
  * GroupNorm with global statistics that allocates nothing (bf16 only).
  *
  * The source paper has no counterpart to this entry point.  It is for callers

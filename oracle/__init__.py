@@ -32,7 +32,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
 
-DTYPE_CODE = {"f32": 0, "bf16": 1}
+DTYPE_CODE = {"f32": 0, "bf16": 1, "f64": 2}
 
 
 def build(force: bool = False) -> str:
@@ -57,7 +57,7 @@ def lib():
         L.oracle_dual_attn.restype = None
         L.oracle_dual_attn.argtypes = [vp, vp, vp, i32, vp] + [i32] * 8 + [vp, i32, i32]
         L.oracle_temporal_conv.restype = None
-        L.oracle_temporal_conv.argtypes = [vp, vp, vp, i32, vp] + [i32] * 5 + [vp, i32, i32]
+        L.oracle_temporal_conv.argtypes = [vp, vp, vp, i32, vp] + [i32] * 5 + [vp, i32, i32, i32]
         L.oracle_groupnorm_global.restype = None
         L.oracle_groupnorm_global.argtypes = ([vp, vp, vp, i32, vp, vp, vp] + [i32] * 5 +
                                               [dbl, vp, i32, i32])
@@ -70,11 +70,13 @@ def max_threads() -> int:
     return int(lib().oracle_max_threads())
 
 
-def _dtype_of(a: np.ndarray) -> str:
+def _dtype_of(a: np.ndarray, allow_f64: bool = False) -> str:
     if a.dtype == np.uint16:
         return "bf16"
     if a.dtype == np.float32:
         return "f32"
+    if allow_f64 and a.dtype == np.float64:
+        return "f64"
     raise TypeError(f"oracle inputs are float32 values or bf16 bits (uint16), got {a.dtype}")
 
 
@@ -128,10 +130,13 @@ def dual_attn(q, k, v, F, N, heads, d, n_pre=8, n_post=8, n_global=16, positions
 
 
 def temporal_conv(x, w, b, F, N, k=3, positions=None, nthreads=0) -> np.ndarray:
-    """Clip-padded temporal conv over [P][F][C] -> [n_pos][F][C] float64."""
+    """Clip-padded temporal conv over [P][F][C] -> [n_pos][F][C] float64.
+
+    x may also be float64 (the exact output of another oracle module)."""
     x, w, b = _c(x), _c(w), _c(b)
-    dt = _dtype_of(x)
-    assert _dtype_of(w) == dt and _dtype_of(b) == dt
+    xdt = _dtype_of(x, allow_f64=True)
+    dt = _dtype_of(w)
+    assert _dtype_of(b) == dt
     _check_common(F, N)
     C = b.size
     P = x.size // (F * C)
@@ -141,8 +146,33 @@ def temporal_conv(x, w, b, F, N, k=3, positions=None, nthreads=0) -> np.ndarray:
     pos = _positions(P, positions)
     y = np.zeros((pos.size, F, C), np.float64)
     lib().oracle_temporal_conv(x.ctypes.data, w.ctypes.data, b.ctypes.data, DTYPE_CODE[dt],
-                               y.ctypes.data, F, N, P, C, k, pos.ctypes.data, pos.size, nthreads)
+                               y.ctypes.data, F, N, P, C, k, pos.ctypes.data, pos.size, nthreads,
+                               DTYPE_CODE[xdt])
     return y
+
+
+def round_bf16(a: np.ndarray) -> np.ndarray:
+    """Values rounded to bf16 (via fp32, round to nearest even), as float64."""
+    f = np.ascontiguousarray(a, dtype=np.float32)
+    u = f.view(np.uint32).astype(np.uint64)
+    u = (u + 0x7FFF + ((u >> 16) & 1)) >> 16 << 16
+    return u.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+def groupnorm_conv(x, gamma, beta, w, b, F, N, groups, eps=1e-5, k=3, positions=None,
+                   nthreads=0, intermediate="f64") -> np.ndarray:
+    """Temporal conv of the global-statistics GroupNorm of x (the ResNet-module
+    order: normalise, then convolve along frames), composed from the two
+    modules above.  intermediate="f64" feeds the exact GroupNorm output to the
+    conv; "bf16" rounds it to bf16 first, as a pipeline whose modules exchange
+    bf16 tensors does.  -> [n_pos][F][C] float64."""
+    P = x.size // (F * gamma.size)
+    pos = _positions(P, positions)
+    z, _, _ = groupnorm_global(x, gamma, beta, F, N, groups, eps, positions=pos,
+                               nthreads=nthreads)
+    if intermediate == "bf16":
+        z = round_bf16(z)
+    return temporal_conv(z, w, b, F, N, k, nthreads=nthreads)
 
 
 def groupnorm_global(x, gamma, beta, F, N, groups, eps=1e-5, positions=None, nthreads=0,

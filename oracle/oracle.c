@@ -27,8 +27,11 @@
 #include <omp.h>
 #endif
 
-/* Exact widening of one input element to double. */
+/* Exact widening of one input element to double (dtype 0: fp32 values,
+   1: bf16 bit patterns, 2: doubles, used to feed one module's exact output
+   into the next). */
 static double in_val(const void* base, int64_t idx, int dtype) {
+  if (dtype == 2) return ((const double*)base)[idx];
   if (dtype == 0) return (double)((const float*)base)[idx];
   uint32_t u = (uint32_t)((const uint16_t*)base)[idx] << 16;
   float f;
@@ -148,11 +151,12 @@ void oracle_dual_attn(const void* q, const void* k, const void* v, int dtype, do
  * the clip's L output frames:
  *   y[p,f,co] = b[co] + sum_t sum_ci W[co,ci,t] * ext[f - s + t][ci]
  * where ext[u] holds frame s - n + u.  Requires odd k and n <= L.
- * w: [C_out][C_in][k]; b: [C]; y: [n_pos][F][C] doubles.
+ * w: [C_out][C_in][k] and b: [C] in `dtype`; x in `x_dtype`;
+ * y: [n_pos][F][C] doubles.
  */
 void oracle_temporal_conv(const void* x, const void* w, const void* b, int dtype, double* y,
                           int F, int N, int P, int C, int k, const int* pos, int n_pos,
-                          int nthreads) {
+                          int nthreads, int x_dtype) {
   (void)P;
   set_threads(nthreads);
   const int L = F / N, n = k / 2, E = L + 2 * n;
@@ -171,7 +175,7 @@ void oracle_temporal_conv(const void* x, const void* w, const void* b, int dtype
         const int present = (from_prev && i > 0) || (from_next && i < N - 1) ||
                             (!from_prev && !from_next);
         for (int c = 0; c < C; ++c)
-          ext[(int64_t)u * C + c] = present ? in_val(x, pbase + (int64_t)f * C + c, dtype) : 0.0;
+          ext[(int64_t)u * C + c] = present ? in_val(x, pbase + (int64_t)f * C + c, x_dtype) : 0.0;
       }
       for (int fl = 0; fl < L; ++fl)
         for (int co = 0; co < C; ++co) {

@@ -119,3 +119,20 @@ def test_binding_signatures_cover_header():
     for n in declared_functions():
         if n not in ("vi_status_string", "vi_launch_count"):
             assert n in _binding.SIGNATURES, n
+
+
+E = 1 << 33
+G = 1 << 34
+
+
+def gnconv(L, x=A, g=B, bt=Cp, w=D, b=E, y=G, F=64, N=4, P=2, C=64, groups=8, eps=1e-5, k=3):
+    return L.vi_groupnorm_conv(x, g, bt, w, b, y, F, N, P, C, groups, eps, k, None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(w=0), INVALID), (dict(groups=7), INVALID), (dict(k=4), INVALID), (dict(F=66), INVALID),
+    (dict(eps=-1.0), INVALID), (dict(b=E + 8), ALIGN), (dict(y=A + 32), INVALID),
+    (dict(C=40, groups=8), UNSUP),            # no fused kernel for C % 64 != 0
+])
+def test_groupnorm_conv_rejects(L, kw, expect):
+    assert gnconv(L, **kw) == expect

@@ -61,6 +61,18 @@ def test_full_size_sampled_positions(cuda_device, w):
     run_case(w, positions=sample_positions(w.P))
 
 
+# Ablation settings of the write-up's study (attention without global context,
+# without local context, and with no context exchange at all) at full size.
+ABLATIONS = [dict(n_pre=8, n_post=8, n_global=0), dict(n_pre=0, n_post=0, n_global=16),
+             dict(n_pre=0, n_post=0, n_global=0)]
+
+
+@pytest.mark.parametrize("ctx", ABLATIONS, ids=["local_only", "global_only", "no_sync"])
+def test_ablation_settings_full_size(cuda_device, ctx):
+    w = synth.BY_NAME["bf16_F1024_P2560_C320"].with_(**ctx)
+    run_case(w, positions=sample_positions(w.P, count=2))
+
+
 def test_fp32_tiny_full_workload_all_positions(cuda_device):
     run_case(synth.WORKLOADS[0])
 
@@ -81,3 +93,24 @@ def test_runs_on_given_stream_and_leaves_neighbours_untouched(cuda_device):
     ref = vi.dual_attn(q, k, v, N=w.N, heads=w.heads)
     torch.cuda.synchronize()
     assert torch.equal(out, ref)
+
+
+def test_no_global_frames_ignores_stale_shared_memory(cuda_device):
+    """With n_global = 0 the global K/V tiles are not loaded; whatever an
+    earlier kernel left in that shared memory (here NaN) must not leak."""
+    w = W("bf16_poison", "bf16", 1024, 64, 64, 5)
+    nan = torch.full((w.P, w.F, w.C), float("nan"), dtype=torch.bfloat16, device="cuda")
+    vi.dual_attn(nan, nan, nan, torch.empty_like(nan), N=w.N, heads=w.heads)   # fills smem
+    torch.cuda.synchronize()
+    ctx = dict(n_pre=0, n_post=0, n_global=0)
+    q, k, v = (synth.make(w, t) for t in ("q", "k", "v"))
+    dq, dk, dv = (to_device(a, w.dtype) for a in (q, k, v))
+    for _ in range(3):
+        vi.dual_attn(nan, nan, nan, torch.empty_like(nan), N=w.N, heads=w.heads)
+        out = vi.dual_attn(dq, dk, dv, N=w.N, heads=w.heads, **ctx)
+        torch.cuda.synchronize()
+        got = from_device(out)
+        assert np.all(np.isfinite(got))
+    pos = [0, 17, 63]
+    ref = oracle.dual_attn(q, k, v, w.F, w.N, w.heads, w.d, positions=pos, **ctx)
+    assert_close(got[pos], ref, w.dtype, "attn", "no global after NaN")

@@ -105,3 +105,26 @@ def test_position_subset_equals_full_slice():
     full = oracle.temporal_conv(x, w, b, F, N)
     np.testing.assert_array_equal(oracle.temporal_conv(x, w, b, F, N, positions=[3, 0]),
                                   full[[3, 0]])
+
+
+def test_groupnorm_then_conv_equals_library_composition():
+    """GroupNorm (whole-tensor statistics) then conv1d, both from the library."""
+    F, N, P, C, G, k = 16, 4, 3, 16, 4, 3
+    x = synth.normal((P, F, C), 21, 0.5, 1.4, seed=7, dtype="f32")
+    gamma = synth.normal((C,), 22, 1.0, 0.3, seed=7, dtype="f32")
+    beta = synth.normal((C,), 23, 0.0, 0.3, seed=7, dtype="f32")
+    w, b = _rand((C, C, k), 24, std=0.3), _rand((C,), 25)
+    got = oracle.groupnorm_conv(x, gamma, beta, w, b, F, N, G, 1e-5, k)
+    xt = torch.from_numpy(x.astype(np.float64)).reshape(P * F, C).T.reshape(1, C, P * F)
+    z = torch.nn.functional.group_norm(xt, G, torch.from_numpy(gamma.astype(np.float64)),
+                                       torch.from_numpy(beta.astype(np.float64)), 1e-5)
+    z = z.reshape(C, P * F).T.reshape(P, F, C).numpy()
+    np.testing.assert_allclose(got, _torch_conv(z, w, b, k), rtol=0, atol=1e-12)
+    sub = oracle.groupnorm_conv(x, gamma, beta, w, b, F, N, G, 1e-5, k, positions=[2, 0])
+    np.testing.assert_array_equal(sub, got[[2, 0]])
+
+
+def test_round_bf16_is_nearest_even():
+    v = np.array([1.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, -2.5, 1.0 + 2 ** -8 + 2 ** -20])
+    np.testing.assert_array_equal(oracle.round_bf16(v), [1.0, 1.0, 1.0 + 2 ** -6, -2.5,
+                                                         1.0 + 2 ** -7])
