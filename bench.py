@@ -327,6 +327,7 @@ def run_ours(args):
 
     result["attn_ablations"] = attn_ablations(w, d, out, stream)
     result["groupnorm_conv_fused"] = fused_gn_conv(w, d, y, z, stream)
+    result["temporal_attention_module"] = attention_module(w, d, out, y, z, stream)
 
     if not args.no_e2e:
         result["e2e"] = run_e2e(args, w, host, dev, stream)
@@ -394,6 +395,39 @@ def fused_gn_conv(w, d, y, z, stream, reps=10):
         ms = e0.elapsed_time(e1) / reps
         res[name] = {"ms": round(ms, 4), "tokens_per_s": round(w.tokens / (ms / 1e3), 1)}
     return res
+
+
+def attention_module(w, d, out, y, z, stream, reps=5):
+    """Temporal attention module (q/k/v projections, dual attention, output
+    projection) on the workload's input, timed after the headline region."""
+    import torch
+
+    import clip_temporal_modules_b200 as vi
+    import synth
+    dev = out.device
+    mk = lambda t: torch.from_numpy(synth.make(w, t)).view(torch.bfloat16).to(dev)
+    wq, bq, wo, bo = (mk(t) for t in ("w_qkv", "b_qkv", "w_out", "b_out"))
+    n = int(vi.lib().vi_temporal_attention_workspace_bytes(w.F, w.P, w.C))
+    ws = torch.empty(n // 2, dtype=torch.bfloat16, device=dev)
+    x = d["conv_x"]
+
+    def run():
+        vi.temporal_attention(x, wq, bq, wo, bo, y, ws, N=w.N, heads=w.heads, n_pre=w.n_pre,
+                              n_post=w.n_post, n_global=w.n_global)
+
+    for _ in range(2):
+        run()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        run()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    del ws
+    flops = 4 * 2 * w.C * w.C * w.tokens
+    return {"ms": round(ms, 4), "tokens_per_s": round(w.tokens / (ms / 1e3), 1),
+            "projection_tflops_total": round(flops / 1e12, 3)}
 
 
 def run_e2e(args, w, host, dev, stream):

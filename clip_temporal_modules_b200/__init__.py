@@ -11,12 +11,13 @@ kernel grid:
   groupnorm_global  GroupNorm with statistics aggregated over every clip
   groupnorm_conv    GroupNorm followed by the conv, fused (no normalised
                     tensor in memory)
+  temporal_attention  q/k/v projections + dual_attn + output projection
 
 Python here only marshals arguments; see _binding.py.
 """
 from ._binding import (LIB_PATH, ViError, dual_attn, groupnorm_conv,  # noqa: F401
                        groupnorm_global, launch_count, lib, take_device_errors,
-                       temporal_conv)
+                       temporal_attention, temporal_conv)
 
-__all__ = ["dual_attn", "temporal_conv", "groupnorm_global", "groupnorm_conv", "take_device_errors", "launch_count", "lib",
+__all__ = ["dual_attn", "temporal_conv", "groupnorm_global", "groupnorm_conv", "temporal_attention", "take_device_errors", "launch_count", "lib",
            "ViError", "LIB_PATH"]

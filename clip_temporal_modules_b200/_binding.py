@@ -29,6 +29,7 @@ SIGNATURES = {
     "vi_groupnorm_global_f32": [_vp, _vp, _vp, _vp] + [_i] * 5 + [_f, _vp],
     "vi_groupnorm_global_noalloc": [_vp, _vp, _vp, _vp] + [_i] * 5 + [_f, _vp],
     "vi_groupnorm_conv": [_vp] * 6 + [_i] * 5 + [_f, _i, _vp],
+    "vi_temporal_attention": [_vp] * 7 + [_i] * 8 + [_vp],
     "vi_version": [],
     "vi_take_device_errors": [],
 }
@@ -54,6 +55,8 @@ def lib() -> ctypes.CDLL:
             fn = getattr(L, name)
             fn.argtypes = args
             fn.restype = ctypes.c_int
+        L.vi_temporal_attention_workspace_bytes.argtypes = [_i, _i, _i]
+        L.vi_temporal_attention_workspace_bytes.restype = ctypes.c_ulonglong
         L.vi_launch_count.argtypes = []
         L.vi_launch_count.restype = ctypes.c_ulonglong
         L.vi_status_string.argtypes = [ctypes.c_int]
@@ -145,6 +148,26 @@ def groupnorm_conv(x, gamma, beta, w, b, out=None, *, N: int, groups: int, eps: 
     _check("vi_groupnorm_conv", lib().vi_groupnorm_conv(
         x.data_ptr(), gamma.data_ptr(), beta.data_ptr(), w.data_ptr(), b.data_ptr(),
         out.data_ptr(), F, N, P, C, groups, float(eps), w.shape[2], _stream_ptr(stream)))
+    return out
+
+
+def temporal_attention(x, w_qkv, b_qkv, w_out, b_out, out=None, workspace=None, *, N: int,
+                       heads: int, n_pre: int = 8, n_post: int = 8, n_global: int = 16,
+                       stream=None):
+    """Projections + dual-domain attention + output projection; bf16 CUDA tensors.
+    w_qkv [3C][C], b_qkv [3C], w_out [C][C], b_out [C] (Linear layout)."""
+    import torch
+    P, F, C = x.shape
+    if out is None:
+        out = torch.empty_like(x)
+    if workspace is None:
+        n = int(lib().vi_temporal_attention_workspace_bytes(F, P, C))
+        workspace = torch.empty(n // 2, dtype=torch.bfloat16, device=x.device)
+    _dev(x, w_qkv, b_qkv, w_out, b_out, out, workspace)
+    _check("vi_temporal_attention", lib().vi_temporal_attention(
+        x.data_ptr(), w_qkv.data_ptr(), b_qkv.data_ptr(), w_out.data_ptr(), b_out.data_ptr(),
+        out.data_ptr(), workspace.data_ptr(), F, N, P, heads, C // heads, n_pre, n_post, n_global,
+        _stream_ptr(stream)))
     return out
 
 

@@ -252,9 +252,74 @@ int gn_conv_entry(const void* x, const void* gamma, const void* beta, const void
   return st;
 }
 
+int temporal_attention_entry(const void* x, const void* w_qkv, const void* b_qkv,
+                             const void* w_out, const void* b_out, void* out, void* workspace,
+                             int F, int N, int P, int heads, int d, int n_pre, int n_post,
+                             int n_global, vi_stream_t stream) {
+  using T = bf16;
+  if (!x || !w_qkv || !b_qkv || !w_out || !b_out || !out || !workspace) return VI_ERR_INVALID_ARG;
+  if (heads <= 0 || d <= 0 || (int64_t)heads * d > 0x7fffffff) return VI_ERR_INVALID_ARG;
+  const int C = heads * d;
+  int st = check_clips(F, N, P, C);
+  if (st != VI_OK) return st;
+  const int L = F / N;
+  if (n_pre < 0 || n_post < 0 || n_global < 0 || n_global > F) return VI_ERR_INVALID_ARG;
+  if (N > 1 && (n_pre > L || n_post > L)) return VI_ERR_INVALID_ARG;
+  if (d != 64) return VI_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(w_qkv) || !aligned16(b_qkv) || !aligned16(w_out) ||
+      !aligned16(b_out) || !aligned16(out) || !aligned16(workspace))
+    return VI_ERR_ALIGNMENT;
+  const size_t S = (size_t)P * F * C * sizeof(T);
+  const size_t ws = 4 * S, cc = (size_t)C * C * sizeof(T);
+  if (overlaps(out, S, x, S) || overlaps(out, S, workspace, ws) || overlaps(workspace, ws, x, S) ||
+      overlaps(out, S, w_qkv, 3 * cc) || overlaps(out, S, w_out, cc) ||
+      overlaps(workspace, ws, w_qkv, 3 * cc) || overlaps(workspace, ws, w_out, cc) ||
+      overlaps(out, S, b_qkv, 3 * C * sizeof(T)) || overlaps(out, S, b_out, C * sizeof(T)) ||
+      overlaps(workspace, ws, b_qkv, 3 * C * sizeof(T)) ||
+      overlaps(workspace, ws, b_out, C * sizeof(T)))
+    return VI_ERR_INVALID_ARG;
+  if (!temporal_conv_tc_ok(F, P, C, 1)) return VI_ERR_UNSUPPORTED;
+  cudaStream_t s = as_stream(stream);
+  const T* xx = static_cast<const T*>(x);
+  const T* wq = static_cast<const T*>(w_qkv);
+  const T* bq = static_cast<const T*>(b_qkv);
+  T* q = static_cast<T*>(workspace);
+  T* k = q + (size_t)P * F * C;
+  T* v = k + (size_t)P * F * C;
+  T* a = v + (size_t)P * F * C;
+  T* qkv[3] = {q, k, v};
+  for (int i = 0; i < 3 && st == VI_OK; ++i)   // single-tap conv = per-frame linear layer
+    st = temporal_conv_bf16_tc(xx, wq + (size_t)i * C * C, bq + (size_t)i * C, qkv[i], F, P, C, 1,
+                               s);
+  if (st == VI_OK) {
+    if (dual_attn_fast_ok(F, N, d, n_pre, n_post, n_global))
+      st = dual_attn_bf16_fast(q, k, v, a, F, N, P, heads, n_pre, n_post, n_global, s);
+    else
+      st = dual_attn_generic_launch<T>(q, k, v, a, F, N, P, heads, d, n_pre, n_post, n_global, s);
+  }
+  if (st == VI_OK)
+    st = temporal_conv_bf16_tc(a, static_cast<const T*>(w_out), static_cast<const T*>(b_out),
+                               static_cast<T*>(out), F, P, C, 1, s);
+  return st;
+}
+
 }  // namespace
 
 extern "C" {
+
+unsigned long long vi_temporal_attention_workspace_bytes(int F, int P, int C) {
+  if (F <= 0 || P <= 0 || C <= 0) return 0ull;
+  return 4ull * (unsigned long long)F * P * C * sizeof(bf16);
+}
+
+int vi_temporal_attention(const void* x, const void* w_qkv, const void* b_qkv, const void* w_out,
+                          const void* b_out, void* out, void* workspace, int F, int N, int P,
+                          int heads, int d, int n_pre, int n_post, int n_global,
+                          vi_stream_t stream) {
+  return temporal_attention_entry(x, w_qkv, b_qkv, w_out, b_out, out, workspace, F, N, P, heads,
+                                  d, n_pre, n_post, n_global, stream);
+}
+
 
 const char* vi_status_string(int status) {
   switch (status) {

@@ -153,6 +153,31 @@ int vi_groupnorm_global_f32(const void* x, const void* gamma, const void* beta, 
                             int N, int P, int C, int groups, float eps, vi_stream_t stream);
 
 /*
+ * Temporal attention module: input projections, dual-domain attention, output
+ * projection (bf16).  The attention-module paragraph redefines how the keys and
+ * values are gathered ("modifying the K-V computation"); the projections
+ * around it are the module's linear layers:
+ *   q = x Wq^T + bq,  k = x Wk^T + bk,  v = x Wv^T + bv      (per frame)
+ *   a = vi_dual_attn(q, k, v; heads, d, n_pre, n_post, n_global)
+ *   out = a Wo^T + bo
+ * Each stage is a separate kernel writing a bf16 tensor (the projections run
+ * on the tensor-core temporal-conv kernel with a single tap).
+ *
+ * x, out : [P][F][C], C = heads*d;  w_qkv : [3C][C] (rows Wq, Wk, Wv, PyTorch
+ * Linear layout);  b_qkv : [3C];  w_out : [C][C];  b_out : [C].
+ * workspace : device buffer of vi_temporal_attention_workspace_bytes(F, P, C)
+ *             bytes (16-byte aligned), owned by the caller, holding q, k, v
+ *             and a between the stages; contents undefined after the call.
+ * Requirements : those of vi_dual_attn; C % 64 == 0; out, x, weights and
+ *                workspace must not overlap.
+ */
+unsigned long long vi_temporal_attention_workspace_bytes(int F, int P, int C);
+int vi_temporal_attention(const void* x, const void* w_qkv, const void* b_qkv, const void* w_out,
+                          const void* b_out, void* out, void* workspace, int F, int N, int P,
+                          int heads, int d, int n_pre, int n_post, int n_global,
+                          vi_stream_t stream);
+
+/*
  * GroupNorm with global statistics followed by the temporal convolution,
  * fused (bf16).  The ResNet module of the write-up normalises and then
  * convolves along frames (GroupNorm-module and conv-module paragraphs);

@@ -108,10 +108,12 @@ def _check_common(F, N):
 
 def dual_attn(q, k, v, F, N, heads, d, n_pre=8, n_post=8, n_global=16, positions=None,
               nthreads=0) -> np.ndarray:
-    """Dual-domain attention over [P][F][heads*d] inputs -> [n_pos][F][C] float64."""
+    """Dual-domain attention over [P][F][heads*d] inputs -> [n_pos][F][C] float64.
+
+    Inputs may also be float64 (the exact output of another oracle module)."""
     q, k, v = _c(q), _c(k), _c(v)
-    dt = _dtype_of(q)
-    assert _dtype_of(k) == dt and _dtype_of(v) == dt
+    dt = _dtype_of(q, allow_f64=True)
+    assert _dtype_of(k, allow_f64=True) == dt and _dtype_of(v, allow_f64=True) == dt
     _check_common(F, N)
     C = heads * d
     P = q.size // (F * C)
@@ -194,3 +196,29 @@ def groupnorm_global(x, gamma, beta, F, N, groups, eps=1e-5, positions=None, nth
                                   mean.ctypes.data, var.ctypes.data, F, N, P, C, groups,
                                   float(eps), pos.ctypes.data, pos.size, nthreads)
     return y, mean, var
+
+
+def _as_f32_exact(a: np.ndarray) -> np.ndarray:
+    """bf16-representable float64 values as float32 (exact)."""
+    return np.ascontiguousarray(a, dtype=np.float32)
+
+
+def temporal_attention(x, w_qkv, b_qkv, w_out, b_out, F, N, heads, d, n_pre=8, n_post=8,
+                       n_global=16, positions=None, nthreads=0, intermediate="bf16"):
+    """Temporal attention module: per-frame input projections (Linear layers,
+    here single-tap temporal convs), dual-domain attention, output projection.
+    intermediate="bf16" rounds q, k, v and the attention output to bf16 as the
+    separate stages exchange them; "f64" keeps them exact.  -> [n_pos][F][C]."""
+    C = heads * d
+    P = x.size // (F * C)
+    pos = _positions(P, positions)
+    rnd = (lambda a: _as_f32_exact(round_bf16(a))) if intermediate == "bf16" else (lambda a: a)
+    proj = []
+    for i in range(3):
+        wi = np.ascontiguousarray(w_qkv[i * C:(i + 1) * C]).reshape(C, C, 1)
+        bi = np.ascontiguousarray(b_qkv[i * C:(i + 1) * C])
+        proj.append(rnd(temporal_conv(x, wi, bi, F, N, 1, positions=pos, nthreads=nthreads)))
+    a = rnd(dual_attn(*proj, F, N, heads, d, n_pre, n_post, n_global, nthreads=nthreads))
+    wo = np.ascontiguousarray(w_out).reshape(C, C, 1)
+    return temporal_conv(a, wo, np.ascontiguousarray(b_out), F, N, 1, nthreads=nthreads)
+

@@ -33,7 +33,8 @@ _LIB = os.path.join(_HERE, "libsynth.so")
 
 # Tensor ids: one independent random stream per input tensor.
 TID = {"q": 1, "k": 2, "v": 3, "conv_x": 4, "conv_w": 5, "conv_b": 6,
-       "gn_x": 7, "gn_gamma": 8, "gn_beta": 9}
+       "gn_x": 7, "gn_gamma": 8, "gn_beta": 9,
+       "attn_x": 10, "w_qkv": 11, "b_qkv": 12, "w_out": 13, "b_out": 14}
 
 
 def build(force: bool = False) -> str:
@@ -187,14 +188,24 @@ def dist(w: Workload, tensor: str):
         "gn_x": (0.5, math.sqrt(2.0)),
         "gn_gamma": (1.0, math.sqrt(0.1)),
         "gn_beta": (0.0, math.sqrt(0.1)),
+        # temporal-attention module: input and Linear layers (fan-in variance)
+        "attn_x": (0.0, 1.0),
+        "w_qkv": (0.0, math.sqrt(1.0 / w.C)), "b_qkv": (0.0, math.sqrt(0.01)),
+        "w_out": (0.0, math.sqrt(1.0 / w.C)), "b_out": (0.0, math.sqrt(0.01)),
     }[tensor]
 
 
 def shape_of(w: Workload, tensor: str):
-    if tensor in ("q", "k", "v", "conv_x", "gn_x"):
+    if tensor in ("q", "k", "v", "conv_x", "gn_x", "attn_x"):
         return w.act_shape
     if tensor == "conv_w":
         return (w.C, w.C, w.k)        # [C_out][C_in][k], PyTorch Conv1d order
+    if tensor == "w_qkv":
+        return (3 * w.C, w.C)         # rows Wq, Wk, Wv; PyTorch Linear order
+    if tensor == "b_qkv":
+        return (3 * w.C,)
+    if tensor == "w_out":
+        return (w.C, w.C)
     return (w.C,)                     # conv_b, gn_gamma, gn_beta
 
 

@@ -117,7 +117,8 @@ def test_groupnorm_rejects(L, kw, expect):
 
 def test_binding_signatures_cover_header():
     for n in declared_functions():
-        if n not in ("vi_status_string", "vi_launch_count"):
+        if n not in ("vi_status_string", "vi_launch_count",
+                     "vi_temporal_attention_workspace_bytes"):
             assert n in _binding.SIGNATURES, n
 
 
@@ -136,3 +137,28 @@ def gnconv(L, x=A, g=B, bt=Cp, w=D, b=E, y=G, F=64, N=4, P=2, C=64, groups=8, ep
 ])
 def test_groupnorm_conv_rejects(L, kw, expect):
     assert gnconv(L, **kw) == expect
+
+
+H_ = 1 << 35
+I_ = 1 << 36
+
+
+def tattn(L, x=A, wqkv=B, bqkv=Cp, wo=D, bo=E, out=G, ws=H_, F=64, N=4, P=2, heads=2, d=64,
+          pre=8, post=8, glob=16):
+    return L.vi_temporal_attention(x, wqkv, bqkv, wo, bo, out, ws, F, N, P, heads, d, pre, post,
+                                   glob, None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(ws=0), INVALID), (dict(x=0), INVALID), (dict(F=63), INVALID), (dict(pre=17), INVALID),
+    (dict(d=32), UNSUP), (dict(ws=H_ + 8), ALIGN),
+    (dict(ws=A + 4096), INVALID),             # workspace overlaps x
+    (dict(out=H_ + 64), INVALID),             # out inside the workspace
+])
+def test_temporal_attention_rejects(L, kw, expect):
+    assert tattn(L, **kw) == expect
+
+
+def test_temporal_attention_workspace_bytes(L):
+    assert L.vi_temporal_attention_workspace_bytes(1024, 2560, 320) == 4 * 1024 * 2560 * 320 * 2
+    assert L.vi_temporal_attention_workspace_bytes(0, 1, 1) == 0

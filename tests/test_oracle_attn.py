@@ -190,3 +190,27 @@ def test_position_subset_equals_full_slice():
     full = oracle.dual_attn(q, k, v, F, N, heads, d)
     sub = oracle.dual_attn(q, k, v, F, N, heads, d, positions=[4, 1])
     np.testing.assert_array_equal(sub, full[[4, 1]])
+
+
+def test_attention_module_equals_library_composition():
+    """Projections + dual attention + output projection; with one clip and no
+    global frames this is Linear -> per-head SDPA -> Linear (library, fp64)."""
+    F, heads, d, P = 16, 2, 8, 2
+    C = heads * d
+    x = _rand((P, F, C), 81)
+    w_qkv, b_qkv = _rand((3 * C, C), 82, std=0.25), _rand((3 * C,), 83)
+    w_out, b_out = _rand((C, C), 84, std=0.25), _rand((C,), 85)
+    got = oracle.temporal_attention(x, w_qkv, b_qkv, w_out, b_out, F, 1, heads, d, 0, 0, 0,
+                                    intermediate="f64")
+    t = lambda a: torch.from_numpy(np.asarray(a, np.float64))
+    xt = t(x)
+    qkv = torch.nn.functional.linear(xt, t(w_qkv), t(b_qkv))          # [P][F][3C]
+    q, k, v = qkv[..., :C], qkv[..., C:2 * C], qkv[..., 2 * C:]
+    hs = lambda a: a.reshape(P, F, heads, d).permute(0, 2, 1, 3)
+    a = torch.nn.functional.scaled_dot_product_attention(hs(q), hs(k), hs(v))
+    a = a.permute(0, 2, 1, 3).reshape(P, F, C)
+    ref = torch.nn.functional.linear(a, t(w_out), t(b_out)).numpy()
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-11)
+    sub = oracle.temporal_attention(x, w_qkv, b_qkv, w_out, b_out, F, 1, heads, d, 0, 0, 0,
+                                    positions=[1], intermediate="f64")
+    np.testing.assert_array_equal(sub, got[[1]])
