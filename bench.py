@@ -474,8 +474,9 @@ def load_traffic(kernel, w):
     """DRAM bytes per launch from the committed ncu summary of this kernel.
 
     None when there is no capture for this workload, or when the kernel's
-    source has changed since the counters were taken (the summary records a
-    hash of the source file it was measured with)."""
+    sources have changed since the counters were taken (the summary records a
+    hash of the source files it was measured with: the kernel's file and the
+    headers it includes)."""
     import hashlib
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
@@ -485,12 +486,15 @@ def load_traffic(kernel, w):
     e = d.get(kernel, {}).get(w.name)
     if e is None:
         return None
-    src = os.path.join(ROOT, "clip_temporal_modules_b200", e["source"])
-    if not os.path.exists(src):
-        return None
-    with open(src, "rb") as fh:
-        if hashlib.sha256(fh.read()).hexdigest()[:16] != e.get("source_sha256_16"):
+    h = hashlib.sha256()
+    for rel in e["sources"]:
+        src = os.path.join(ROOT, "clip_temporal_modules_b200", rel)
+        if not os.path.exists(src):
             return None
+        with open(src, "rb") as fh:
+            h.update(fh.read())
+    if h.hexdigest()[:16] != e.get("sources_sha256_16"):
+        return None
     return e.get("bytes_per_launch")
 
 

@@ -16,8 +16,9 @@ kernel grid:
 Python here only marshals arguments; see _binding.py.
 """
 from ._binding import (LIB_PATH, ViError, dual_attn, groupnorm_conv,  # noqa: F401
-                       groupnorm_global, launch_count, lib, take_device_errors,
-                       temporal_attention, temporal_conv)
+                       groupnorm_global, launch_count, lib, set_conv_tiles_per_job,
+                       take_device_errors, temporal_attention, temporal_conv)
 
 __all__ = ["dual_attn", "temporal_conv", "groupnorm_global", "groupnorm_conv", "temporal_attention", "take_device_errors", "launch_count", "lib",
+           "set_conv_tiles_per_job",
            "ViError", "LIB_PATH"]

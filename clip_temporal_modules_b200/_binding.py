@@ -30,6 +30,8 @@ SIGNATURES = {
     "vi_groupnorm_global_noalloc": [_vp, _vp, _vp, _vp] + [_i] * 5 + [_f, _vp],
     "vi_groupnorm_conv": [_vp] * 6 + [_i] * 5 + [_f, _i, _vp],
     "vi_temporal_attention": [_vp] * 7 + [_i] * 8 + [_vp],
+    "vi_selftest_wait_timeout": [_i, _vp],
+    "vi_set_conv_tiles_per_job": [_i],
     "vi_version": [],
     "vi_take_device_errors": [],
 }
@@ -174,6 +176,13 @@ def temporal_attention(x, w_qkv, b_qkv, w_out, b_out, out=None, workspace=None, 
 def launch_count() -> int:
     """Kernels libvi has launched in this process so far."""
     return int(lib().vi_launch_count())
+
+
+def set_conv_tiles_per_job(tiles: int) -> int:
+    """Tiles per job of the tensor-core conv (0 automatic, 1 or 2); returns the previous value."""
+    r = int(lib().vi_set_conv_tiles_per_job(int(tiles)))
+    _check("vi_set_conv_tiles_per_job", min(r, 0))
+    return r
 
 
 def take_device_errors() -> None:

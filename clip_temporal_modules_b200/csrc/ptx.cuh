@@ -15,6 +15,7 @@ namespace vi {
 unsigned int* device_error_word();
 constexpr unsigned int VI_DEV_ERR_TMA_TIMEOUT = 1u;
 constexpr unsigned int VI_DEV_ERR_MMA_TIMEOUT = 2u;
+constexpr unsigned int VI_DEV_ERR_SELFTEST = 4u;
 
 // A bounded wait gives up after this many nanoseconds of %globaltimer.
 constexpr uint64_t VI_WAIT_LIMIT_NS = 2000000000ull;
@@ -59,13 +60,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 // Wait for the barrier phase with the given parity to complete.  Returns false
-// (and raises `err` in g_device_error) if it has not after VI_WAIT_LIMIT_NS.
+// (and ORs `err` into *err_word) if it has not after limit_ns of %globaltimer.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
-                                                  unsigned int* err_word, unsigned int err) {
+                                                  unsigned int* err_word, unsigned int err,
+                                                  uint64_t limit_ns = VI_WAIT_LIMIT_NS) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer_ns() - t0 > VI_WAIT_LIMIT_NS) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       atomicOr(err_word, err);
       return false;
     }

@@ -31,15 +31,24 @@
 // CTA's barriers, commits are multicast to both CTAs, and the odd CTA's
 // epilogue arrives remotely on the even CTA's accumulator-empty barrier.
 //
-// One of two TMEM accumulators (NJ columns each) is drained by four epilogue
-// warps (TMEM -> registers, + bias, -> bf16 -> global) while the MMAs of the
-// next job fill the other.  Every CTA walks the K-blocks of a job starting at
-// its own offset, so the CTAs do not all stream the same weight tile at once.
+// MT = 2 (the default where it keeps the slab width): a job covers TWO tiles
+// (consecutive in position-major order) on one SM, and every weight stage
+// feeds both: per K-block the CTA loads two x boxes and one set of weight
+// tiles and issues 2 x 4k MMAs into two accumulators.  Weight bytes per flop,
+// through L2 and through shared memory, halve; shared memory (TMA writes plus
+// the tensor core's operand reads) is what limits the one-tile form.
+//
+// TMEM holds a ring of MT + 1 (at least 2) accumulators of NJ columns: four
+// epilogue warps (TMEM -> registers, + bias, -> bf16 -> global) drain the
+// oldest while the MMAs of the next tiles fill the others.  Every CTA walks
+// the K-blocks of a job starting at its own offset, so the CTAs do not all
+// stream the same weight tile at once.
 //
 // Warp roles (192 threads, one CTA per SM, persistent over jobs):
 //   warp 0      TMA producer (one elected thread)
 //   warp 1      TMEM allocator + MMA issuer (one thread, even CTA of a pair)
 //   warps 2..5  epilogue; warp w reads TMEM lanes 32*(w%4) .. +31
+#include <atomic>
 #include <mutex>
 
 #include "ptx.cuh"
@@ -69,13 +78,16 @@ struct TcPlan {
   int F, P, C, k;
   int NJ;                // output channels per job (UMMA N), multiple of 32
   int H;                 // CTAs per MMA (1, or 2 for a pair); each holds NJ/H weight rows
+  int MT;                // tiles per job per CTA (1, or 2 sharing every weight stage)
+  int n_acc;             // TMEM accumulators in the ring (MT + 1, at least 2), NJ columns each
   int n_slabs;           // C / NJ
   int n_fblk;            // ceil(F / 128)
   long long n_tiles;     // P * n_fblk
-  long long n_jobs;      // ceil(n_tiles / H) * n_slabs
+  long long n_jobs;      // ceil(n_tiles / (H * MT)) * n_slabs
   int n_cb;              // C / 64
   int a_rows;            // 127 + k
-  int a_stage;           // bytes per A stage (a_rows x 128 B), 1024-aligned
+  int a_tile;            // bytes of one tile's x box (a_rows x 128 B), 1024-aligned
+  int a_stage;           // bytes per A stage = MT * a_tile
   int b_rows;            // weight rows per CTA per tap = NJ / H
   int b_tap;             // bytes of one tap's block = b_rows * 128
   int b_stage;           // bytes per B stage = k * b_tap (one K-block, all taps)
@@ -91,28 +103,34 @@ struct TcArgs {
   unsigned int* err;
 };
 
-// Ring depths (measured on B200 at F = 1024): with C <= 640 three x stages
-// and two weight stages beat two and three (1.48 vs 1.53 ms at C = 320); at
-// C = 1280 two x stages and as many weight stages as fit are best.  With the
-// GroupNorm transform, three x stages.  sb_pref / sa_pref override (0 = default).
+// Ring depths (measured on B200 at F = 1024): with one tile per job and
+// C <= 640 three x stages and two weight stages beat two and three (1.48 vs
+// 1.53 ms at C = 320); at C = 1280 two x stages and as many weight stages as
+// fit are best.  With the GroupNorm transform, three x stages.  Two tiles per
+// job: two stages of each.  sb_pref / sa_pref / mt_pref override (0 = default).
 static int g_tc_sb_pref = 0, g_tc_sa_pref = 0;
+static std::atomic<int> g_tc_mt_pref{0};
 
-static bool tc_plan(int F, int P, int C, int k, bool pair, TcPlan& pl, bool norm = false) {
+static bool tc_plan(int F, int P, int C, int k, bool pair, TcPlan& pl, bool norm = false,
+                    int mt = 1) {
   if (k < 1 || k % 2 == 0 || 127 + k > 256 || C % TC_KB != 0) return false;
+  if (mt != 1 && (mt != 2 || pair || norm)) return false;
   const int H = pair ? 2 : 1;
+  const int n_acc = mt + 1 > 2 ? mt + 1 : 2;
   const int a_rows = 127 + k;
-  const int a_stage = ((a_rows * 128 + 1023) / 1024) * 1024;
+  const int a_tile = ((a_rows * 128 + 1023) / 1024) * 1024;
+  const int a_stage = mt * a_tile;
   const int fixed = 1024 /* align slack */ + 4 * C + 64 /* bias, padded */ + 512 /* bars */ +
                     (norm ? 16 * C : 0) /* GroupNorm coefficients */;
   // Widest slab (<= 160 output channels, a multiple of 32 dividing C) whose
   // all-tap weight stages leave room for at least two of each ring.
   for (int nj = TC_NJ_MAX; nj >= 32; nj -= 32) {
-    if (C % nj != 0 || (nj / H) % 8 != 0) continue;
+    if (C % nj != 0 || (nj / H) % 8 != 0 || n_acc * nj > TC_TMEM_COLS) continue;
     const int b_stage = k * (nj / H) * 128;
     const bool few_k = C <= 640 || norm;
-    int sa = g_tc_sa_pref > 0 ? g_tc_sa_pref : (few_k ? 3 : 2);
+    int sa = g_tc_sa_pref > 0 ? g_tc_sa_pref : (mt == 2 ? 2 : few_k ? 3 : 2);
     if (sa > TC_SA_MAX) sa = TC_SA_MAX;
-    int sb = g_tc_sb_pref > 0 ? g_tc_sb_pref : (few_k ? 2 : TC_SB_MAX);
+    int sb = g_tc_sb_pref > 0 ? g_tc_sb_pref : (mt == 2 ? 2 : few_k ? 2 : TC_SB_MAX);
     const int sb_fit = (TC_SMEM_LIMIT - fixed - sa * a_stage) / b_stage;
     if (sb > sb_fit) sb = sb_fit;
     if (sb < 2) {            // not enough room: fall back to the minimum x ring
@@ -124,12 +142,15 @@ static bool tc_plan(int F, int P, int C, int k, bool pair, TcPlan& pl, bool norm
     pl.F = F; pl.P = P; pl.C = C; pl.k = k;
     pl.NJ = nj;
     pl.H = H;
+    pl.MT = mt;
+    pl.n_acc = n_acc;
     pl.n_slabs = C / nj;
     pl.n_fblk = (F + TC_M - 1) / TC_M;
     pl.n_tiles = (long long)P * pl.n_fblk;
-    pl.n_jobs = ((pl.n_tiles + H - 1) / H) * pl.n_slabs;
+    pl.n_jobs = ((pl.n_tiles + H * mt - 1) / (H * mt)) * pl.n_slabs;
     pl.n_cb = C / TC_KB;
     pl.a_rows = a_rows;
+    pl.a_tile = a_tile;
     pl.a_stage = a_stage;
     pl.b_rows = nj / H;
     pl.b_tap = pl.b_rows * 128;
@@ -153,11 +174,11 @@ __global__ void __launch_bounds__(TC_THREADS + (NORM ? 128 : 0), 1)
   const uint32_t sB = sA + pl.sa * pl.a_stage;
   const uint32_t sBias = sB + pl.sb * pl.b_stage;
   const uint32_t sBar = sBias + ((4 * pl.C + 63) / 64) * 64;
-  // barrier block: a_full[SA] a_empty[SA] b_full[SB] b_empty[SB] acc_full[2] acc_empty[2] drain tmem_slot
+  // barrier block: a_full[SA] a_empty[SA] b_full[SB] b_empty[SB] acc_full[4] acc_empty[4] drain tmem_slot
   const uint32_t a_full = sBar, a_empty = a_full + 8 * TC_SA_MAX;
   const uint32_t b_full = a_empty + 8 * TC_SA_MAX, b_empty = b_full + 8 * TC_SB_MAX;
-  const uint32_t acc_full = b_empty + 8 * TC_SB_MAX, acc_empty = acc_full + 16;
-  const uint32_t drain = acc_empty + 16, tmem_slot = drain + 8;
+  const uint32_t acc_full = b_empty + 8 * TC_SB_MAX, acc_empty = acc_full + 32;
+  const uint32_t drain = acc_empty + 32, tmem_slot = drain + 8;
   const uint32_t a_ready = tmem_slot + 8;      // NORM: x stage normalised [SA]
   const uint32_t sCoef = sBar + 512;           // NORM: float4 per channel
   float* bias_s = reinterpret_cast<float*>(smem_raw + (sBias - smem_u32(smem_raw)));
@@ -175,7 +196,7 @@ __global__ void __launch_bounds__(TC_THREADS + (NORM ? 128 : 0), 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < pl.sa; ++i) { mbar_init(a_full + 8 * i, PAIR ? 2 : 1); mbar_init(a_empty + 8 * i, 1); }
     for (int i = 0; i < pl.sb; ++i) { mbar_init(b_full + 8 * i, PAIR ? 2 : 1); mbar_init(b_empty + 8 * i, 1); }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < pl.n_acc; ++i) {
       mbar_init(acc_full + 8 * i, 1);
       mbar_init(acc_empty + 8 * i, PAIR ? 8 : 4);
     }
@@ -217,10 +238,16 @@ __global__ void __launch_bounds__(TC_THREADS + (NORM ? 128 : 0), 1)
       bool ok = true;
       for (long long job = cluster_id; job < pl.n_jobs && ok; job += n_clusters) {
         const int slab = (int)(job % pl.n_slabs);
-        const long long tile = (job / pl.n_slabs) * pl.H + rank;
-        const int fb = (int)(tile % pl.n_fblk);
-        const int p = (int)(tile / pl.n_fblk);     // == P past the last tile: reads as zeros
-        const int f0 = fb * TC_M;
+        const long long tile0 = (job / pl.n_slabs) * (pl.H * pl.MT) + rank;
+        // Frame row and position of each tile of the job; p == P past the
+        // last tile, which reads as zeros.
+        int frow[2], pos[2];
+#pragma unroll
+        for (int m = 0; m < 2; ++m) {
+          const long long tile = tile0 + m;
+          frow[m] = (int)(tile % pl.n_fblk) * TC_M - halo;
+          pos[m] = (int)(tile / pl.n_fblk);
+        }
         int wrow = (slab * pl.n_cb * pl.k * pl.H + (int)rank) * pl.b_rows;   // row of (slab, cb 0, t 0)
         const int wrow_cb = pl.k * pl.H * pl.b_rows, wrow_t = pl.H * pl.b_rows;
         for (int ib = 0; ib < pl.n_cb && ok; ++ib) {
@@ -230,10 +257,12 @@ __global__ void __launch_bounds__(TC_THREADS + (NORM ? 128 : 0), 1)
           const uint32_t dst = sA + sa * pl.a_stage;
           if constexpr (PAIR) {
             mbar_arrive_expect_tx_cluster(lead_a_full + 8 * sa, (uint32_t)pl.a_rows * 128u);
-            tma_load_3d_pair(dst, &tmx, cb * TC_KB, f0 - halo, p, lead_a_full + 8 * sa);
+            tma_load_3d_pair(dst, &tmx, cb * TC_KB, frow[0], pos[0], lead_a_full + 8 * sa);
           } else {
-            mbar_arrive_expect_tx(a_full + 8 * sa, (uint32_t)pl.a_rows * 128u);
-            tma_load_3d(dst, &tmx, cb * TC_KB, f0 - halo, p, a_full + 8 * sa);
+            mbar_arrive_expect_tx(a_full + 8 * sa, (uint32_t)(pl.MT * pl.a_rows) * 128u);
+            tma_load_3d(dst, &tmx, cb * TC_KB, frow[0], pos[0], a_full + 8 * sa);
+            if (pl.MT == 2)
+              tma_load_3d(dst + pl.a_tile, &tmx, cb * TC_KB, frow[1], pos[1], a_full + 8 * sa);
           }
           if (++sa == pl.sa) { sa = 0; pa ^= 1; a_used = true; }
           // One B stage = this CTA's weight blocks of every tap of K-block cb.
@@ -263,15 +292,21 @@ __global__ void __launch_bounds__(TC_THREADS + (NORM ? 128 : 0), 1)
       const uint32_t a_st16 = (uint32_t)pl.a_stage >> 4, b_st16 = (uint32_t)pl.b_stage >> 4;
       const uint32_t bt16 = (uint32_t)pl.b_tap >> 4;  // one tap's block in w
       const uint32_t bk16 = (2u * lbo_b) >> 4;     // one K step of 16 in w
-      int sa = 0, pa = 0, sbi = 0, pb = 0, buf = 0, pacc = 0;
-      bool acc_used = false;
+      const uint32_t at16 = (uint32_t)pl.a_tile >> 4;  // second tile of an x stage
+      int sa = 0, pa = 0, sbi = 0, pb = 0;
+      // Accumulator ring: n_acc slots of NJ columns, one per tile, in order.
+      int slot = 0, pslot = 0;
+      bool slot_used = false;
       bool ok = true;
       for (long long job = cluster_id; job < pl.n_jobs && ok; job += n_clusters) {
-        if (acc_used && !tc_wait<PAIR>(acc_empty + 8 * buf, (uint32_t)(pacc ^ 1), args.err,
-                                       VI_DEV_ERR_MMA_TIMEOUT)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t d_tmem = tmem_base + (uint32_t)(buf * pl.NJ);
-        uint32_t acc = 0u;
+        // This job's accumulator slots and the parity of their last release.
+        int js[2], jp[2];
+        bool ju[2];
+#pragma unroll
+        for (int m = 0; m < 2; ++m) {
+          js[m] = slot; jp[m] = pslot; ju[m] = slot_used;
+          if (m < pl.MT && ++slot == pl.n_acc) { slot = 0; pslot ^= 1; slot_used = true; }
+        }
         for (int ib = 0; ib < pl.n_cb && ok; ++ib) {
           if (!tc_wait<PAIR>((NORM ? a_ready : a_full) + 8 * sa, (uint32_t)pa, args.err,
                              VI_DEV_ERR_TMA_TIMEOUT) ||
@@ -280,28 +315,46 @@ __global__ void __launch_bounds__(TC_THREADS + (NORM ? 128 : 0), 1)
             break;
           }
           tc_fence_after();
-          // k taps x 4 K steps = 4k MMAs back to back (12 for k = 3): enough
-          // tensor work queued to hide the wait/commit of the next K-block.
-          const uint64_t ad_stage = ad_base + (uint64_t)(sa * a_st16);
           const uint64_t bd_stage = bd_base + (uint64_t)(sbi * b_st16);
-          for (int t = 0; t < pl.k; ++t) {
-            // Tap t: the x tile shifted down by t rows of 128 B (8 units of 16 B).
-            const uint64_t ad = ad_stage + (uint64_t)(8u * t);
-            const uint64_t bd = bd_stage + (uint64_t)(t * bt16);
-            // K steps of 16: +32 B inside the swizzled x rows, +2 columns of 8 in w.
-            if constexpr (PAIR) {
-              umma_bf16_pair(d_tmem, ad, bd, idesc, acc);
-              umma_bf16_pair(d_tmem, ad + 2u, bd + bk16, idesc, 1u);
-              umma_bf16_pair(d_tmem, ad + 4u, bd + 2u * bk16, idesc, 1u);
-              umma_bf16_pair(d_tmem, ad + 6u, bd + 3u * bk16, idesc, 1u);
-            } else {
-              umma_bf16(d_tmem, ad, bd, idesc, acc);
-              umma_bf16(d_tmem, ad + 2u, bd + bk16, idesc, 1u);
-              umma_bf16(d_tmem, ad + 4u, bd + 2u * bk16, idesc, 1u);
-              umma_bf16(d_tmem, ad + 6u, bd + 3u * bk16, idesc, 1u);
+#pragma unroll
+          for (int m = 0; m < 2; ++m) {
+            if (m >= pl.MT) break;
+            if (ib == 0) {
+              // The slot must have been drained by the epilogue of its last job.
+              if (ju[m] && !tc_wait<PAIR>(acc_empty + 8 * js[m], (uint32_t)(jp[m] ^ 1), args.err,
+                                          VI_DEV_ERR_MMA_TIMEOUT)) { ok = false; break; }
+              tc_fence_after();
             }
-            acc = 1u;
+            const uint32_t d_tmem = tmem_base + (uint32_t)(js[m] * pl.NJ);
+            // k taps x 4 K steps = 4k MMAs back to back per tile (12 for k = 3;
+            // 24 per stage with two tiles): enough tensor work queued to hide
+            // the wait/commit of the next K-block.
+            const uint64_t ad_stage = ad_base + (uint64_t)(sa * a_st16 + m * at16);
+            uint32_t acc = ib > 0 ? 1u : 0u;
+            for (int t = 0; t < pl.k; ++t) {
+              // Tap t: the x tile shifted down by t rows of 128 B (8 units of 16 B).
+              const uint64_t ad = ad_stage + (uint64_t)(8u * t);
+              const uint64_t bd = bd_stage + (uint64_t)(t * bt16);
+              // K steps of 16: +32 B inside the swizzled x rows, +2 columns of 8 in w.
+              if constexpr (PAIR) {
+                umma_bf16_pair(d_tmem, ad, bd, idesc, acc);
+                umma_bf16_pair(d_tmem, ad + 2u, bd + bk16, idesc, 1u);
+                umma_bf16_pair(d_tmem, ad + 4u, bd + 2u * bk16, idesc, 1u);
+                umma_bf16_pair(d_tmem, ad + 6u, bd + 3u * bk16, idesc, 1u);
+              } else {
+                umma_bf16(d_tmem, ad, bd, idesc, acc);
+                umma_bf16(d_tmem, ad + 2u, bd + bk16, idesc, 1u);
+                umma_bf16(d_tmem, ad + 4u, bd + 2u * bk16, idesc, 1u);
+                umma_bf16(d_tmem, ad + 6u, bd + 3u * bk16, idesc, 1u);
+              }
+              acc = 1u;
+            }
+            if (ib == pl.n_cb - 1) {                  // accumulator ready for the epilogue
+              if constexpr (PAIR) umma_commit_pair_mc(acc_full + 8 * js[m], 0x3);
+              else umma_commit(acc_full + 8 * js[m]);
+            }
           }
+          if (!ok) break;
           if constexpr (PAIR) {
             umma_commit_pair_mc(b_empty + 8 * sbi, 0x3);
             umma_commit_pair_mc(a_empty + 8 * sa, 0x3);
@@ -312,9 +365,6 @@ __global__ void __launch_bounds__(TC_THREADS + (NORM ? 128 : 0), 1)
           if (++sbi == pl.sb) { sbi = 0; pb ^= 1; }
           if (++sa == pl.sa) { sa = 0; pa ^= 1; }
         }
-        if constexpr (PAIR) umma_commit_pair_mc(acc_full + 8 * buf, 0x3);
-        else umma_commit(acc_full + 8 * buf);         // accumulator ready for the epilogue
-        if (++buf == 2) { buf = 0; pacc ^= 1; acc_used = true; }
       }
       // Every MMA this thread issued must finish before TMEM is released.
       if constexpr (PAIR) umma_commit_pair_mc(drain, 0x3);
@@ -338,7 +388,7 @@ __global__ void __launch_bounds__(TC_THREADS + (NORM ? 128 : 0), 1)
       int sa = 0, pa = 0;
       bool ok = true;
       for (long long job = cluster_id; job < pl.n_jobs && ok; job += n_clusters) {
-        const long long tile = (job / pl.n_slabs) * pl.H + rank;
+        const long long tile = (job / pl.n_slabs) * (pl.H * pl.MT) + rank;
         const int fb = (int)(tile % pl.n_fblk);
         const int f_first = fb * TC_M - halo;
         for (int ib = 0; ib < pl.n_cb && ok; ++ib) {
@@ -374,43 +424,48 @@ __global__ void __launch_bounds__(TC_THREADS + (NORM ? 128 : 0), 1)
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;                      // TMEM lane quadrant of this warp
     const int m = 32 * q + lane;                 // frame within the tile
-    int buf = 0, pacc = 0;
-    for (long long job = cluster_id; job < pl.n_jobs; job += n_clusters) {
-      if (!tc_wait<PAIR>(acc_full + 8 * buf, (uint32_t)pacc, args.err, VI_DEV_ERR_MMA_TIMEOUT))
-        break;
-      tc_fence_after();
+    int buf = 0, pacc = 0;                       // accumulator ring, as the MMA issuer walks it
+    bool ok = true;
+    for (long long job = cluster_id; job < pl.n_jobs && ok; job += n_clusters) {
       const int slab = (int)(job % pl.n_slabs);
-      const long long tile = (job / pl.n_slabs) * pl.H + rank;
-      const int fb = (int)(tile % pl.n_fblk);
-      const long long p = tile / pl.n_fblk;
-      const int f = fb * TC_M + m;
-      const bool valid = tile < pl.n_tiles && f < pl.F;
-      bf16* out = args.y + ((size_t)(valid ? p : 0) * pl.F + (valid ? f : 0)) * pl.C +
-                  (size_t)slab * pl.NJ;
       const float* bs = bias_s + slab * pl.NJ;
-      for (int c0 = 0; c0 < pl.NJ; c0 += 32) {
-        uint32_t r[32];
-        tmem_ld32(tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * pl.NJ + c0), r);
-        tmem_wait_ld();
-        if (valid) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i)
-            pk[i] = pack2_bf16(__uint_as_float(r[2 * i]) + bs[c0 + 2 * i],
-                               __uint_as_float(r[2 * i + 1]) + bs[c0 + 2 * i + 1]);
-          uint4* o = reinterpret_cast<uint4*>(out + c0);
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            o[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+      for (int mt = 0; mt < pl.MT; ++mt) {
+        if (!tc_wait<PAIR>(acc_full + 8 * buf, (uint32_t)pacc, args.err, VI_DEV_ERR_MMA_TIMEOUT)) {
+          ok = false;
+          break;
         }
+        tc_fence_after();
+        const long long tile = (job / pl.n_slabs) * (pl.H * pl.MT) + rank + mt;
+        const int fb = (int)(tile % pl.n_fblk);
+        const long long p = tile / pl.n_fblk;
+        const int f = fb * TC_M + m;
+        const bool valid = tile < pl.n_tiles && f < pl.F;
+        bf16* out = args.y + ((size_t)(valid ? p : 0) * pl.F + (valid ? f : 0)) * pl.C +
+                    (size_t)slab * pl.NJ;
+        for (int c0 = 0; c0 < pl.NJ; c0 += 32) {
+          uint32_t r[32];
+          tmem_ld32(tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * pl.NJ + c0), r);
+          tmem_wait_ld();
+          if (valid) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              pk[i] = pack2_bf16(__uint_as_float(r[2 * i]) + bs[c0 + 2 * i],
+                                 __uint_as_float(r[2 * i + 1]) + bs[c0 + 2 * i + 1]);
+            uint4* o = reinterpret_cast<uint4*>(out + c0);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              o[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if constexpr (PAIR) mbar_arrive_cluster(lead_acc_empty + 8 * buf);
+          else mbar_arrive(acc_empty + 8 * buf);
+        }
+        if (++buf == pl.n_acc) { buf = 0; pacc ^= 1; }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        if constexpr (PAIR) mbar_arrive_cluster(lead_acc_empty + 8 * buf);
-        else mbar_arrive(acc_empty + 8 * buf);
-      }
-      if (++buf == 2) { buf = 0; pacc ^= 1; }
     }
   }
   tc_fence_before();
@@ -452,6 +507,13 @@ bool encode_tmap(CUtensorMap* map, const void* base, int rank, const uint64_t* d
 // The CTA-pair form is correct but, measured on B200, slower than the
 // one-SM form at every workload here, so the dispatcher takes the one-SM form.
 constexpr bool TC_USE_PAIR = false;
+// Tiles per job of the one-SM form when the plan fits (2: every weight stage
+// feeds two 128-frame tiles).
+constexpr int TC_MT_DEFAULT = 2;
+
+// Tiles per job of the one-SM form: 0 = automatic, 1 or 2 = that form where
+// its plan fits.  Returns the previous setting.
+int conv_set_tiles_per_job(int mt) { return g_tc_mt_pref.exchange(mt); }
 
 bool temporal_conv_tc_ok(int F, int P, int C, int k) {
   TcPlan pl;
@@ -518,7 +580,15 @@ int temporal_conv_bf16_tc(const bf16* x, const bf16* w, const bf16* b, bf16* y, 
   TcPlan pl;
   const bool norm = coef != nullptr;
   const bool pair = !norm && TC_USE_PAIR && tc_plan(F, P, C, k, true, pl);
-  if (!pair && !tc_plan(F, P, C, k, false, pl, norm)) return VI_ERR_UNSUPPORTED;
+  if (!pair) {
+    if (!tc_plan(F, P, C, k, false, pl, norm)) return VI_ERR_UNSUPPORTED;
+    // Two tiles per job when that plan keeps the slab width (a narrower MMA
+    // N costs more than the weight traffic it saves).
+    const int pref = g_tc_mt_pref.load(std::memory_order_relaxed);
+    const int mt = pref > 0 ? pref : TC_MT_DEFAULT;
+    TcPlan pl2;
+    if (mt == 2 && !norm && tc_plan(F, P, C, k, false, pl2, false, 2) && pl2.NJ >= pl.NJ) pl = pl2;
+  }
   unsigned int* err = device_error_word();
   if (!err) return VI_ERR_CUDA;
   // x as [P][F][C]: box of 64 channels x a_rows frames x 1 position, 128B swizzle.

@@ -36,6 +36,7 @@ int temporal_conv_bf16_tc(const bf16*, const bf16*, const bf16*, bf16*, int, int
                           cudaStream_t, const float* coef = nullptr);
 bool temporal_conv_tc_ok(int F, int P, int C, int k);
 bool temporal_conv_tc_norm_ok(int F, int P, int C, int k);
+int conv_set_tiles_per_job(int mt);
 template <typename T>
 int gn_stats_launch(const T*, const T*, const T*, int64_t, int, int, float, void*, cudaStream_t,
                     const float**);
@@ -73,6 +74,19 @@ cudaError_t scratch_alloc(void** p, size_t bytes, cudaStream_t stream) {
 }
 
 cudaError_t scratch_free(void* p, cudaStream_t stream) { return cudaFreeAsync(p, stream); }
+
+// One thread waits, with the library's bounded wait, on an mbarrier that
+// nothing ever arrives at: the wait runs out after limit_ns and the kernel
+// records the timeout and returns (the timeout path of every pipeline).
+__global__ void selftest_wait_timeout_kernel(unsigned int* err_word, uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  const uint32_t b = smem_u32(&bar);
+  if (threadIdx.x == 0) {
+    mbar_init(b, 1);
+    fence_barrier_init();
+    mbar_wait_bounded(b, 0, err_word, VI_DEV_ERR_SELFTEST, limit_ns);
+  }
+}
 
 int sm_count() {
   static int cached[64] = {0};
@@ -336,6 +350,21 @@ const char* vi_status_string(int status) {
 int vi_version(void) { return 100; }
 
 unsigned long long vi_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int vi_selftest_wait_timeout(int limit_us, vi_stream_t stream) {
+  if (limit_us <= 0 || limit_us > 1000000) return VI_ERR_INVALID_ARG;
+  unsigned int* err = device_error_word();
+  if (!err) return VI_ERR_CUDA;
+  selftest_wait_timeout_kernel<<<1, 32, 0, as_stream(stream)>>>(err, (uint64_t)limit_us * 1000ull);
+  if (cudaGetLastError() != cudaSuccess) return VI_ERR_CUDA;
+  note_launch();
+  return VI_OK;
+}
+
+int vi_set_conv_tiles_per_job(int tiles) {
+  if (tiles < 0 || tiles > 2) return VI_ERR_INVALID_ARG;
+  return conv_set_tiles_per_job(tiles);
+}
 
 int vi_take_device_errors(void) {
   if (!device_error_word()) return VI_ERR_CUDA;

@@ -81,6 +81,26 @@ int vi_take_device_errors(void);
 unsigned long long vi_launch_count(void);
 
 /*
+ * Self-test of the bounded-wait path: enqueues one tiny kernel that waits on
+ * an mbarrier nothing ever arrives at, gives up after limit_us microseconds
+ * (1 .. 1000000), records the timeout in the device error word and returns.
+ * The next vi_take_device_errors() then reports VI_ERR_DEVICE_TIMEOUT.  No
+ * fault, trap or hang is involved; the GPU context stays usable.
+ */
+int vi_selftest_wait_timeout(int limit_us, vi_stream_t stream);
+
+/*
+ * Tuning knob of the bf16 tensor-core conv (vi_temporal_conv and the
+ * projections of vi_temporal_attention): how many 128-frame tiles one job of
+ * a CTA covers.  0 = automatic (2 where that keeps the widest output-channel
+ * slab, else 1), 1 or 2 = that form wherever its plan fits.  Both forms give
+ * the same result up to fp32 summation order.  Process-wide; returns the
+ * previous setting, or VI_ERR_INVALID_ARG for a value outside 0..2.  It has no
+ * counterpart in the method: it exists for measurement and tests.
+ */
+int vi_set_conv_tiles_per_job(int tiles);
+
+/*
  * Dual-domain temporal attention (attention-module paragraph of the source).
  *
  * For every position p, head h and clip i (frames [s, e), s = i*L, e = s+L),

@@ -162,3 +162,13 @@ def test_temporal_attention_rejects(L, kw, expect):
 def test_temporal_attention_workspace_bytes(L):
     assert L.vi_temporal_attention_workspace_bytes(1024, 2560, 320) == 4 * 1024 * 2560 * 320 * 2
     assert L.vi_temporal_attention_workspace_bytes(0, 1, 1) == 0
+
+
+def test_conv_tiles_per_job_knob(L):
+    """The tuning knob takes 0..2, returns the previous value, and needs no GPU."""
+    assert L.vi_set_conv_tiles_per_job(3) == -1
+    assert L.vi_set_conv_tiles_per_job(-1) == -1
+    prev = L.vi_set_conv_tiles_per_job(1)
+    assert prev in (0, 1, 2)
+    assert L.vi_set_conv_tiles_per_job(2) == 1
+    assert L.vi_set_conv_tiles_per_job(prev) == 2

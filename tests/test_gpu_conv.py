@@ -62,3 +62,18 @@ def test_result_does_not_depend_on_clip_count(cuda_device):
     torch.cuda.synchronize()
     for y in ys[1:]:
         assert torch.equal(y, ys[0])
+
+
+@pytest.mark.parametrize("tiles", [1, 2])
+@pytest.mark.parametrize("w", [W("bf16_F48_C64_odd_tiles", "bf16", 48, 3, 5, 64),
+                               W("bf16_F200_C320_ragged", "bf16", 200, 8, 3, 320),
+                               W("bf16_F24_C320_k1", "bf16", 24, 3, 3, 320, k=1)],
+                         ids=lambda w: w.name)
+def test_one_and_two_tiles_per_job(cuda_device, w, tiles):
+    """Both job forms of the tensor-core conv (one 128-frame tile per job, or
+    two sharing every weight stage; odd tile counts leave a zero tile)."""
+    prev = vi.set_conv_tiles_per_job(tiles)
+    try:
+        run_case(w)
+    finally:
+        vi.set_conv_tiles_per_job(prev)
