@@ -38,16 +38,25 @@
 // through L2 and through shared memory, halve; shared memory (TMA writes plus
 // the tensor core's operand reads) is what limits the one-tile form.
 //
-// TMEM holds a ring of MT + 1 (at least 2) accumulators of NJ columns: four
+// TMEM holds a ring of MT + 1 (at least 2) accumulators of NJ columns: eight
 // epilogue warps (TMEM -> registers, + bias, -> bf16 -> global) drain the
 // oldest while the MMAs of the next tiles fill the others.  Every CTA walks
 // the K-blocks of a job starting at its own offset, so the CTAs do not all
 // stream the same weight tile at once.
 //
+// The epilogue writes y through shared memory: per 32-channel chunk of an
+// accumulator the four warps write 128 rows x 64 bytes (64-byte swizzle, so
+// the 16-byte writes of eight consecutive rows hit distinct banks) into one of
+// two staging buffers, and one thread stores the chunk with a TMA tensor
+// store, which also drops the rows past the last frame.  Full 64-byte row
+// segments reach L2 in one piece (direct 16-byte stores from every row left
+// partial sectors and cost a quarter of the kernel's time).
+//
 // Warp roles (192 threads, one CTA per SM, persistent over jobs):
 //   warp 0      TMA producer (one elected thread)
 //   warp 1      TMEM allocator + MMA issuer (one thread, even CTA of a pair)
 //   warps 2..5  epilogue; warp w reads TMEM lanes 32*(w%4) .. +31
+//   warps 6..9  (GroupNorm fusion only) normalise the landed x tiles
 #include <atomic>
 #include <mutex>
 
@@ -61,7 +70,9 @@ constexpr int TC_KB = 64;        // input channels per K-block
 constexpr int TC_SA_MAX = 6;     // A (x) stages at most
 constexpr int TC_SB_MAX = 8;     // B (w) stages at most
 constexpr int TC_NJ_MAX = 160;   // a B stage holds all k taps of one K-block
-constexpr int TC_THREADS = 192;          // + 128 transform threads with NORM
+constexpr int TC_EPI_WARPS = 4;          // one per TMEM lane quadrant
+constexpr int TC_THREADS = 64 + 32 * TC_EPI_WARPS;   // + 128 transform threads with NORM
+constexpr int TC_OUT_CHUNK = 128 * 64;   // staged output: 128 frames x 32 channels of bf16
 constexpr int TC_TMEM_COLS = 512;
 constexpr int TC_SMEM_LIMIT = 232448;   // 227 KB opt-in per CTA
 
@@ -120,7 +131,8 @@ static bool tc_plan(int F, int P, int C, int k, bool pair, TcPlan& pl, bool norm
   const int a_rows = 127 + k;
   const int a_tile = ((a_rows * 128 + 1023) / 1024) * 1024;
   const int a_stage = mt * a_tile;
-  const int fixed = 1024 /* align slack */ + 4 * C + 64 /* bias, padded */ + 512 /* bars */ +
+  const int fixed = 1024 /* align slack */ + 2 * TC_OUT_CHUNK /* output staging */ + 4 * C +
+                    64 /* bias, padded */ + 512 /* bars */ +
                     (norm ? 16 * C : 0) /* GroupNorm coefficients */;
   // Widest slab (<= 160 output channels, a multiple of 32 dividing C) whose
   // all-tap weight stages leave room for at least two of each ring.
@@ -166,13 +178,15 @@ static bool tc_plan(int F, int P, int C, int k, bool pair, TcPlan& pl, bool norm
 template <bool PAIR, bool NORM>
 __global__ void __launch_bounds__(TC_THREADS + (NORM ? 128 : 0), 1)
     temporal_conv_tc_kernel(const __grid_constant__ CUtensorMap tmx,
-                            const __grid_constant__ CUtensorMap tmw, const TcPlan pl,
+                            const __grid_constant__ CUtensorMap tmw,
+                            const __grid_constant__ CUtensorMap tmy, const TcPlan pl,
                             const TcArgs args) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
   const uint32_t sA = base;
   const uint32_t sB = sA + pl.sa * pl.a_stage;
-  const uint32_t sBias = sB + pl.sb * pl.b_stage;
+  const uint32_t sOut = sB + pl.sb * pl.b_stage;       // 2 staging buffers, 1024-aligned
+  const uint32_t sBias = sOut + 2 * TC_OUT_CHUNK;
   const uint32_t sBar = sBias + ((4 * pl.C + 63) / 64) * 64;
   // barrier block: a_full[SA] a_empty[SA] b_full[SB] b_empty[SB] acc_full[4] acc_empty[4] drain tmem_slot
   const uint32_t a_full = sBar, a_empty = a_full + 8 * TC_SA_MAX;
@@ -198,7 +212,7 @@ __global__ void __launch_bounds__(TC_THREADS + (NORM ? 128 : 0), 1)
     for (int i = 0; i < pl.sb; ++i) { mbar_init(b_full + 8 * i, PAIR ? 2 : 1); mbar_init(b_empty + 8 * i, 1); }
     for (int i = 0; i < pl.n_acc; ++i) {
       mbar_init(acc_full + 8 * i, 1);
-      mbar_init(acc_empty + 8 * i, PAIR ? 8 : 4);
+      mbar_init(acc_empty + 8 * i, PAIR ? 2 * TC_EPI_WARPS : TC_EPI_WARPS);
     }
     mbar_init(drain, 1);
     if (NORM)
@@ -371,7 +385,7 @@ __global__ void __launch_bounds__(TC_THREADS + (NORM ? 128 : 0), 1)
       else umma_commit(drain);
       tc_wait<PAIR>(drain, 0, args.err, VI_DEV_ERR_MMA_TIMEOUT);
     }
-  } else if (warp >= 6) {
+  } else if (warp >= 2 + TC_EPI_WARPS) {
     // ------------------------------------------------------------ transform (NORM)
     // Normalise each landed x stage in place, x -> (x - m_c) a_c + beta_c,
     // then hand it to the MMA.  Rows outside [0, F) stay zero: the conv pads
@@ -424,39 +438,58 @@ __global__ void __launch_bounds__(TC_THREADS + (NORM ? 128 : 0), 1)
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;                      // TMEM lane quadrant of this warp
     const int m = 32 * q + lane;                 // frame within the tile
+    const bool leader = warp == 2 && lane == 0;  // issues the TMA stores
+    // Row m of a staging buffer: 64 bytes; its 16-byte chunk i sits at
+    // i ^ ((m >> 1) & 3) (64-byte swizzle, buffers 1024-aligned).
+    const uint32_t row_off = (uint32_t)m * 64u;
+    const uint32_t swz = (uint32_t)((m >> 1) & 3);
+    int ob = 0;                                  // staging buffer of the next chunk
     int buf = 0, pacc = 0;                       // accumulator ring, as the MMA issuer walks it
     bool ok = true;
     for (long long job = cluster_id; job < pl.n_jobs && ok; job += n_clusters) {
       const int slab = (int)(job % pl.n_slabs);
       const float* bs = bias_s + slab * pl.NJ;
       for (int mt = 0; mt < pl.MT; ++mt) {
-        if (!tc_wait<PAIR>(acc_full + 8 * buf, (uint32_t)pacc, args.err, VI_DEV_ERR_MMA_TIMEOUT)) {
+        // The four warps take the (bounded) wait's outcome together, so that
+        // none of them is left at the staging barriers below.
+        bool got = tc_wait<PAIR>(acc_full + 8 * buf, (uint32_t)pacc, args.err,
+                                 VI_DEV_ERR_MMA_TIMEOUT);
+        got = named_bar_and(1, 32 * TC_EPI_WARPS, got);
+        if (!got) {
           ok = false;
           break;
         }
         tc_fence_after();
         const long long tile = (job / pl.n_slabs) * (pl.H * pl.MT) + rank + mt;
         const int fb = (int)(tile % pl.n_fblk);
-        const long long p = tile / pl.n_fblk;
-        const int f = fb * TC_M + m;
-        const bool valid = tile < pl.n_tiles && f < pl.F;
-        bf16* out = args.y + ((size_t)(valid ? p : 0) * pl.F + (valid ? f : 0)) * pl.C +
-                    (size_t)slab * pl.NJ;
+        const int p = (int)(tile / pl.n_fblk);
+        const bool tile_ok = tile < pl.n_tiles;
         for (int c0 = 0; c0 < pl.NJ; c0 += 32) {
           uint32_t r[32];
           tmem_ld32(tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * pl.NJ + c0), r);
           tmem_wait_ld();
-          if (valid) {
+          const uint32_t stage = sOut + (uint32_t)ob * TC_OUT_CHUNK;
+          if (leader) bulk_wait_read_le1();   // the store that last read this buffer is done
+          named_bar_sync(1, 32 * TC_EPI_WARPS);
+          if (tile_ok) {
             uint32_t pk[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i)
               pk[i] = pack2_bf16(__uint_as_float(r[2 * i]) + bs[c0 + 2 * i],
                                  __uint_as_float(r[2 * i + 1]) + bs[c0 + 2 * i + 1]);
-            uint4* o = reinterpret_cast<uint4*>(out + c0);
 #pragma unroll
             for (int i = 0; i < 4; ++i)
-              o[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+              sts128(stage + row_off + (((uint32_t)i ^ swz) << 4),
+                     make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]));
           }
+          fence_proxy_async_smem();           // the writes are visible to the TMA store
+          named_bar_sync(1, 32 * TC_EPI_WARPS);
+          if (leader && tile_ok) {
+            // Rows past the last frame fall outside the tensor map and are dropped.
+            tma_store_3d(&tmy, stage, slab * pl.NJ + c0, fb * TC_M, p);
+            bulk_commit();
+          }
+          ob ^= 1;
         }
         tc_fence_before();
         __syncwarp();
@@ -467,6 +500,7 @@ __global__ void __launch_bounds__(TC_THREADS + (NORM ? 128 : 0), 1)
         if (++buf == pl.n_acc) { buf = 0; pacc ^= 1; }
       }
     }
+    if (leader) bulk_wait_all();                 // every output chunk has reached global memory
   }
   tc_fence_before();
   __syncthreads();
@@ -526,8 +560,8 @@ bool temporal_conv_tc_norm_ok(int F, int P, int C, int k) {
 }
 
 template <bool PAIR, bool NORM>
-static int tc_launch(const CUtensorMap& tmx, const CUtensorMap& tmw, const TcPlan& pl,
-                     const TcArgs& a, cudaStream_t stream) {
+static int tc_launch(const CUtensorMap& tmx, const CUtensorMap& tmw, const CUtensorMap& tmy,
+                     const TcPlan& pl, const TcArgs& a, cudaStream_t stream) {
   static std::mutex mu;
   static bool attr_done[64] = {false};
   int dev = 0;
@@ -568,7 +602,7 @@ static int tc_launch(const CUtensorMap& tmx, const CUtensorMap& tmw, const TcPla
     if (grid > pl.n_jobs) grid = pl.n_jobs;
   }
   cfg.gridDim = dim3((unsigned)grid);
-  VI_CUDA_TRY(cudaLaunchKernelEx(&cfg, temporal_conv_tc_kernel<PAIR, NORM>, tmx, tmw, pl, a));
+  VI_CUDA_TRY(cudaLaunchKernelEx(&cfg, temporal_conv_tc_kernel<PAIR, NORM>, tmx, tmw, tmy, pl, a));
   note_launch();
   return VI_OK;
 }
@@ -592,7 +626,16 @@ int temporal_conv_bf16_tc(const bf16* x, const bf16* w, const bf16* b, bf16* y, 
   unsigned int* err = device_error_word();
   if (!err) return VI_ERR_CUDA;
   // x as [P][F][C]: box of 64 channels x a_rows frames x 1 position, 128B swizzle.
-  CUtensorMap tmx, tmw;
+  CUtensorMap tmx, tmw, tmy;
+  {
+    // y as [P][F][C]: box of 32 channels x 128 frames x 1 position, 64B swizzle.
+    const uint64_t dims[3] = {(uint64_t)C, (uint64_t)F, (uint64_t)P};
+    const uint64_t strides[2] = {(uint64_t)C * 2, (uint64_t)F * C * 2};
+    const uint32_t box[3] = {32, (uint32_t)TC_M, 1};
+    if (!encode_tmap(&tmy, y, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_64B,
+                     CU_TENSOR_MAP_DATA_TYPE_BFLOAT16))
+      return VI_ERR_CUDA;
+  }
   {
     const uint64_t dims[3] = {(uint64_t)C, (uint64_t)F, (uint64_t)P};
     const uint64_t strides[2] = {(uint64_t)C * 2, (uint64_t)F * C * 2};
@@ -624,9 +667,9 @@ int temporal_conv_bf16_tc(const bf16* x, const bf16* w, const bf16* b, bf16* y, 
   }
   if (st == VI_OK) {
     TcArgs a{coef, b, y, err};
-    st = norm ? tc_launch<false, true>(tmx, tmw, pl, a, stream)
-              : pair ? tc_launch<true, false>(tmx, tmw, pl, a, stream)
-                     : tc_launch<false, false>(tmx, tmw, pl, a, stream);
+    st = norm ? tc_launch<false, true>(tmx, tmw, tmy, pl, a, stream)
+              : pair ? tc_launch<true, false>(tmx, tmw, tmy, pl, a, stream)
+                     : tc_launch<false, false>(tmx, tmw, tmy, pl, a, stream);
   }
   if (scratch_free(wpk, stream) != cudaSuccess && st == VI_OK) st = VI_ERR_CUDA;
   return st;
