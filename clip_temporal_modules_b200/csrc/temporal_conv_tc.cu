@@ -125,7 +125,7 @@ static std::atomic<int> g_tc_mt_pref{0};
 static bool tc_plan(int F, int P, int C, int k, bool pair, TcPlan& pl, bool norm = false,
                     int mt = 1) {
   if (k < 1 || k % 2 == 0 || 127 + k > 256 || C % TC_KB != 0) return false;
-  if (mt != 1 && (mt != 2 || pair || norm)) return false;
+  if (mt != 1 && (mt != 2 || pair)) return false;
   const int H = pair ? 2 : 1;
   const int n_acc = mt + 1 > 2 ? mt + 1 : 2;
   const int a_rows = 127 + k;
@@ -222,8 +222,12 @@ __global__ void __launch_bounds__(TC_THREADS + (NORM ? 128 : 0), 1)
   for (int c = threadIdx.x; c < pl.C; c += blockDim.x) bias_s[c] = to_f32(args.bias[c]);
   if constexpr (NORM) {
     float4* coef_s = reinterpret_cast<float4*>(smem_raw + (sCoef - smem_u32(smem_raw)));
-    for (int c = threadIdx.x; c < pl.C; c += blockDim.x)
-      coef_s[c] = reinterpret_cast<const float4*>(args.coef)[c];
+    // Channel cb*64 + 8c + e sits at slot cb*64 + 8e + c: the transform threads
+    // of one quarter-warp, which hold the 8 different c of a K-block, then
+    // read 8 consecutive slots (no bank conflict).
+    for (int ch = threadIdx.x; ch < pl.C; ch += blockDim.x)
+      coef_s[(ch & ~63) + (ch & 7) * 8 + ((ch >> 3) & 7)] =
+          reinterpret_cast<const float4*>(args.coef)[ch];
   }
   if (warp == 1) {
     if constexpr (PAIR) {
@@ -402,30 +406,35 @@ __global__ void __launch_bounds__(TC_THREADS + (NORM ? 128 : 0), 1)
       int sa = 0, pa = 0;
       bool ok = true;
       for (long long job = cluster_id; job < pl.n_jobs && ok; job += n_clusters) {
-        const long long tile = (job / pl.n_slabs) * (pl.H * pl.MT) + rank;
-        const int fb = (int)(tile % pl.n_fblk);
-        const int f_first = fb * TC_M - halo;
+        const long long tile0 = (job / pl.n_slabs) * (pl.H * pl.MT) + rank;
+        int f_first[2];                            // frame of row 0 of each tile's x box
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt) f_first[mt] = (int)((tile0 + mt) % pl.n_fblk) * TC_M - halo;
         for (int ib = 0; ib < pl.n_cb && ok; ++ib) {
           const int cb = (ib + cb_rot) % pl.n_cb;
           float m[8], a[8], bt[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            const float4 k4 = coef_s[cb * TC_KB + c * 8 + e];
+            const float4 k4 = coef_s[cb * TC_KB + e * 8 + c];
             m[e] = k4.x; a[e] = k4.y; bt[e] = k4.z;
           }
           if (!mbar_wait_bounded(a_full + 8 * sa, (uint32_t)pa, args.err, VI_DEV_ERR_TMA_TIMEOUT)) {
             ok = false;
             break;
           }
-          uint4* st = stage0 + (size_t)sa * (pl.a_stage / 16);
-          for (int r = r0; r < pl.a_rows; r += 16) {
-            const int f = f_first + r;
-            if (f < 0 || f >= pl.F) continue;
-            float v[8];
-            unpack(st[r * 8 + pc], v);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) v[e] = fmaf(v[e] - m[e], a[e], bt[e]);
-            st[r * 8 + pc] = pack(v);
+          for (int mt = 0; mt < 2; ++mt) {
+            if (mt >= pl.MT) break;
+            uint4* st = stage0 + (size_t)sa * (pl.a_stage / 16) + (size_t)mt * (pl.a_tile / 16);
+            for (int r = r0; r < pl.a_rows; r += 16) {
+              const int f = f_first[mt] + r;
+              if (f < 0 || f >= pl.F) continue;
+              float v[8];
+              unpack(st[r * 8 + pc], v);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) v[e] = fmaf(v[e] - m[e], a[e], bt[e]);
+              st[r * 8 + pc] = pack(v);
+            }
           }
           fence_proxy_async_smem();
           __syncwarp();
@@ -621,7 +630,7 @@ int temporal_conv_bf16_tc(const bf16* x, const bf16* w, const bf16* b, bf16* y, 
     const int pref = g_tc_mt_pref.load(std::memory_order_relaxed);
     const int mt = pref > 0 ? pref : TC_MT_DEFAULT;
     TcPlan pl2;
-    if (mt == 2 && !norm && tc_plan(F, P, C, k, false, pl2, false, 2) && pl2.NJ >= pl.NJ) pl = pl2;
+    if (mt == 2 && tc_plan(F, P, C, k, false, pl2, norm, 2) && pl2.NJ >= pl.NJ) pl = pl2;
   }
   unsigned int* err = device_error_word();
   if (!err) return VI_ERR_CUDA;

@@ -81,3 +81,17 @@ def test_unsupported_channel_count_is_reported(cuda_device):
     with pytest.raises(vi.ViError) as e:
         vi.groupnorm_conv(x, g, bt, wt, b, N=w.N, groups=w.groups)
     assert e.value.status == -3
+
+
+@pytest.mark.parametrize("tiles", [1, 2])
+@pytest.mark.parametrize("w", [W("gnconv_F48_C64_G8_odd_tiles", 48, 3, 5, 64, 8),
+                               W("gnconv_F200_C320_G32_ragged", 200, 8, 3, 320, 32)],
+                         ids=lambda w: w.name)
+def test_one_and_two_tiles_per_job(cuda_device, w, tiles):
+    """Both job forms of the fused conv (the transform warps normalise one or
+    two x boxes per stage)."""
+    prev = vi.set_conv_tiles_per_job(tiles)
+    try:
+        run_case(w)
+    finally:
+        vi.set_conv_tiles_per_job(prev)
