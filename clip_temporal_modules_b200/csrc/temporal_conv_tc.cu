@@ -247,6 +247,9 @@ __global__ void __launch_bounds__(TC_THREADS + (NORM ? 128 : 0), 1)
 
   const int halo = pl.k / 2;
   const int cb_rot = (int)(cluster_id % pl.n_cb);
+  // Equal x and w rings (the two-tile form): one barrier pair per stage covers
+  // both, so a K-block costs one wait and one commit.
+  const bool uni = !PAIR && pl.sa == pl.sb;
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -273,27 +276,33 @@ __global__ void __launch_bounds__(TC_THREADS + (NORM ? 128 : 0), 1)
           if (a_used && !tc_wait<PAIR>(a_empty + 8 * sa, (uint32_t)(pa ^ 1), args.err,
                                        VI_DEV_ERR_TMA_TIMEOUT)) { ok = false; break; }
           const uint32_t dst = sA + sa * pl.a_stage;
+          const uint32_t a_bar = a_full + 8 * sa;
           if constexpr (PAIR) {
             mbar_arrive_expect_tx_cluster(lead_a_full + 8 * sa, (uint32_t)pl.a_rows * 128u);
             tma_load_3d_pair(dst, &tmx, cb * TC_KB, frow[0], pos[0], lead_a_full + 8 * sa);
           } else {
-            mbar_arrive_expect_tx(a_full + 8 * sa, (uint32_t)(pl.MT * pl.a_rows) * 128u);
-            tma_load_3d(dst, &tmx, cb * TC_KB, frow[0], pos[0], a_full + 8 * sa);
+            mbar_arrive_expect_tx(a_bar, (uint32_t)(pl.MT * pl.a_rows) * 128u +
+                                             (uni ? (uint32_t)pl.b_stage : 0u));
+            tma_load_3d(dst, &tmx, cb * TC_KB, frow[0], pos[0], a_bar);
             if (pl.MT == 2)
-              tma_load_3d(dst + pl.a_tile, &tmx, cb * TC_KB, frow[1], pos[1], a_full + 8 * sa);
+              tma_load_3d(dst + pl.a_tile, &tmx, cb * TC_KB, frow[1], pos[1], a_bar);
           }
           if (++sa == pl.sa) { sa = 0; pa ^= 1; a_used = true; }
           // One B stage = this CTA's weight blocks of every tap of K-block cb.
-          if (b_used && !tc_wait<PAIR>(b_empty + 8 * sbi, (uint32_t)(pb ^ 1), args.err,
-                                       VI_DEV_ERR_TMA_TIMEOUT)) { ok = false; break; }
-          if constexpr (PAIR) mbar_arrive_expect_tx_cluster(lead_b_full + 8 * sbi, (uint32_t)pl.b_stage);
-          else mbar_arrive_expect_tx(b_full + 8 * sbi, (uint32_t)pl.b_stage);
+          uint32_t b_bar = a_bar;                  // shared stage: same barrier as x
+          if (!uni) {
+            if (b_used && !tc_wait<PAIR>(b_empty + 8 * sbi, (uint32_t)(pb ^ 1), args.err,
+                                         VI_DEV_ERR_TMA_TIMEOUT)) { ok = false; break; }
+            b_bar = PAIR ? lead_b_full + 8 * sbi : b_full + 8 * sbi;
+            if constexpr (PAIR) mbar_arrive_expect_tx_cluster(b_bar, (uint32_t)pl.b_stage);
+            else mbar_arrive_expect_tx(b_bar, (uint32_t)pl.b_stage);
+          }
           for (int t = 0; t < pl.k; ++t) {
             // Row of this CTA's weight block in the packed [..][128 B] view.
             const int row = wrow + cb * wrow_cb + t * wrow_t;
             const uint32_t dstb = sB + sbi * pl.b_stage + t * pl.b_tap;
-            if constexpr (PAIR) tma_load_2d_pair(dstb, &tmw, 0, row, lead_b_full + 8 * sbi);
-            else tma_load_2d(dstb, &tmw, 0, row, b_full + 8 * sbi);
+            if constexpr (PAIR) tma_load_2d_pair(dstb, &tmw, 0, row, b_bar);
+            else tma_load_2d(dstb, &tmw, 0, row, b_bar);
           }
           if (++sbi == pl.sb) { sbi = 0; pb ^= 1; b_used = true; }
         }
@@ -328,7 +337,8 @@ __global__ void __launch_bounds__(TC_THREADS + (NORM ? 128 : 0), 1)
         for (int ib = 0; ib < pl.n_cb && ok; ++ib) {
           if (!tc_wait<PAIR>((NORM ? a_ready : a_full) + 8 * sa, (uint32_t)pa, args.err,
                              VI_DEV_ERR_TMA_TIMEOUT) ||
-              !tc_wait<PAIR>(b_full + 8 * sbi, (uint32_t)pb, args.err, VI_DEV_ERR_TMA_TIMEOUT)) {
+              (!uni &&
+               !tc_wait<PAIR>(b_full + 8 * sbi, (uint32_t)pb, args.err, VI_DEV_ERR_TMA_TIMEOUT))) {
             ok = false;
             break;
           }
@@ -377,8 +387,8 @@ __global__ void __launch_bounds__(TC_THREADS + (NORM ? 128 : 0), 1)
             umma_commit_pair_mc(b_empty + 8 * sbi, 0x3);
             umma_commit_pair_mc(a_empty + 8 * sa, 0x3);
           } else {
-            umma_commit(b_empty + 8 * sbi);       // frees the w stage when these MMAs finish
-            umma_commit(a_empty + 8 * sa);        // frees the x stage
+            if (!uni) umma_commit(b_empty + 8 * sbi);   // frees the w stage when these MMAs finish
+            umma_commit(a_empty + 8 * sa);        // frees the x stage (and the w stage if shared)
           }
           if (++sbi == pl.sb) { sbi = 0; pb ^= 1; }
           if (++sa == pl.sa) { sa = 0; pa ^= 1; }
@@ -476,7 +486,7 @@ __global__ void __launch_bounds__(TC_THREADS + (NORM ? 128 : 0), 1)
         for (int c0 = 0; c0 < pl.NJ; c0 += 32) {
           uint32_t r[32];
           tmem_ld32(tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * pl.NJ + c0), r);
-          tmem_wait_ld();
+          tmem_wait_ld_dep(r);
           const uint32_t stage = sOut + (uint32_t)ob * TC_OUT_CHUNK;
           if (leader) bulk_wait_read_le1();   // the store that last read this buffer is done
           named_bar_sync(1, 32 * TC_EPI_WARPS);
