@@ -50,6 +50,8 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-chunks", type=int, default=16,
+                    help="position chunks of the end-to-end pipeline")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
@@ -431,43 +433,39 @@ def attention_module(w, d, out, y, z, stream, reps=5):
 
 
 def run_e2e(args, w, host, dev, stream):
-    """Same step through host buffers: H2D of every input, 3 kernels, D2H of every output."""
+    """Same step from and to pinned host buffers, through the package's
+    HostPipeline: copy-in, compute and copy-out streams over position chunks."""
     import torch
 
     import clip_temporal_modules_b200 as vi
     world, _, _ = dist_env()
     res = {k: torch.empty_like(host["q"]).pin_memory() for k in ("out", "y", "z")}
-    d = {}
+    shape = vi.StepShape(F=w.F, N=w.N, P=w.P, C=w.C, heads=w.heads, n_pre=w.n_pre,
+                         n_post=w.n_post, n_global=w.n_global, k=w.k, groups=w.groups, eps=w.eps)
+    pipe = vi.HostPipeline(shape, dev, host["q"].dtype, chunks=args.e2e_chunks)
 
-    def e2e_step():
-        for k_, v_ in host.items():
-            d[k_] = v_.to(dev, non_blocking=True)
-        o = vi.dual_attn(d["q"], d["k"], d["v"], N=w.N, heads=w.heads, n_pre=w.n_pre,
-                         n_post=w.n_post, n_global=w.n_global)
-        yy = vi.temporal_conv(d["conv_x"], d["conv_w"], d["conv_b"], N=w.N)
-        zz = vi.groupnorm_global(d["gn_x"], d["gn_gamma"], d["gn_beta"], N=w.N, groups=w.groups,
-                                 eps=w.eps)
-        res["out"].copy_(o, non_blocking=True)
-        res["y"].copy_(yy, non_blocking=True)
-        res["z"].copy_(zz, non_blocking=True)
-
-    e2e_step()
+    pipe.run(host, res)
     torch.cuda.synchronize()
     barrier(dev)
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
     for _ in range(args.e2e_steps):
-        e2e_step()
+        pipe.run(host, res)
     b.record(stream)
     torch.cuda.synchronize()
     ms = max_over_ranks(a.elapsed_time(b), dev)
     barrier(dev)
-    h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = sum(t.numel() * t.element_size() for t in res.values())
+    del pipe
     return {"value": round(w.tokens * world * args.e2e_steps / (ms / 1e3), 1), "unit": "tokens/s",
-            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "h2d_bytes_per_step": vi.HostPipeline.h2d_bytes(host),
+            "d2h_bytes_per_step": vi.HostPipeline.d2h_bytes(res),
             "steps": args.e2e_steps, "ms_per_step": round(ms / args.e2e_steps, 3),
-            "path": "pinned host -> cudaMemcpyAsync -> libvi C ABI x3 -> pinned host"}
+            "path": f"pinned host -> HostPipeline ({pipe_desc(args.e2e_chunks)}) -> libvi C ABI"
+                    " -> pinned host"}
+
+
+def pipe_desc(chunks: int) -> str:
+    return f"copy-in / compute / copy-out streams, {chunks} position chunks"
 
 
 def load_traffic(kernel, w):

@@ -18,7 +18,8 @@ Python here only marshals arguments; see _binding.py.
 from ._binding import (LIB_PATH, ViError, dual_attn, groupnorm_conv,  # noqa: F401
                        groupnorm_global, launch_count, lib, set_conv_tiles_per_job,
                        take_device_errors, temporal_attention, temporal_conv)
+from .host_pipeline import HostPipeline, StepShape  # noqa: F401
 
 __all__ = ["dual_attn", "temporal_conv", "groupnorm_global", "groupnorm_conv", "temporal_attention", "take_device_errors", "launch_count", "lib",
-           "set_conv_tiles_per_job",
+           "set_conv_tiles_per_job", "HostPipeline", "StepShape",
            "ViError", "LIB_PATH"]
