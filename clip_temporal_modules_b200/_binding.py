@@ -95,6 +95,13 @@ def _dev(*ts):
         raise TypeError("all tensors of one call share a dtype")
 
 
+def _shape(t, shape, what: str) -> None:
+    """The C ABI takes sizes, not shapes: a tensor smaller than the sizes say
+    would be read or written out of bounds, so shapes are checked here."""
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{what}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
 def dual_attn(q, k, v, out=None, *, N: int, heads: int, n_pre: int = 8, n_post: int = 8,
               n_global: int = 16, stream=None):
     """Dual-domain temporal attention; q, k, v, out are [P][F][heads*d] CUDA tensors."""
@@ -103,6 +110,8 @@ def dual_attn(q, k, v, out=None, *, N: int, heads: int, n_pre: int = 8, n_post: 
         out = torch.empty_like(q)
     _dev(q, k, v, out)
     P, F, C = q.shape
+    for t, n in ((k, "k"), (v, "v"), (out, "out")):
+        _shape(t, q.shape, n)
     name = "vi_dual_attn" + _suffix(q)
     _check(name, getattr(lib(), name)(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
                                       F, N, P, heads, C // heads, n_pre, n_post, n_global,
@@ -117,7 +126,12 @@ def temporal_conv(x, w, b, out=None, *, N: int, stream=None):
         out = torch.empty_like(x)
     _dev(x, w, b, out)
     P, F, C = x.shape
+    if w.dim() != 3:
+        raise ValueError("w: expected [C_out][C_in][k]")
     k = w.shape[2]
+    _shape(w, (C, C, k), "w")
+    _shape(b, (C,), "b")
+    _shape(out, x.shape, "out")
     name = "vi_temporal_conv" + _suffix(x)
     _check(name, getattr(lib(), name)(x.data_ptr(), w.data_ptr(), b.data_ptr(), out.data_ptr(),
                                       F, N, P, C, k, _stream_ptr(stream)))
@@ -132,6 +146,9 @@ def groupnorm_global(x, gamma, beta, out=None, *, N: int, groups: int, eps: floa
         out = torch.empty_like(x)
     _dev(x, gamma, beta, out)
     P, F, C = x.shape
+    _shape(gamma, (C,), "gamma")
+    _shape(beta, (C,), "beta")
+    _shape(out, x.shape, "out")
     name = "vi_groupnorm_global" + _suffix(x)
     _check(name, getattr(lib(), name)(x.data_ptr(), gamma.data_ptr(), beta.data_ptr(),
                                       out.data_ptr(), F, N, P, C, groups, float(eps),
@@ -147,6 +164,12 @@ def groupnorm_conv(x, gamma, beta, w, b, out=None, *, N: int, groups: int, eps: 
         out = torch.empty_like(x)
     _dev(x, gamma, beta, w, b, out)
     P, F, C = x.shape
+    if w.dim() != 3:
+        raise ValueError("w: expected [C_out][C_in][k]")
+    _shape(w, (C, C, w.shape[2]), "w")
+    for t, n in ((gamma, "gamma"), (beta, "beta"), (b, "b")):
+        _shape(t, (C,), n)
+    _shape(out, x.shape, "out")
     _check("vi_groupnorm_conv", lib().vi_groupnorm_conv(
         x.data_ptr(), gamma.data_ptr(), beta.data_ptr(), w.data_ptr(), b.data_ptr(),
         out.data_ptr(), F, N, P, C, groups, float(eps), w.shape[2], _stream_ptr(stream)))
@@ -166,6 +189,13 @@ def temporal_attention(x, w_qkv, b_qkv, w_out, b_out, out=None, workspace=None, 
         n = int(lib().vi_temporal_attention_workspace_bytes(F, P, C))
         workspace = torch.empty(n // 2, dtype=torch.bfloat16, device=x.device)
     _dev(x, w_qkv, b_qkv, w_out, b_out, out, workspace)
+    _shape(w_qkv, (3 * C, C), "w_qkv")
+    _shape(b_qkv, (3 * C,), "b_qkv")
+    _shape(w_out, (C, C), "w_out")
+    _shape(b_out, (C,), "b_out")
+    _shape(out, x.shape, "out")
+    if workspace.numel() * workspace.element_size() < 4 * P * F * C * 2:
+        raise ValueError("workspace: smaller than vi_temporal_attention_workspace_bytes")
     _check("vi_temporal_attention", lib().vi_temporal_attention(
         x.data_ptr(), w_qkv.data_ptr(), b_qkv.data_ptr(), w_out.data_ptr(), b_out.data_ptr(),
         out.data_ptr(), workspace.data_ptr(), F, N, P, heads, C // heads, n_pre, n_post, n_global,

@@ -597,12 +597,13 @@ extern "C" int vi_groupnorm_global_noalloc(const void* x, const void* gamma, con
   using namespace vi;
   using T = bf16;
   // The argument checks of vi_groupnorm_global.
-  if (!x || !gamma || !beta || !y) return VI_ERR_INVALID_ARG;
-  if (F <= 0 || N <= 0 || P <= 0 || C <= 0 || F % N != 0) return VI_ERR_INVALID_ARG;
+  if (F <= 0 || N <= 0 || P < 0 || C <= 0 || F % N != 0) return VI_ERR_INVALID_ARG;
   if ((double)P * (double)F * (double)C > 1.099511627776e12) return VI_ERR_UNSUPPORTED;
   if (groups <= 0 || C % groups != 0) return VI_ERR_INVALID_ARG;
   if (!(eps >= 0.f) || !isfinite(eps)) return VI_ERR_INVALID_ARG;
   if (groups > GN_MAX_GROUPS) return VI_ERR_UNSUPPORTED;
+  if (P == 0) return VI_OK;                 // no positions: nothing to read or write
+  if (!x || !gamma || !beta || !y) return VI_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(gamma) || !aligned16(beta) || !aligned16(y))
     return VI_ERR_ALIGNMENT;
   if ((C * sizeof(T)) % 16 != 0) return VI_ERR_ALIGNMENT;

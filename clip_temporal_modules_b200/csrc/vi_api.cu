@@ -142,10 +142,14 @@ namespace {
 
 inline cudaStream_t as_stream(vi_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
 
-// Sizes shared by all three calls.
+// A valid call with no positions (P == 0): nothing to compute or read.
+constexpr int kEmpty = 1;
+
+// Sizes shared by all the calls: VI_OK, kEmpty, or a negative status.
 int check_clips(int F, int N, int P, int C) {
-  if (F <= 0 || N <= 0 || P <= 0 || C <= 0) return VI_ERR_INVALID_ARG;
+  if (F <= 0 || N <= 0 || P < 0 || C <= 0) return VI_ERR_INVALID_ARG;
   if (F % N != 0) return VI_ERR_INVALID_ARG;
+  if (P == 0) return kEmpty;
   // Element offsets are 64-bit; cap the tensor at 2^40 elements.
   if ((double)P * (double)F * (double)C > 1.099511627776e12) return VI_ERR_UNSUPPORTED;
   return VI_OK;
@@ -154,16 +158,17 @@ int check_clips(int F, int N, int P, int C) {
 template <typename T>
 int attn_entry(const void* q, const void* k, const void* v, void* out, int F, int N, int P,
                int heads, int d, int n_pre, int n_post, int n_global, vi_stream_t stream) {
-  if (!q || !k || !v || !out) return VI_ERR_INVALID_ARG;
   if (heads <= 0 || d <= 0) return VI_ERR_INVALID_ARG;
   if ((int64_t)heads * d > 0x7fffffff) return VI_ERR_INVALID_ARG;
   const int C = heads * d;
   int st = check_clips(F, N, P, C);
-  if (st != VI_OK) return st;
+  if (st < 0) return st;
   const int L = F / N;
   if (n_pre < 0 || n_post < 0 || n_global < 0 || n_global > F) return VI_ERR_INVALID_ARG;
   if (N > 1 && (n_pre > L || n_post > L)) return VI_ERR_INVALID_ARG;
   if (d != 64) return VI_ERR_UNSUPPORTED;
+  if (st == kEmpty) return VI_OK;
+  if (!q || !k || !v || !out) return VI_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
     return VI_ERR_ALIGNMENT;
   if ((C * sizeof(T)) % 16 != 0) return VI_ERR_ALIGNMENT;
@@ -187,10 +192,11 @@ int attn_entry(const void* q, const void* k, const void* v, void* out, int F, in
 template <typename T>
 int conv_entry(const void* x, const void* w, const void* b, void* y, int F, int N, int P, int C,
                int k, vi_stream_t stream) {
-  if (!x || !w || !b || !y) return VI_ERR_INVALID_ARG;
   int st = check_clips(F, N, P, C);
-  if (st != VI_OK) return st;
+  if (st < 0) return st;
   if (k <= 0 || k % 2 == 0 || k / 2 > F / N) return VI_ERR_INVALID_ARG;
+  if (st == kEmpty) return VI_OK;
+  if (!x || !w || !b || !y) return VI_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(w) || !aligned16(b) || !aligned16(y)) return VI_ERR_ALIGNMENT;
   if ((C * sizeof(T)) % 16 != 0) return VI_ERR_ALIGNMENT;
   const size_t bytes = (size_t)P * F * C * sizeof(T);
@@ -211,12 +217,13 @@ int conv_entry(const void* x, const void* w, const void* b, void* y, int F, int 
 template <typename T>
 int gn_entry(const void* x, const void* gamma, const void* beta, void* y, int F, int N, int P,
              int C, int groups, float eps, vi_stream_t stream) {
-  if (!x || !gamma || !beta || !y) return VI_ERR_INVALID_ARG;
   int st = check_clips(F, N, P, C);
-  if (st != VI_OK) return st;
+  if (st < 0) return st;
   if (groups <= 0 || C % groups != 0) return VI_ERR_INVALID_ARG;
   if (!(eps >= 0.f) || !isfinite(eps)) return VI_ERR_INVALID_ARG;
   if (groups > 1024) return VI_ERR_UNSUPPORTED;
+  if (st == kEmpty) return VI_OK;
+  if (!x || !gamma || !beta || !y) return VI_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(gamma) || !aligned16(beta) || !aligned16(y))
     return VI_ERR_ALIGNMENT;
   if ((C * sizeof(T)) % 16 != 0) return VI_ERR_ALIGNMENT;
@@ -233,13 +240,14 @@ int gn_conv_entry(const void* x, const void* gamma, const void* beta, const void
                   const void* b, void* y, int F, int N, int P, int C, int groups, float eps, int k,
                   vi_stream_t stream) {
   using T = bf16;
-  if (!x || !gamma || !beta || !w || !b || !y) return VI_ERR_INVALID_ARG;
   int st = check_clips(F, N, P, C);
-  if (st != VI_OK) return st;
+  if (st < 0) return st;
   if (groups <= 0 || C % groups != 0) return VI_ERR_INVALID_ARG;
   if (!(eps >= 0.f) || !isfinite(eps)) return VI_ERR_INVALID_ARG;
   if (k <= 0 || k % 2 == 0 || k / 2 > F / N) return VI_ERR_INVALID_ARG;
   if (groups > 1024) return VI_ERR_UNSUPPORTED;
+  if (st == kEmpty) return VI_OK;
+  if (!x || !gamma || !beta || !w || !b || !y) return VI_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(gamma) || !aligned16(beta) || !aligned16(w) || !aligned16(b) ||
       !aligned16(y))
     return VI_ERR_ALIGNMENT;
@@ -271,15 +279,17 @@ int temporal_attention_entry(const void* x, const void* w_qkv, const void* b_qkv
                              int F, int N, int P, int heads, int d, int n_pre, int n_post,
                              int n_global, vi_stream_t stream) {
   using T = bf16;
-  if (!x || !w_qkv || !b_qkv || !w_out || !b_out || !out || !workspace) return VI_ERR_INVALID_ARG;
   if (heads <= 0 || d <= 0 || (int64_t)heads * d > 0x7fffffff) return VI_ERR_INVALID_ARG;
   const int C = heads * d;
   int st = check_clips(F, N, P, C);
-  if (st != VI_OK) return st;
+  if (st < 0) return st;
   const int L = F / N;
   if (n_pre < 0 || n_post < 0 || n_global < 0 || n_global > F) return VI_ERR_INVALID_ARG;
   if (N > 1 && (n_pre > L || n_post > L)) return VI_ERR_INVALID_ARG;
   if (d != 64) return VI_ERR_UNSUPPORTED;
+  if (st == kEmpty) return VI_OK;
+  st = VI_OK;
+  if (!x || !w_qkv || !b_qkv || !w_out || !b_out || !out || !workspace) return VI_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(w_qkv) || !aligned16(b_qkv) || !aligned16(w_out) ||
       !aligned16(b_out) || !aligned16(out) || !aligned16(workspace))
     return VI_ERR_ALIGNMENT;

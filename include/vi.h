@@ -32,6 +32,10 @@
  *   cudaFreeAsync); the pool keeps up to 64 MiB of freed memory mapped so
  *   later calls reuse it.  Calls on different streams may run concurrently;
  *   calls on one stream run in order.
+ * Empty calls.  P == 0 (no positions) is a valid call with nothing to
+ *   compute: once the scalar arguments pass their checks it returns VI_OK,
+ *   enqueues nothing and reads no pointer (they may be NULL).  F, N, C and the
+ *   other sizes must still be positive.
  * Errors.  Every argument is checked on the host before anything is launched;
  *   a failed check returns a negative vi_status and enqueues nothing.
  *   VI_ERR_CUDA reports a CUDA error seen while launching.  A fault that
@@ -115,7 +119,7 @@ int vi_set_conv_tiles_per_job(int tiles);
  *
  * q, k, v, out : [P][F][heads*d] (bf16, or fp32 for _f32); out must not
  *                overlap q, k or v.
- * Requirements : all sizes > 0 except the context sizes (>= 0); F % N == 0;
+ * Requirements : all sizes > 0 except P (>= 0) and the context sizes (>= 0); F % N == 0;
  *                d == 64; if N > 1 then n_pre <= L and n_post <= L;
  *                n_global <= F.  Otherwise VI_ERR_INVALID_ARG, or
  *                VI_ERR_UNSUPPORTED for d != 64.
@@ -138,7 +142,7 @@ int vi_dual_attn_f32(const void* q, const void* k, const void* v, void* out, int
  * zero-padded Conv1d of the whole video, and does not depend on N.
  *
  * x, y : [P][F][C];  w : [C_out=C][C_in=C][k] (PyTorch Conv1d order);  b : [C].
- * Requirements : sizes > 0; F % N == 0; k odd; k/2 <= L; y must not overlap
+ * Requirements : sizes > 0 (P >= 0); F % N == 0; k odd; k/2 <= L; y must not overlap
  *                x, w or b.  Otherwise VI_ERR_INVALID_ARG.
  * Scratch      : the bf16 path repacks w into a stream-ordered scratch buffer
  *                of k*C*C*2 bytes (library pool), freed on the stream after
@@ -160,7 +164,7 @@ int vi_temporal_conv_f32(const void* x, const void* w, const void* b, void* y, i
  * which equals GroupNorm (batch 1) of the unpartitioned latent for any N.
  *
  * x, y : [P][F][C] (y may equal x: in place);  gamma, beta : [C].
- * Requirements : sizes > 0; F % N == 0; C % groups == 0; eps >= 0 and finite.
+ * Requirements : sizes > 0 (P >= 0); F % N == 0; C % groups == 0; eps >= 0 and finite.
  *                y may alias x exactly but must not partly overlap it.
  * Scratch      : (24 * groups * blocks + 16*C + 16*groups + 64) bytes of stream-ordered
  *                scratch (library pool) for per-block partial sums and the

@@ -172,3 +172,39 @@ def test_conv_tiles_per_job_knob(L):
     assert prev in (0, 1, 2)
     assert L.vi_set_conv_tiles_per_job(2) == 1
     assert L.vi_set_conv_tiles_per_job(prev) == 2
+
+
+def test_empty_calls_succeed_without_touching_pointers(L):
+    """P == 0: valid, nothing to compute; NULL pointers are fine and nothing is
+    launched (no device here, so any CUDA call would have failed)."""
+    n0 = vi.launch_count()
+    assert attn(L, q=None, k=None, v=None, o=None, P=0) == OK
+    assert attn(L, q=None, k=None, v=None, o=None, P=0, f32=True) == OK
+    assert conv(L, x=None, w=None, b=None, y=None, P=0) == OK
+    assert gn(L, x=None, g=None, bt=None, y=None, P=0) == OK
+    assert gnconv(L, x=None, g=None, bt=None, w=None, b=None, y=None, P=0) == OK
+    assert tattn(L, x=None, wqkv=None, bqkv=None, wo=None, bo=None, out=None, ws=None, P=0) == OK
+    assert L.vi_groupnorm_global_noalloc(None, None, None, None, 64, 4, 0, 64, 8, 1e-5, None) == OK
+    assert vi.launch_count() == n0
+
+
+@pytest.mark.parametrize("call,expect", [
+    (lambda L: attn(L, P=0, F=0), INVALID), (lambda L: attn(L, P=0, d=32), UNSUP),
+    (lambda L: attn(L, P=0, pre=17), INVALID), (lambda L: conv(L, P=0, k=2), INVALID),
+    (lambda L: gn(L, P=0, groups=7), INVALID), (lambda L: gnconv(L, P=0, N=3), INVALID),
+    (lambda L: tattn(L, P=0, heads=0), INVALID),
+])
+def test_empty_calls_still_check_scalar_arguments(L, call, expect):
+    assert call(L) == expect
+
+
+def test_binding_checks_shapes_before_the_call():
+    """Sizes come from the first tensor; the others must match it (a smaller
+    tensor would be read out of bounds by the kernel)."""
+    import torch
+    from clip_temporal_modules_b200._binding import _shape
+    _shape(torch.empty(2, 3, 4), (2, 3, 4), "x")
+    with pytest.raises(ValueError):
+        _shape(torch.empty(2, 3, 4), (2, 3, 5), "x")
+    with pytest.raises(ValueError):
+        _shape(torch.empty(12), (3, 4), "w")
