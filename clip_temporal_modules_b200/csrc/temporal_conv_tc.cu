@@ -90,6 +90,8 @@ struct TcPlan {
   int NJ;                // output channels per job (UMMA N), multiple of 32
   int H;                 // CTAs per MMA (1, or 2 for a pair); each holds NJ/H weight rows
   int MT;                // tiles per job per CTA (1, or 2 sharing every weight stage)
+  int KS;                // K-blocks per pipeline stage (1, or 2 for single-tap convs)
+  int n_stage;           // stages per job = ceil(n_cb / KS)
   int n_acc;             // TMEM accumulators in the ring (MT + 1, at least 2), NJ columns each
   int n_slabs;           // C / NJ
   int n_fblk;            // ceil(F / 128)
@@ -98,10 +100,11 @@ struct TcPlan {
   int n_cb;              // C / 64
   int a_rows;            // 127 + k
   int a_tile;            // bytes of one tile's x box (a_rows x 128 B), 1024-aligned
-  int a_stage;           // bytes per A stage = MT * a_tile
+  int a_stage;           // bytes per A stage = KS * MT * a_tile
   int b_rows;            // weight rows per CTA per tap = NJ / H
   int b_tap;             // bytes of one tap's block = b_rows * 128
-  int b_stage;           // bytes per B stage = k * b_tap (one K-block, all taps)
+  int b_kb;              // weight bytes of one K-block = k * b_tap (all taps)
+  int b_stage;           // bytes per B stage = KS * b_kb
   int sa;                // A stages
   int sb;                // B stages
   int smem;              // dynamic shared memory bytes
@@ -123,14 +126,15 @@ static int g_tc_sb_pref = 0, g_tc_sa_pref = 0;
 static std::atomic<int> g_tc_mt_pref{0};
 
 static bool tc_plan(int F, int P, int C, int k, bool pair, TcPlan& pl, bool norm = false,
-                    int mt = 1) {
+                    int mt = 1, int ks = 1) {
   if (k < 1 || k % 2 == 0 || 127 + k > 256 || C % TC_KB != 0) return false;
   if (mt != 1 && (mt != 2 || pair)) return false;
+  if (ks != 1 && (ks != 2 || pair || norm)) return false;
   const int H = pair ? 2 : 1;
   const int n_acc = mt + 1 > 2 ? mt + 1 : 2;
   const int a_rows = 127 + k;
   const int a_tile = ((a_rows * 128 + 1023) / 1024) * 1024;
-  const int a_stage = mt * a_tile;
+  const int a_stage = ks * mt * a_tile;
   const int fixed = 1024 /* align slack */ + 2 * TC_OUT_CHUNK /* output staging */ + 4 * C +
                     64 /* bias, padded */ + 512 /* bars */ +
                     (norm ? 16 * C : 0) /* GroupNorm coefficients */;
@@ -138,7 +142,7 @@ static bool tc_plan(int F, int P, int C, int k, bool pair, TcPlan& pl, bool norm
   // all-tap weight stages leave room for at least two of each ring.
   for (int nj = TC_NJ_MAX; nj >= 32; nj -= 32) {
     if (C % nj != 0 || (nj / H) % 8 != 0 || n_acc * nj > TC_TMEM_COLS) continue;
-    const int b_stage = k * (nj / H) * 128;
+    const int b_stage = ks * k * (nj / H) * 128;
     const bool few_k = C <= 640 || norm;
     int sa = g_tc_sa_pref > 0 ? g_tc_sa_pref : (mt == 2 ? 2 : few_k ? 3 : 2);
     if (sa > TC_SA_MAX) sa = TC_SA_MAX;
@@ -155,17 +159,20 @@ static bool tc_plan(int F, int P, int C, int k, bool pair, TcPlan& pl, bool norm
     pl.NJ = nj;
     pl.H = H;
     pl.MT = mt;
+    pl.KS = ks;
     pl.n_acc = n_acc;
     pl.n_slabs = C / nj;
     pl.n_fblk = (F + TC_M - 1) / TC_M;
     pl.n_tiles = (long long)P * pl.n_fblk;
     pl.n_jobs = ((pl.n_tiles + H * mt - 1) / (H * mt)) * pl.n_slabs;
     pl.n_cb = C / TC_KB;
+    pl.n_stage = (pl.n_cb + ks - 1) / ks;
     pl.a_rows = a_rows;
     pl.a_tile = a_tile;
     pl.a_stage = a_stage;
     pl.b_rows = nj / H;
     pl.b_tap = pl.b_rows * 128;
+    pl.b_kb = k * pl.b_tap;
     pl.b_stage = b_stage;
     pl.sa = sa;
     pl.sb = sb;
@@ -271,38 +278,48 @@ __global__ void __launch_bounds__(TC_THREADS + (NORM ? 128 : 0), 1)
         }
         int wrow = (slab * pl.n_cb * pl.k * pl.H + (int)rank) * pl.b_rows;   // row of (slab, cb 0, t 0)
         const int wrow_cb = pl.k * pl.H * pl.b_rows, wrow_t = pl.H * pl.b_rows;
-        for (int ib = 0; ib < pl.n_cb && ok; ++ib) {
-          const int cb = (ib + cb_rot) % pl.n_cb;
+        for (int is = 0; is < pl.n_stage && ok; ++is) {
+          // Stage `is` holds K-blocks kb0 .. kb0 + nkb - 1 of the job (in the
+          // CTA's rotated order); only a job's last stage can hold fewer than KS.
+          const int kb0 = is * pl.KS;
+          const int nkb = min(pl.KS, pl.n_cb - kb0);
           if (a_used && !tc_wait<PAIR>(a_empty + 8 * sa, (uint32_t)(pa ^ 1), args.err,
                                        VI_DEV_ERR_TMA_TIMEOUT)) { ok = false; break; }
           const uint32_t dst = sA + sa * pl.a_stage;
           const uint32_t a_bar = a_full + 8 * sa;
           if constexpr (PAIR) {
+            const int cb = (kb0 + cb_rot) % pl.n_cb;
             mbar_arrive_expect_tx_cluster(lead_a_full + 8 * sa, (uint32_t)pl.a_rows * 128u);
             tma_load_3d_pair(dst, &tmx, cb * TC_KB, frow[0], pos[0], lead_a_full + 8 * sa);
           } else {
-            mbar_arrive_expect_tx(a_bar, (uint32_t)(pl.MT * pl.a_rows) * 128u +
-                                             (uni ? (uint32_t)pl.b_stage : 0u));
-            tma_load_3d(dst, &tmx, cb * TC_KB, frow[0], pos[0], a_bar);
-            if (pl.MT == 2)
-              tma_load_3d(dst + pl.a_tile, &tmx, cb * TC_KB, frow[1], pos[1], a_bar);
+            mbar_arrive_expect_tx(a_bar, (uint32_t)nkb * ((uint32_t)(pl.MT * pl.a_rows) * 128u +
+                                                          (uni ? (uint32_t)pl.b_kb : 0u)));
+            for (int kb = 0; kb < nkb; ++kb) {
+              const int cb = (kb0 + kb + cb_rot) % pl.n_cb;
+              const uint32_t d = dst + (uint32_t)(kb * pl.MT) * pl.a_tile;
+              tma_load_3d(d, &tmx, cb * TC_KB, frow[0], pos[0], a_bar);
+              if (pl.MT == 2) tma_load_3d(d + pl.a_tile, &tmx, cb * TC_KB, frow[1], pos[1], a_bar);
+            }
           }
           if (++sa == pl.sa) { sa = 0; pa ^= 1; a_used = true; }
-          // One B stage = this CTA's weight blocks of every tap of K-block cb.
+          // One B stage = this CTA's weight blocks of every tap of the stage's K-blocks.
           uint32_t b_bar = a_bar;                  // shared stage: same barrier as x
           if (!uni) {
             if (b_used && !tc_wait<PAIR>(b_empty + 8 * sbi, (uint32_t)(pb ^ 1), args.err,
                                          VI_DEV_ERR_TMA_TIMEOUT)) { ok = false; break; }
             b_bar = PAIR ? lead_b_full + 8 * sbi : b_full + 8 * sbi;
             if constexpr (PAIR) mbar_arrive_expect_tx_cluster(b_bar, (uint32_t)pl.b_stage);
-            else mbar_arrive_expect_tx(b_bar, (uint32_t)pl.b_stage);
+            else mbar_arrive_expect_tx(b_bar, (uint32_t)(nkb * pl.b_kb));
           }
-          for (int t = 0; t < pl.k; ++t) {
-            // Row of this CTA's weight block in the packed [..][128 B] view.
-            const int row = wrow + cb * wrow_cb + t * wrow_t;
-            const uint32_t dstb = sB + sbi * pl.b_stage + t * pl.b_tap;
-            if constexpr (PAIR) tma_load_2d_pair(dstb, &tmw, 0, row, b_bar);
-            else tma_load_2d(dstb, &tmw, 0, row, b_bar);
+          for (int kb = 0; kb < nkb; ++kb) {
+            const int cb = (kb0 + kb + cb_rot) % pl.n_cb;
+            for (int t = 0; t < pl.k; ++t) {
+              // Row of this CTA's weight block in the packed [..][128 B] view.
+              const int row = wrow + cb * wrow_cb + t * wrow_t;
+              const uint32_t dstb = sB + sbi * pl.b_stage + (uint32_t)(kb * pl.k + t) * pl.b_tap;
+              if constexpr (PAIR) tma_load_2d_pair(dstb, &tmw, 0, row, b_bar);
+              else tma_load_2d(dstb, &tmw, 0, row, b_bar);
+            }
           }
           if (++sbi == pl.sb) { sbi = 0; pb ^= 1; b_used = true; }
         }
@@ -334,7 +351,9 @@ __global__ void __launch_bounds__(TC_THREADS + (NORM ? 128 : 0), 1)
           js[m] = slot; jp[m] = pslot; ju[m] = slot_used;
           if (m < pl.MT && ++slot == pl.n_acc) { slot = 0; pslot ^= 1; slot_used = true; }
         }
-        for (int ib = 0; ib < pl.n_cb && ok; ++ib) {
+        for (int is = 0; is < pl.n_stage && ok; ++is) {
+          const int nkb = min(pl.KS, pl.n_cb - is * pl.KS);
+          const bool last_stage = is == pl.n_stage - 1;
           if (!tc_wait<PAIR>((NORM ? a_ready : a_full) + 8 * sa, (uint32_t)pa, args.err,
                              VI_DEV_ERR_TMA_TIMEOUT) ||
               (!uni &&
@@ -344,42 +363,47 @@ __global__ void __launch_bounds__(TC_THREADS + (NORM ? 128 : 0), 1)
           }
           tc_fence_after();
           const uint64_t bd_stage = bd_base + (uint64_t)(sbi * b_st16);
+          const uint64_t ad_stage = ad_base + (uint64_t)(sa * a_st16);
+          for (int kb = 0; kb < nkb && ok; ++kb) {
 #pragma unroll
-          for (int m = 0; m < 2; ++m) {
-            if (m >= pl.MT) break;
-            if (ib == 0) {
-              // The slot must have been drained by the epilogue of its last job.
-              if (ju[m] && !tc_wait<PAIR>(acc_empty + 8 * js[m], (uint32_t)(jp[m] ^ 1), args.err,
-                                          VI_DEV_ERR_MMA_TIMEOUT)) { ok = false; break; }
-              tc_fence_after();
-            }
-            const uint32_t d_tmem = tmem_base + (uint32_t)(js[m] * pl.NJ);
-            // k taps x 4 K steps = 4k MMAs back to back per tile (12 for k = 3;
-            // 24 per stage with two tiles): enough tensor work queued to hide
-            // the wait/commit of the next K-block.
-            const uint64_t ad_stage = ad_base + (uint64_t)(sa * a_st16 + m * at16);
-            uint32_t acc = ib > 0 ? 1u : 0u;
-            for (int t = 0; t < pl.k; ++t) {
-              // Tap t: the x tile shifted down by t rows of 128 B (8 units of 16 B).
-              const uint64_t ad = ad_stage + (uint64_t)(8u * t);
-              const uint64_t bd = bd_stage + (uint64_t)(t * bt16);
-              // K steps of 16: +32 B inside the swizzled x rows, +2 columns of 8 in w.
-              if constexpr (PAIR) {
-                umma_bf16_pair(d_tmem, ad, bd, idesc, acc);
-                umma_bf16_pair(d_tmem, ad + 2u, bd + bk16, idesc, 1u);
-                umma_bf16_pair(d_tmem, ad + 4u, bd + 2u * bk16, idesc, 1u);
-                umma_bf16_pair(d_tmem, ad + 6u, bd + 3u * bk16, idesc, 1u);
-              } else {
-                umma_bf16(d_tmem, ad, bd, idesc, acc);
-                umma_bf16(d_tmem, ad + 2u, bd + bk16, idesc, 1u);
-                umma_bf16(d_tmem, ad + 4u, bd + 2u * bk16, idesc, 1u);
-                umma_bf16(d_tmem, ad + 6u, bd + 3u * bk16, idesc, 1u);
+            for (int m = 0; m < 2; ++m) {
+              if (m >= pl.MT) break;
+              if (is == 0 && kb == 0) {
+                // The slot must have been drained by the epilogue of its last job.
+                if (ju[m] && !tc_wait<PAIR>(acc_empty + 8 * js[m], (uint32_t)(jp[m] ^ 1),
+                                            args.err, VI_DEV_ERR_MMA_TIMEOUT)) { ok = false; break; }
+                tc_fence_after();
               }
-              acc = 1u;
-            }
-            if (ib == pl.n_cb - 1) {                  // accumulator ready for the epilogue
-              if constexpr (PAIR) umma_commit_pair_mc(acc_full + 8 * js[m], 0x3);
-              else umma_commit(acc_full + 8 * js[m]);
+              const uint32_t d_tmem = tmem_base + (uint32_t)(js[m] * pl.NJ);
+              // k taps x 4 K steps = 4k MMAs back to back per tile and K-block;
+              // a stage queues KS x MT x 4k of them (24 for k = 3 with two
+              // tiles, 16 for k = 1 with two tiles and two K-blocks): enough
+              // tensor work to hide the stage's wait/commit.
+              const uint64_t ad_tile = ad_stage + (uint64_t)((kb * pl.MT + m) * at16);
+              const uint64_t bd_kb = bd_stage + (uint64_t)(kb * pl.k * bt16);
+              uint32_t acc = (is > 0 || kb > 0) ? 1u : 0u;
+              for (int t = 0; t < pl.k; ++t) {
+                // Tap t: the x tile shifted down by t rows of 128 B (8 units of 16 B).
+                const uint64_t ad = ad_tile + (uint64_t)(8u * t);
+                const uint64_t bd = bd_kb + (uint64_t)(t * bt16);
+                // K steps of 16: +32 B inside the swizzled x rows, +2 columns of 8 in w.
+                if constexpr (PAIR) {
+                  umma_bf16_pair(d_tmem, ad, bd, idesc, acc);
+                  umma_bf16_pair(d_tmem, ad + 2u, bd + bk16, idesc, 1u);
+                  umma_bf16_pair(d_tmem, ad + 4u, bd + 2u * bk16, idesc, 1u);
+                  umma_bf16_pair(d_tmem, ad + 6u, bd + 3u * bk16, idesc, 1u);
+                } else {
+                  umma_bf16(d_tmem, ad, bd, idesc, acc);
+                  umma_bf16(d_tmem, ad + 2u, bd + bk16, idesc, 1u);
+                  umma_bf16(d_tmem, ad + 4u, bd + 2u * bk16, idesc, 1u);
+                  umma_bf16(d_tmem, ad + 6u, bd + 3u * bk16, idesc, 1u);
+                }
+                acc = 1u;
+              }
+              if (last_stage && kb == nkb - 1) {      // accumulator ready for the epilogue
+                if constexpr (PAIR) umma_commit_pair_mc(acc_full + 8 * js[m], 0x3);
+                else umma_commit(acc_full + 8 * js[m]);
+              }
             }
           }
           if (!ok) break;
@@ -641,6 +665,11 @@ int temporal_conv_bf16_tc(const bf16* x, const bf16* w, const bf16* b, bf16* y, 
     const int mt = pref > 0 ? pref : TC_MT_DEFAULT;
     TcPlan pl2;
     if (mt == 2 && tc_plan(F, P, C, k, false, pl2, norm, 2) && pl2.NJ >= pl.NJ) pl = pl2;
+    // Single tap: two K-blocks per stage where they fit at the same width, so
+    // a stage still queues 16 MMAs per wait/commit.
+    if (k == 1 && pl.MT == 2 && !norm && tc_plan(F, P, C, k, false, pl2, false, 2, 2) &&
+        pl2.NJ >= pl.NJ)
+      pl = pl2;
   }
   unsigned int* err = device_error_word();
   if (!err) return VI_ERR_CUDA;
