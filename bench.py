@@ -208,6 +208,38 @@ def host_inputs(w, pinned: bool):
     return out
 
 
+INPUT_NAMES = ("q", "k", "v", "conv_x", "conv_w", "conv_b", "gn_x", "gn_gamma", "gn_beta")
+
+
+def shared_host_inputs(w, rank: int, world: int, pinned: bool, device=None):
+    """Every rank's copy of the seeded inputs of workload w.
+
+    With one rank this is host_inputs().  With several, rank 0 generates them
+    once and broadcasts each tensor (through `device` for NCCL, on the host for
+    gloo): every replica gets the same video without each rank repeating the
+    generation on the shared host cores.  A setup step, outside any timed region."""
+    import torch
+    import torch.distributed as dist
+
+    if world == 1 or not dist.is_initialized():
+        return host_inputs(w, pinned)
+    import synth
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    src = host_inputs(w, pinned) if rank == 0 else None
+    out = {}
+    for name in INPUT_NAMES:
+        shape = synth.shape_of(w, name)
+        t = src[name] if rank == 0 else torch.empty(shape, dtype=dt)
+        if device is not None:
+            d = t.to(device) if rank == 0 else torch.empty(shape, dtype=dt, device=device)
+            dist.broadcast(d, src=0)
+            t = d.cpu() if rank != 0 else t
+        else:
+            dist.broadcast(t, src=0)
+        out[name] = t.pin_memory() if pinned and not t.is_pinned() else t
+    return out
+
+
 # ---------------------------------------------------------------------------
 # our arm
 
@@ -225,7 +257,7 @@ def run_ours(args):
     w = synth.BY_NAME[args.workload]
     stream = torch.cuda.current_stream()
 
-    host = host_inputs(w, pinned=True)
+    host = shared_host_inputs(w, rank, world, pinned=True, device=dev)
     d = {k: v.to(dev, non_blocking=True) for k, v in host.items()}
     out = torch.empty_like(d["q"])
     y = torch.empty_like(d["conv_x"])

@@ -51,6 +51,35 @@ def test_max_over_ranks_gloo_world2():
     assert res == {0: 15.0, 1: 15.0}
 
 
+def _share_main(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), WORLD_SIZE=str(world),
+                      RANK=str(rank), LOCAL_RANK=str(rank))
+    bench.init_dist("gloo")
+    w = synth.BY_NAME["tiny_f32_F32_P64_C64"]
+    got = bench.shared_host_inputs(w, rank, world, pinned=False)
+    ref = bench.host_inputs(w, pinned=False)
+    same = all(got[n].shape == ref[n].shape and bool((got[n] == ref[n]).all())
+               for n in bench.INPUT_NAMES)
+    q.put((rank, same))
+    bench.cleanup()
+
+
+def test_inputs_generated_once_and_broadcast_gloo_world2():
+    """Rank 0 generates the seeded inputs and broadcasts them; every rank ends
+    with exactly what host_inputs() gives."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_share_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    res = dict(q.get(timeout=5) for _ in range(2))
+    assert res == {0: True, 1: True}
+
+
 def test_kernel_work_accounting():
     w = synth.BY_NAME["bf16_F1024_P2560_C320"]
     work = bench.kernel_work(w)
