@@ -31,6 +31,8 @@
 // Generic path (fp32 I/O, or shapes outside the fast path): one warp per
 //   (position, head, query frame), keys streamed with an online softmax in
 //   fp32, expf, and the exact key list walked in order.
+#include <atomic>
+
 #include "ptx.cuh"
 #include "vi_internal.cuh"
 
@@ -320,13 +322,14 @@ int dual_attn_bf16_fast(const bf16* q, const bf16* k, const bf16* v, bf16* out, 
     maps.vg = maps.v;
   }
   if (!ok) return VI_ERR_CUDA;
-  static bool attr_set[64] = {false};
+  static std::atomic<bool> attr_set[64] = {};
   int dev = 0;
   VI_CUDA_TRY(cudaGetDevice(&dev));
-  if (dev < 64 && !attr_set[dev]) {
+  if (dev < 0 || dev >= 64 || !attr_set[dev].load(std::memory_order_acquire)) {
+    // Idempotent, so concurrent first calls may both set it.
     VI_CUDA_TRY(cudaFuncSetAttribute(dual_attn_bf16_mma,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, FA_SMEM_BYTES));
-    attr_set[dev] = true;
+    if (dev >= 0 && dev < 64) attr_set[dev].store(true, std::memory_order_release);
   }
   const int nblk = (N + FA_CLIPS - 1) / FA_CLIPS;
   const int64_t grid = (int64_t)P * heads * nblk;
