@@ -32,6 +32,10 @@ SIGNATURES = {
     "vi_temporal_attention": [_vp] * 7 + [_i] * 8 + [_vp],
     "vi_selftest_wait_timeout": [_i, _vp],
     "vi_set_conv_tiles_per_job": [_i],
+    "vi_dual_attn_shard": [_vp] * 6 + [_i] * 10 + [_vp],
+    "vi_temporal_conv_shard": [_vp] * 4 + [_i] * 4 + [_vp],
+    "vi_groupnorm_shard_stats": [_vp] + [_i] * 4 + [_vp, _vp],
+    "vi_groupnorm_shard_apply": [_vp, _vp, _i, _vp, _vp, _vp] + [_i] * 4 + [_f, _vp],
     "vi_version": [],
     "vi_take_device_errors": [],
 }
@@ -200,6 +204,87 @@ def temporal_attention(x, w_qkv, b_qkv, w_out, b_out, out=None, workspace=None, 
         x.data_ptr(), w_qkv.data_ptr(), b_qkv.data_ptr(), w_out.data_ptr(), b_out.data_ptr(),
         out.data_ptr(), workspace.data_ptr(), F, N, P, heads, C // heads, n_pre, n_post, n_global,
         _stream_ptr(stream)))
+    return out
+
+
+def dual_attn_shard(q, k_ext, v_ext, k_glob, v_glob, out=None, *, N_loc: int, clip0: int,
+                    N: int, heads: int, n_pre: int = 8, n_post: int = 8, n_global: int = 16,
+                    stream=None):
+    """Dual-domain attention of one shard of a video cut along frames (bf16).
+
+    q, out [P][F_loc][C]; k_ext, v_ext [P][F_loc + 16][C] (8 frames before and
+    after the shard around it); k_glob, v_glob [P][n_global][C]."""
+    import torch
+    if out is None:
+        out = torch.empty_like(q)
+    if n_global == 0 and (k_glob is None or v_glob is None):
+        k_glob, v_glob = k_ext, v_ext          # not read without global frames
+    _dev(q, k_ext, v_ext, k_glob, v_glob, out)
+    P, F_loc, C = q.shape
+    _shape(out, q.shape, "out")
+    _shape(k_ext, (P, F_loc + 16, C), "k_ext")
+    _shape(v_ext, (P, F_loc + 16, C), "v_ext")
+    if n_global > 0:
+        _shape(k_glob, (P, n_global, C), "k_glob")
+        _shape(v_glob, (P, n_global, C), "v_glob")
+    _check("vi_dual_attn_shard", lib().vi_dual_attn_shard(
+        q.data_ptr(), k_ext.data_ptr(), v_ext.data_ptr(), k_glob.data_ptr(), v_glob.data_ptr(),
+        out.data_ptr(), F_loc, N_loc, clip0, N, P, heads, C // heads, n_pre, n_post, n_global,
+        _stream_ptr(stream)))
+    return out
+
+
+def temporal_conv_shard(x_ext, w, b, out=None, *, stream=None):
+    """Temporal conv of one shard: x_ext [P][F_loc + 2(k/2)][C] -> [P][F_loc][C] (bf16)."""
+    import torch
+    _dev(x_ext, w, b)
+    if w.dim() != 3:
+        raise ValueError("w: expected [C_out][C_in][k]")
+    P, Fx, C = x_ext.shape
+    k = w.shape[2]
+    F_loc = Fx - 2 * (k // 2)
+    if out is None:
+        out = torch.empty((P, F_loc, C), dtype=x_ext.dtype, device=x_ext.device)
+    _dev(x_ext, w, b, out)
+    _shape(w, (C, C, k), "w")
+    _shape(b, (C,), "b")
+    _shape(out, (P, F_loc, C), "out")
+    _check("vi_temporal_conv_shard", lib().vi_temporal_conv_shard(
+        x_ext.data_ptr(), w.data_ptr(), b.data_ptr(), out.data_ptr(), F_loc, P, C, k,
+        _stream_ptr(stream)))
+    return out
+
+
+def groupnorm_shard_stats(x, *, groups: int, stream=None):
+    """Per-group (mean, var) of one shard's rows: a [groups][2] float64 CUDA tensor."""
+    import torch
+    _dev(x)
+    P, F_loc, C = x.shape
+    stats = torch.empty((groups, 2), dtype=torch.float64, device=x.device)
+    _check("vi_groupnorm_shard_stats", lib().vi_groupnorm_shard_stats(
+        x.data_ptr(), F_loc, P, C, groups, stats.data_ptr(), _stream_ptr(stream)))
+    return stats
+
+
+def groupnorm_shard_apply(x, shard_stats, gamma, beta, out=None, *, eps: float = 1e-5,
+                          stream=None):
+    """Normalise one shard with the W shards' statistics shard_stats [W][groups][2]."""
+    import torch
+    if out is None:
+        out = torch.empty_like(x)
+    _dev(x, gamma, beta, out)
+    if not shard_stats.is_cuda or shard_stats.dtype != torch.float64 or shard_stats.dim() != 3 \
+            or not shard_stats.is_contiguous():
+        raise ValueError("shard_stats: expected a contiguous [W][groups][2] float64 CUDA tensor")
+    P, F_loc, C = x.shape
+    W, groups = shard_stats.shape[0], shard_stats.shape[1]
+    _shape(shard_stats, (W, groups, 2), "shard_stats")
+    _shape(gamma, (C,), "gamma")
+    _shape(beta, (C,), "beta")
+    _shape(out, x.shape, "out")
+    _check("vi_groupnorm_shard_apply", lib().vi_groupnorm_shard_apply(
+        x.data_ptr(), shard_stats.data_ptr(), W, gamma.data_ptr(), beta.data_ptr(),
+        out.data_ptr(), F_loc, P, C, groups, float(eps), _stream_ptr(stream)))
     return out
 
 

@@ -152,11 +152,15 @@ struct FaMaps {
   CUtensorMap q, k, v, kg, vg, o;
 };
 
+// N clips of the q map are computed; they are clips clip0 .. clip0 + N - 1 of
+// a video of n_total clips (which decides the absent ends), and frame 0 of
+// the q map is row kv_off of the k/v maps (0 for a whole video on one GPU,
+// the halo width for a shard whose neighbours' frames are stacked around it).
 __global__ void __launch_bounds__(256) dual_attn_bf16_mma(const __grid_constant__ FaMaps maps,
                                                           int F, int N, int heads, int nblk,
                                                           int n_pre, int n_post, int n_global,
-                                                          float scale_log2,
-                                                          unsigned int* err_word) {
+                                                          float scale_log2, int kv_off, int clip0,
+                                                          int n_total, unsigned int* err_word) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
   const uint32_t sQ = base + FA_OFF_Q, sKW = base + FA_OFF_KW, sVW = base + FA_OFF_VW;
@@ -178,8 +182,8 @@ __global__ void __launch_bounds__(256) dual_attn_bf16_mma(const __grid_constant_
                            (n_global > 0 ? 2 * FA_NG * FA_ROW_BYTES : 0);
     mbar_arrive_expect_tx(bar, bytes);
     tma_load_3d(sQ, &maps.q, h * 64, f0, p, bar);
-    tma_load_3d(sKW, &maps.k, h * 64, f0 - FA_HALO, p, bar);
-    tma_load_3d(sVW, &maps.v, h * 64, f0 - FA_HALO, p, bar);
+    tma_load_3d(sKW, &maps.k, h * 64, f0 - FA_HALO + kv_off, p, bar);
+    tma_load_3d(sVW, &maps.v, h * 64, f0 - FA_HALO + kv_off, p, bar);
     if (n_global > 0) {
       tma_load_3d(sKG, &maps.kg, h * 64, 0, p, bar);
       tma_load_3d(sVG, &maps.vg, h * 64, 0, p, bar);
@@ -189,6 +193,7 @@ __global__ void __launch_bounds__(256) dual_attn_bf16_mma(const __grid_constant_
 
   const int clip = blk * FA_CLIPS + warp;
   if (clip < N) {
+    const int gclip = clip0 + clip;              // index in the whole video
     const int g = lane >> 2, qd = lane & 3;
     // ---- S = Q K^T over 48 keys (6 n-tiles of 8), 4 k-steps of 16 dims ----
     uint32_t qa[4][4];
@@ -223,9 +228,9 @@ __global__ void __launch_bounds__(256) dual_attn_bf16_mma(const __grid_constant_
       for (int c = 0; c < 2; ++c) {
         const int kk = nt * 8 + 2 * qd + c;     // key index in the warp's list
         bool valid;
-        if (kk < FA_HALO) valid = clip > 0 && kk >= FA_HALO - n_pre;
+        if (kk < FA_HALO) valid = gclip > 0 && kk >= FA_HALO - n_pre;
         else if (kk < FA_HALO + FA_L) valid = true;
-        else if (kk < 32) valid = clip < N - 1 && kk - (FA_HALO + FA_L) < n_post;
+        else if (kk < 32) valid = gclip < n_total - 1 && kk - (FA_HALO + FA_L) < n_post;
         else valid = kk - 32 < n_global;
         s[nt][c] = valid ? s[nt][c] * scale_log2 : -INFINITY;
         s[nt][c + 2] = valid ? s[nt][c + 2] * scale_log2 : -INFINITY;
@@ -338,7 +343,63 @@ int dual_attn_bf16_fast(const bf16* q, const bf16* k, const bf16* v, bf16* out, 
   unsigned int* err = device_error_word();
   if (!err) return VI_ERR_CUDA;
   dual_attn_bf16_mma<<<(unsigned)grid, 256, FA_SMEM_BYTES, stream>>>(
-      maps, F, N, heads, nblk, n_pre, n_post, n_global, scale_log2, err);
+      maps, F, N, heads, nblk, n_pre, n_post, n_global, scale_log2, 0, 0, N, err);
+  VI_LAUNCHED();
+  return VI_OK;
+}
+
+// One shard of a video cut along frames (clip-parallel over several GPUs):
+// q/out [P][F_loc][C] hold clips clip0 .. clip0 + N_loc - 1 of the video's N;
+// k_ext/v_ext [P][F_loc + 2*FA_HALO][C] hold FA_HALO frames before the shard,
+// the shard's frames and FA_HALO frames after it (rows past a video end are
+// masked out, and must hold finite values); k_glob/v_glob [P][n_global][C]
+// hold the video's global frames.
+int dual_attn_bf16_shard(const bf16* q, const bf16* k_ext, const bf16* v_ext, const bf16* k_glob,
+                         const bf16* v_glob, bf16* out, int F_loc, int N_loc, int clip0, int N,
+                         int P, int heads, int n_pre, int n_post, int n_global,
+                         cudaStream_t stream) {
+  const int C = heads * 64;
+  const int F_ext = F_loc + 2 * FA_HALO;
+  FaMaps maps;
+  const uint64_t dims[3] = {(uint64_t)C, (uint64_t)F_loc, (uint64_t)P};
+  const uint64_t strides[2] = {(uint64_t)C * 2, (uint64_t)F_loc * C * 2};
+  const uint64_t edims[3] = {(uint64_t)C, (uint64_t)F_ext, (uint64_t)P};
+  const uint64_t estrides[2] = {(uint64_t)C * 2, (uint64_t)F_ext * C * 2};
+  const uint32_t boxQ[3] = {64, FA_ROWS_Q, 1}, boxW[3] = {64, FA_ROWS_W, 1};
+  const CUtensorMapDataType BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const CUtensorMapSwizzle SW = CU_TENSOR_MAP_SWIZZLE_128B;
+  bool ok = encode_tmap(&maps.q, q, 3, dims, strides, boxQ, SW, BF) &&
+            encode_tmap(&maps.k, k_ext, 3, edims, estrides, boxW, SW, BF) &&
+            encode_tmap(&maps.v, v_ext, 3, edims, estrides, boxW, SW, BF) &&
+            encode_tmap(&maps.o, out, 3, dims, strides, boxQ, SW, BF);
+  if (n_global > 0) {
+    const uint64_t gdims[3] = {(uint64_t)C, (uint64_t)n_global, (uint64_t)P};
+    const uint64_t gstrides[2] = {(uint64_t)C * 2, (uint64_t)n_global * C * 2};
+    const uint32_t boxG[3] = {64, FA_NG, 1};
+    ok = ok && encode_tmap(&maps.kg, k_glob, 3, gdims, gstrides, boxG, SW, BF) &&
+         encode_tmap(&maps.vg, v_glob, 3, gdims, gstrides, boxG, SW, BF);
+  } else {
+    maps.kg = maps.k;
+    maps.vg = maps.v;
+  }
+  if (!ok) return VI_ERR_CUDA;
+  static std::atomic<bool> attr_set[64] = {};
+  int dev = 0;
+  VI_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64 || !attr_set[dev].load(std::memory_order_acquire)) {
+    VI_CUDA_TRY(cudaFuncSetAttribute(dual_attn_bf16_mma,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, FA_SMEM_BYTES));
+    if (dev >= 0 && dev < 64) attr_set[dev].store(true, std::memory_order_release);
+  }
+  const int nblk = (N_loc + FA_CLIPS - 1) / FA_CLIPS;
+  const int64_t grid = (int64_t)P * heads * nblk;
+  if (grid > 0x7fffffff) return VI_ERR_UNSUPPORTED;
+  const float scale_log2 = 1.4426950408889634f / 8.0f;    // log2(e) / sqrt(64)
+  unsigned int* err = device_error_word();
+  if (!err) return VI_ERR_CUDA;
+  dual_attn_bf16_mma<<<(unsigned)grid, 256, FA_SMEM_BYTES, stream>>>(
+      maps, F_loc, N_loc, heads, nblk, n_pre, n_post, n_global, scale_log2, FA_HALO, clip0, N,
+      err);
   VI_LAUNCHED();
   return VI_OK;
 }

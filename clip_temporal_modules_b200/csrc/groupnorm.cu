@@ -74,10 +74,11 @@ __device__ void gn_finalize(const GnScratch& s, int nparts, int groups, int C, i
     const double m1 = red[g][1] / nn;
     const double var = fmax(red[g][2] / nn - m1 * m1, 0.0);
     const double mu = (double)to_f32(x[(size_t)g * cg]) + m1;
-    const double a = (double)to_f32(gamma[c]) / sqrt(var + (double)eps);
+    // gamma/beta are null when only the statistics are wanted (a shard's pass).
+    const double a = (gamma ? (double)to_f32(gamma[c]) : 1.0) / sqrt(var + (double)eps);
     s.coef[4 * c] = (float)mu;
     s.coef[4 * c + 1] = (float)a;
-    s.coef[4 * c + 2] = to_f32(beta[c]);
+    s.coef[4 * c + 2] = beta ? to_f32(beta[c]) : 0.f;
     s.coef[4 * c + 3] = 0.f;
     if (c == g * cg) {
       s.stats[2 * g] = mu;
@@ -531,6 +532,98 @@ size_t gn_scratch_size_bf16(int64_t rows, int C, int groups) {
 
 template int gn_stats_launch<bf16>(const bf16*, const bf16*, const bf16*, int64_t, int, int, float,
                                    void*, cudaStream_t, const float**);
+
+// ---------------------------------------------------------------------------
+// A video cut along frames over several GPUs (clip parallelism): each shard
+// reduces its own rows (a6), the shards' statistics are exchanged and merged
+// (a7), and each shard normalises its rows with the merged statistics (a8).
+
+// a6 on one shard: per-group (mean, var) of the shard's rows, fp64, into
+// stats [groups][2] (device memory).
+template <typename T>
+int gn_shard_stats(const T* x, int64_t rows, int C, int groups, double* stats,
+                   cudaStream_t stream) {
+  const size_t bytes = gn_scratch_bytes<T>(rows, C, groups);
+  void* scratch = nullptr;
+  VI_CUDA_TRY(scratch_alloc(&scratch, bytes, stream));
+  const float* coef = nullptr;
+  int st = cudaMemsetAsync(scratch, 0, 64, stream) == cudaSuccess ? VI_OK : VI_ERR_CUDA;
+  if (st == VI_OK)
+    st = gn_stats_launch<T>(x, nullptr, nullptr, rows, C, groups, 1e-5f, scratch, stream, &coef);
+  if (st == VI_OK) {
+    const GnScratch s = gn_carve(scratch, groups, C);
+    if (cudaMemcpyAsync(stats, s.stats, sizeof(double) * 2 * groups, cudaMemcpyDeviceToDevice,
+                        stream) != cudaSuccess)
+      st = VI_ERR_CUDA;
+  }
+  if (scratch_free(scratch, stream) != cudaSuccess && st == VI_OK) st = VI_ERR_CUDA;
+  return st;
+}
+
+// a7: merge W shards of equal row counts, shard_stats [W][groups][2] of
+// (mean, var): mean = average of the means, var = average of (var_w +
+// (mean_w - mean)^2) (the pooled biased variance); then the per-channel
+// coefficients (m_c, a_c, beta_c, 0) of the normalisation.
+template <typename T>
+__global__ void gn_merge_coef(const double* __restrict__ shard_stats, int W, int groups, int C,
+                              const T* __restrict__ gamma, const T* __restrict__ beta, float eps,
+                              float* __restrict__ coef) {
+  const int cg = C / groups;
+  for (int c = blockIdx.x * blockDim.x + threadIdx.x; c < C; c += gridDim.x * blockDim.x) {
+    const int g = c / cg;
+    double mean = 0.0;
+    for (int w = 0; w < W; ++w) mean += shard_stats[((size_t)w * groups + g) * 2];
+    mean /= W;
+    double var = 0.0;
+    for (int w = 0; w < W; ++w) {
+      const double dm = shard_stats[((size_t)w * groups + g) * 2] - mean;
+      var += shard_stats[((size_t)w * groups + g) * 2 + 1] + dm * dm;
+    }
+    var /= W;
+    const double a = (double)to_f32(gamma[c]) / sqrt(var + (double)eps);
+    coef[4 * c] = (float)mean;
+    coef[4 * c + 1] = (float)a;
+    coef[4 * c + 2] = to_f32(beta[c]);
+    coef[4 * c + 3] = 0.f;
+  }
+}
+
+// a7 + a8 on one shard: merged statistics, then y = (x - m_c) a_c + beta_c.
+template <typename T>
+int gn_shard_apply(const T* x, const double* shard_stats, int W, const T* gamma, const T* beta,
+                   T* y, int64_t rows, int C, int groups, float eps, cudaStream_t stream) {
+  const GnPlan pl = gn_plan<T>(rows, C, groups);
+  float* coef = nullptr;
+  VI_CUDA_TRY(scratch_alloc(reinterpret_cast<void**>(&coef), sizeof(float) * 4 * (size_t)C,
+                            stream));
+  int st = VI_OK;
+  gn_merge_coef<T><<<(C + 255) / 256, 256, 0, stream>>>(shard_stats, W, groups, C, gamma, beta,
+                                                        eps, coef);
+  if (cudaGetLastError() != cudaSuccess) st = VI_ERR_CUDA; else note_launch();
+  if (st == VI_OK && pl.ring) {
+    unsigned int* err = device_error_word();
+    if (!err) st = VI_ERR_CUDA;
+    else if (cudaFuncSetAttribute(gn_apply_ring<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)pl.smem) != cudaSuccess)
+      st = VI_ERR_CUDA;
+    if (st == VI_OK) {
+      gn_apply_ring<T><<<pl.blocks, pl.threads, pl.smem, stream>>>(x, y, pl.rg, coef, err);
+      if (cudaGetLastError() != cudaSuccess) st = VI_ERR_CUDA; else note_launch();
+    }
+  } else if (st == VI_OK) {
+    const int64_t n = rows * C;
+    int64_t blocks = (n + 255) / 256;
+    if (blocks > (int64_t)sm_count() * 16) blocks = (int64_t)sm_count() * 16;
+    gn_apply_scalar<T><<<(int)blocks, 256, 0, stream>>>(x, y, n, C, coef);
+    if (cudaGetLastError() != cudaSuccess) st = VI_ERR_CUDA; else note_launch();
+  }
+  if (scratch_free(coef, stream) != cudaSuccess && st == VI_OK) st = VI_ERR_CUDA;
+  return st;
+}
+
+template int gn_shard_stats<bf16>(const bf16*, int64_t, int, int, double*, cudaStream_t);
+template int gn_shard_apply<bf16>(const bf16*, const double*, int, const bf16*, const bf16*, bf16*,
+                                  int64_t, int, int, float, cudaStream_t);
 
 template <typename T>
 int groupnorm_global(const T* x, const T* gamma, const T* beta, T* y, int64_t rows, int C,

@@ -115,6 +115,7 @@ struct TcArgs {
   const bf16* bias;
   bf16* y;
   unsigned int* err;
+  int x_off;             // row of output frame 0 in the x map (k/2 for a shard with halos)
 };
 
 // Ring depths (measured on B200 at F = 1024): with one tile per job and
@@ -273,7 +274,7 @@ __global__ void __launch_bounds__(TC_THREADS + (NORM ? 128 : 0), 1)
 #pragma unroll
         for (int m = 0; m < 2; ++m) {
           const long long tile = tile0 + m;
-          frow[m] = (int)(tile % pl.n_fblk) * TC_M - halo;
+          frow[m] = (int)(tile % pl.n_fblk) * TC_M - halo + args.x_off;
           pos[m] = (int)(tile / pl.n_fblk);
         }
         int wrow = (slab * pl.n_cb * pl.k * pl.H + (int)rank) * pl.b_rows;   // row of (slab, cb 0, t 0)
@@ -652,8 +653,8 @@ static int tc_launch(const CUtensorMap& tmx, const CUtensorMap& tmw, const CUten
 
 // coef != nullptr: normalise x on the fly with the GroupNorm coefficients
 // (m_c, a_c, beta_c) before the contraction (fused GroupNorm -> conv).
-int temporal_conv_bf16_tc(const bf16* x, const bf16* w, const bf16* b, bf16* y, int F, int P,
-                          int C, int k, cudaStream_t stream, const float* coef) {
+static int tc_run(const bf16* x, int x_rows, int x_off, const bf16* w, const bf16* b, bf16* y,
+                  int F, int P, int C, int k, cudaStream_t stream, const float* coef) {
   TcPlan pl;
   const bool norm = coef != nullptr;
   const bool pair = !norm && TC_USE_PAIR && tc_plan(F, P, C, k, true, pl);
@@ -673,7 +674,7 @@ int temporal_conv_bf16_tc(const bf16* x, const bf16* w, const bf16* b, bf16* y, 
   }
   unsigned int* err = device_error_word();
   if (!err) return VI_ERR_CUDA;
-  // x as [P][F][C]: box of 64 channels x a_rows frames x 1 position, 128B swizzle.
+  // x as [P][x_rows][C]: box of 64 channels x a_rows frames x 1 position, 128B swizzle.
   CUtensorMap tmx, tmw, tmy;
   {
     // y as [P][F][C]: box of 32 channels x 128 frames x 1 position, 64B swizzle.
@@ -685,8 +686,8 @@ int temporal_conv_bf16_tc(const bf16* x, const bf16* w, const bf16* b, bf16* y, 
       return VI_ERR_CUDA;
   }
   {
-    const uint64_t dims[3] = {(uint64_t)C, (uint64_t)F, (uint64_t)P};
-    const uint64_t strides[2] = {(uint64_t)C * 2, (uint64_t)F * C * 2};
+    const uint64_t dims[3] = {(uint64_t)C, (uint64_t)x_rows, (uint64_t)P};
+    const uint64_t strides[2] = {(uint64_t)C * 2, (uint64_t)x_rows * C * 2};
     const uint32_t box[3] = {(uint32_t)TC_KB, (uint32_t)pl.a_rows, 1};
     if (!encode_tmap(&tmx, x, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_DATA_TYPE_BFLOAT16))
@@ -714,13 +715,27 @@ int temporal_conv_bf16_tc(const bf16* x, const bf16* w, const bf16* b, bf16* y, 
     if (cudaGetLastError() != cudaSuccess) st = VI_ERR_CUDA; else note_launch();
   }
   if (st == VI_OK) {
-    TcArgs a{coef, b, y, err};
+    TcArgs a{coef, b, y, err, x_off};
     st = norm ? tc_launch<false, true>(tmx, tmw, tmy, pl, a, stream)
               : pair ? tc_launch<true, false>(tmx, tmw, tmy, pl, a, stream)
                      : tc_launch<false, false>(tmx, tmw, tmy, pl, a, stream);
   }
   if (scratch_free(wpk, stream) != cudaSuccess && st == VI_OK) st = VI_ERR_CUDA;
   return st;
+}
+
+int temporal_conv_bf16_tc(const bf16* x, const bf16* w, const bf16* b, bf16* y, int F, int P,
+                          int C, int k, cudaStream_t stream, const float* coef) {
+  return tc_run(x, F, 0, w, b, y, F, P, C, k, stream, coef);
+}
+
+// One shard of a video cut along frames: x_ext [P][F_loc + 2(k/2)][C] holds
+// the k/2 frames before the shard (zeros at the start of the video), the
+// shard's frames and the k/2 frames after it (zeros at the end); y is
+// [P][F_loc][C].
+int temporal_conv_bf16_tc_shard(const bf16* x_ext, const bf16* w, const bf16* b, bf16* y,
+                                int F_loc, int P, int C, int k, cudaStream_t stream) {
+  return tc_run(x_ext, F_loc + 2 * (k / 2), k / 2, w, b, y, F_loc, P, C, k, stream, nullptr);
 }
 
 }  // namespace vi

@@ -29,6 +29,15 @@ int dual_attn_generic_launch(const T*, const T*, const T*, T*, int, int, int, in
 int dual_attn_bf16_fast(const bf16*, const bf16*, const bf16*, bf16*, int, int, int, int, int,
                         int, int, cudaStream_t);
 bool dual_attn_fast_ok(int F, int N, int d, int n_pre, int n_post, int n_global);
+int dual_attn_bf16_shard(const bf16*, const bf16*, const bf16*, const bf16*, const bf16*, bf16*,
+                         int, int, int, int, int, int, int, int, int, cudaStream_t);
+int temporal_conv_bf16_tc_shard(const bf16*, const bf16*, const bf16*, bf16*, int, int, int, int,
+                                cudaStream_t);
+template <typename T>
+int gn_shard_stats(const T*, int64_t, int, int, double*, cudaStream_t);
+template <typename T>
+int gn_shard_apply(const T*, const double*, int, const T*, const T*, T*, int64_t, int, int, float,
+                   cudaStream_t);
 template <typename T>
 int temporal_conv_generic_launch(const T*, const T*, const T*, T*, int, int, int, int,
                                  cudaStream_t);
@@ -330,9 +339,125 @@ int temporal_attention_entry(const void* x, const void* w_qkv, const void* b_qkv
   return st;
 }
 
+// ---- shards of a video cut along frames (clip parallelism over GPUs) -------
+
+int attn_shard_entry(const void* q, const void* k_ext, const void* v_ext, const void* k_glob,
+                     const void* v_glob, void* out, int F_loc, int N_loc, int clip0, int N, int P,
+                     int heads, int d, int n_pre, int n_post, int n_global, vi_stream_t stream) {
+  using T = bf16;
+  if (heads <= 0 || d <= 0 || (int64_t)heads * d > 0x7fffffff) return VI_ERR_INVALID_ARG;
+  const int C = heads * d;
+  if (F_loc <= 0 || N_loc <= 0 || P < 0 || F_loc % N_loc != 0) return VI_ERR_INVALID_ARG;
+  if (N < N_loc || clip0 < 0 || clip0 > N - N_loc) return VI_ERR_INVALID_ARG;
+  const int L = F_loc / N_loc;
+  if ((double)N * L > 2147483647.0) return VI_ERR_INVALID_ARG;
+  if (n_pre < 0 || n_post < 0 || n_global < 0 || n_global > N * L) return VI_ERR_INVALID_ARG;
+  if (N > 1 && (n_pre > L || n_post > L)) return VI_ERR_INVALID_ARG;
+  if ((double)P * (double)(F_loc + 16) * (double)C > 1.099511627776e12) return VI_ERR_UNSUPPORTED;
+  if (!dual_attn_fast_ok(L, 1, d, n_pre, n_post, n_global)) return VI_ERR_UNSUPPORTED;
+  if (P == 0) return VI_OK;
+  if (!q || !k_ext || !v_ext || !out || (n_global > 0 && (!k_glob || !v_glob)))
+    return VI_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_ext) || !aligned16(v_ext) || !aligned16(out) ||
+      (n_global > 0 && (!aligned16(k_glob) || !aligned16(v_glob))))
+    return VI_ERR_ALIGNMENT;
+  if ((C * sizeof(T)) % 16 != 0) return VI_ERR_ALIGNMENT;
+  const size_t S = (size_t)P * F_loc * C * sizeof(T), E = (size_t)P * (F_loc + 16) * C * sizeof(T);
+  const size_t G = (size_t)P * n_global * C * sizeof(T);
+  if (overlaps(out, S, q, S) || overlaps(out, S, k_ext, E) || overlaps(out, S, v_ext, E) ||
+      (n_global > 0 && (overlaps(out, S, k_glob, G) || overlaps(out, S, v_glob, G))))
+    return VI_ERR_INVALID_ARG;
+  return dual_attn_bf16_shard(static_cast<const T*>(q), static_cast<const T*>(k_ext),
+                              static_cast<const T*>(v_ext), static_cast<const T*>(k_glob),
+                              static_cast<const T*>(v_glob), static_cast<T*>(out), F_loc, N_loc,
+                              clip0, N, P, heads, n_pre, n_post, n_global, as_stream(stream));
+}
+
+int conv_shard_entry(const void* x_ext, const void* w, const void* b, void* y, int F_loc, int P,
+                     int C, int k, vi_stream_t stream) {
+  using T = bf16;
+  if (F_loc <= 0 || P < 0 || C <= 0) return VI_ERR_INVALID_ARG;
+  if (k <= 0 || k % 2 == 0) return VI_ERR_INVALID_ARG;
+  if ((double)P * (double)(F_loc + k) * (double)C > 1.099511627776e12) return VI_ERR_UNSUPPORTED;
+  if (P > 0 && !temporal_conv_tc_ok(F_loc, P, C, k)) return VI_ERR_UNSUPPORTED;
+  if (P == 0) return VI_OK;
+  if (!x_ext || !w || !b || !y) return VI_ERR_INVALID_ARG;
+  if (!aligned16(x_ext) || !aligned16(w) || !aligned16(b) || !aligned16(y)) return VI_ERR_ALIGNMENT;
+  const size_t S = (size_t)P * F_loc * C * sizeof(T);
+  const size_t X = (size_t)P * (F_loc + 2 * (k / 2)) * C * sizeof(T);
+  const size_t wbytes = (size_t)C * C * k * sizeof(T), bbytes = (size_t)C * sizeof(T);
+  if (overlaps(y, S, x_ext, X) || overlaps(y, S, w, wbytes) || overlaps(y, S, b, bbytes))
+    return VI_ERR_INVALID_ARG;
+  return temporal_conv_bf16_tc_shard(static_cast<const T*>(x_ext), static_cast<const T*>(w),
+                                     static_cast<const T*>(b), static_cast<T*>(y), F_loc, P, C, k,
+                                     as_stream(stream));
+}
+
+int gn_shard_check(int F_loc, int P, int C, int groups) {
+  if (F_loc <= 0 || P <= 0 || C <= 0) return VI_ERR_INVALID_ARG;
+  if (groups <= 0 || C % groups != 0) return VI_ERR_INVALID_ARG;
+  if (groups > 1024) return VI_ERR_UNSUPPORTED;
+  if ((double)P * (double)F_loc * (double)C > 1.099511627776e12) return VI_ERR_UNSUPPORTED;
+  if ((C * sizeof(bf16)) % 16 != 0) return VI_ERR_ALIGNMENT;
+  return VI_OK;
+}
+
+int gn_shard_stats_entry(const void* x, int F_loc, int P, int C, int groups, double* stats,
+                         vi_stream_t stream) {
+  int st = gn_shard_check(F_loc, P, C, groups);
+  if (st != VI_OK) return st;
+  if (!x || !stats) return VI_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(stats)) return VI_ERR_ALIGNMENT;
+  return gn_shard_stats<bf16>(static_cast<const bf16*>(x), (int64_t)P * F_loc, C, groups, stats,
+                              as_stream(stream));
+}
+
+int gn_shard_apply_entry(const void* x, const double* shard_stats, int W, const void* gamma,
+                         const void* beta, void* y, int F_loc, int P, int C, int groups, float eps,
+                         vi_stream_t stream) {
+  int st = gn_shard_check(F_loc, P, C, groups);
+  if (st != VI_OK) return st;
+  if (W <= 0 || !(eps >= 0.f) || !isfinite(eps)) return VI_ERR_INVALID_ARG;
+  if (!x || !shard_stats || !gamma || !beta || !y) return VI_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(shard_stats) || !aligned16(gamma) || !aligned16(beta) ||
+      !aligned16(y))
+    return VI_ERR_ALIGNMENT;
+  const size_t S = (size_t)P * F_loc * C * sizeof(bf16), cb = (size_t)C * sizeof(bf16);
+  if (y != x && overlaps(y, S, x, S)) return VI_ERR_INVALID_ARG;
+  if (overlaps(y, S, gamma, cb) || overlaps(y, S, beta, cb) ||
+      overlaps(y, S, shard_stats, sizeof(double) * 2 * (size_t)W * groups))
+    return VI_ERR_INVALID_ARG;
+  return gn_shard_apply<bf16>(static_cast<const bf16*>(x), shard_stats, W,
+                              static_cast<const bf16*>(gamma), static_cast<const bf16*>(beta),
+                              static_cast<bf16*>(y), (int64_t)P * F_loc, C, groups, eps,
+                              as_stream(stream));
+}
+
 }  // namespace
 
 extern "C" {
+
+int vi_dual_attn_shard(const void* q, const void* k_ext, const void* v_ext, const void* k_glob,
+                       const void* v_glob, void* out, int F_loc, int N_loc, int clip0, int N,
+                       int P, int heads, int d, int n_pre, int n_post, int n_global,
+                       vi_stream_t stream) {
+  return attn_shard_entry(q, k_ext, v_ext, k_glob, v_glob, out, F_loc, N_loc, clip0, N, P, heads,
+                          d, n_pre, n_post, n_global, stream);
+}
+int vi_temporal_conv_shard(const void* x_ext, const void* w, const void* b, void* y, int F_loc,
+                           int P, int C, int k, vi_stream_t stream) {
+  return conv_shard_entry(x_ext, w, b, y, F_loc, P, C, k, stream);
+}
+int vi_groupnorm_shard_stats(const void* x, int F_loc, int P, int C, int groups, double* stats,
+                             vi_stream_t stream) {
+  return gn_shard_stats_entry(x, F_loc, P, C, groups, stats, stream);
+}
+int vi_groupnorm_shard_apply(const void* x, const double* shard_stats, int W, const void* gamma,
+                             const void* beta, void* y, int F_loc, int P, int C, int groups,
+                             float eps, vi_stream_t stream) {
+  return gn_shard_apply_entry(x, shard_stats, W, gamma, beta, y, F_loc, P, C, groups, eps, stream);
+}
+
 
 unsigned long long vi_temporal_attention_workspace_bytes(int F, int P, int C) {
   if (F <= 0 || P <= 0 || C <= 0) return 0ull;

@@ -254,6 +254,76 @@ int vi_groupnorm_global_noalloc(const void* x, const void* gamma, const void* be
                                 int F, int N, int P, int C, int groups, float eps,
                                 vi_stream_t stream);
 
+/*
+ * ---- Shards of a video cut along frames (clip parallelism over GPUs) ----
+ *
+ * Source: the write-up's clip-parallelism paragraphs: each device holds some
+ * clips of the video and receives, before its temporal modules run, the
+ * frames its clips need from the neighbouring devices (the end of the previous
+ * clip and the start of the next) and the globally sampled frames, and the
+ * devices exchange GroupNorm statistics.  These calls are the per-device
+ * compute of that scheme; the exchange itself is the caller's (NCCL, or the
+ * package's ClipParallel).  A shard holds F_loc consecutive frames of every
+ * position; bf16 only.
+ */
+
+/*
+ * Dual-domain attention of one shard (attention-module paragraph).
+ *
+ * q, out        : [P][F_loc][C], the shard's frames: clips clip0 ..
+ *                 clip0 + N_loc - 1 of the video's N clips (L = F_loc / N_loc).
+ * k_ext, v_ext  : [P][F_loc + 16][C]: the 8 frames before the shard, the
+ *                 shard's F_loc frames, the 8 frames after it.  Rows past a
+ *                 video end are masked out but are read: they must hold finite
+ *                 values (zeros).
+ * k_glob, v_glob: [P][n_global][C]: the video's global frames
+ *                 j * floor(F / n_global), j < n_global (unused if n_global == 0).
+ * Result       : exactly vi_dual_attn of the whole video, restricted to the
+ *                 shard's frames.
+ * Requirements : L == 16, d == 64, n_pre, n_post <= 8, n_global <= 16
+ *                 (VI_ERR_UNSUPPORTED otherwise); 0 <= clip0 <= N - N_loc;
+ *                 out must not overlap any input; P == 0 is an empty call.
+ */
+int vi_dual_attn_shard(const void* q, const void* k_ext, const void* v_ext, const void* k_glob,
+                       const void* v_glob, void* out, int F_loc, int N_loc, int clip0, int N,
+                       int P, int heads, int d, int n_pre, int n_post, int n_global,
+                       vi_stream_t stream);
+
+/*
+ * Temporal conv of one shard (conv-module paragraph: each clip padded with
+ * the neighbours' boundary frames).
+ *
+ * x_ext : [P][F_loc + 2*(k/2)][C]: k/2 frames before the shard (zeros at the
+ *         start of the video), the shard's frames, k/2 frames after it (zeros
+ *         at the end).   y : [P][F_loc][C].   w : [C][C][k];  b : [C].
+ * Result       : vi_temporal_conv of the whole video on the shard's frames.
+ * Requirements : k odd; the tensor-core path (C % 64 == 0), else
+ *                VI_ERR_UNSUPPORTED; y must not overlap x_ext, w or b.
+ */
+int vi_temporal_conv_shard(const void* x_ext, const void* w, const void* b, void* y, int F_loc,
+                           int P, int C, int k, vi_stream_t stream);
+
+/*
+ * GroupNorm across shards (GroupNorm-module paragraph): every shard reduces
+ * its rows (vi_groupnorm_shard_stats), the W shards' statistics are gathered
+ * onto every device, and each shard normalises its rows with the merged
+ * statistics (vi_groupnorm_shard_apply).  All shards must hold the same
+ * number of rows (F_loc * P).
+ *
+ * stats       : [groups][2] fp64 device array, (mean, var) of this shard's rows
+ *               (biased variance).
+ * shard_stats : [W][groups][2], the W shards' stats in any order.  Merged as
+ *               mean = average of the means, var = average of (var_w +
+ *               (mean_w - mean)^2), which is the variance of the union.
+ * Requirements : P > 0 (a shard with no rows has no statistics); C % groups
+ *                == 0; groups <= 1024; y may equal x.
+ */
+int vi_groupnorm_shard_stats(const void* x, int F_loc, int P, int C, int groups, double* stats,
+                             vi_stream_t stream);
+int vi_groupnorm_shard_apply(const void* x, const double* shard_stats, int W, const void* gamma,
+                             const void* beta, void* y, int F_loc, int P, int C, int groups,
+                             float eps, vi_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
