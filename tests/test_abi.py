@@ -208,3 +208,43 @@ def test_binding_checks_shapes_before_the_call():
         _shape(torch.empty(2, 3, 4), (2, 3, 5), "x")
     with pytest.raises(ValueError):
         _shape(torch.empty(12), (3, 4), "w")
+
+
+def attn_shard(L, q=A, ke=B, ve=Cp, kg=D, vg=E, o=G, F_loc=64, N_loc=4, clip0=4, N=16, P=2,
+               heads=2, d=64, pre=8, post=8, glob=16):
+    return L.vi_dual_attn_shard(q, ke, ve, kg, vg, o, F_loc, N_loc, clip0, N, P, heads, d, pre,
+                                post, glob, None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(N_loc=0), INVALID), (dict(F_loc=62), INVALID), (dict(clip0=13), INVALID),
+    (dict(clip0=-1), INVALID), (dict(N=3), INVALID), (dict(pre=17), INVALID),
+    (dict(glob=17), UNSUP), (dict(F_loc=128), UNSUP), (dict(d=32), UNSUP), (dict(P=-1), INVALID),
+    (dict(q=A + 8), ALIGN), (dict(o=A), INVALID), (dict(q=None), INVALID),
+    (dict(P=0, q=None, ke=None, ve=None, kg=None, vg=None, o=None), OK),
+])
+def test_attention_shard_rejects(L, kw, expect):
+    assert attn_shard(L, **kw) == expect
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(k=2), INVALID), (dict(F_loc=0), INVALID), (dict(C=40), UNSUP), (dict(x=A + 8), ALIGN),
+    (dict(y=A), INVALID), (dict(P=0, x=None, w=None, b=None, y=None), OK),
+])
+def test_conv_shard_rejects(L, kw, expect):
+    a = dict(x=A, w=B, b=Cp, y=D, F_loc=64, P=2, C=64, k=3)
+    a.update(kw)
+    assert L.vi_temporal_conv_shard(a["x"], a["w"], a["b"], a["y"], a["F_loc"], a["P"], a["C"],
+                                    a["k"], None) == expect
+
+
+def test_groupnorm_shard_rejects(L):
+    st = L.vi_groupnorm_shard_stats
+    ap = L.vi_groupnorm_shard_apply
+    assert st(A, 64, 0, 64, 8, B, None) == INVALID          # a shard with no rows has no stats
+    assert st(A, 64, 2, 64, 7, B, None) == INVALID
+    assert st(None, 64, 2, 64, 8, B, None) == INVALID
+    assert st(A + 8, 64, 2, 64, 8, B, None) == ALIGN
+    assert ap(A, B, 0, Cp, D, E, 64, 2, 64, 8, 1e-5, None) == INVALID     # W = 0
+    assert ap(A, B, 2, Cp, D, E, 64, 2, 64, 8, -1.0, None) == INVALID     # eps < 0
+    assert ap(A, B, 2, Cp, D, A + 64, 64, 2, 64, 8, 1e-5, None) == INVALID  # y inside x
