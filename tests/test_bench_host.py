@@ -113,3 +113,12 @@ def test_reference_arm_other_ranks_do_nothing(monkeypatch):
     with redirect_stdout(buf):
         bench.run_reference(bench.parse_args(["--impl", "reference"]))
     assert buf.getvalue() == ""
+
+
+def test_clock_anomaly_rules():
+    ok = {"sm_mhz": 1965, "sm_max_mhz": 1965, "reasons": [], "samples": 9}
+    assert bench.clock_anomaly(ok) is None
+    assert bench.clock_anomaly({**ok, "sm_mhz": 1500, "reasons": ["sw_power_cap"]}) is None
+    assert "no reason" in bench.clock_anomaly({**ok, "sm_mhz": 1597})
+    assert "hw_slowdown" in bench.clock_anomaly({**ok, "reasons": ["hw_slowdown"]})
+    assert bench.clock_anomaly({**ok, "sm_mhz": None, "reasons": ["unsampled"]}) is None
