@@ -38,6 +38,9 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 DEFAULT_WORKLOAD = "bf16_F1024_P2560_C320"
+# Nominal per-GPU figures (B200 HGX: HBM3e 7.7 TB/s, dense bf16 2.25 PFLOP/s), reported
+# beside the measured denominators for context.
+NOMINAL = {"hbm_gbs": 7700.0, "bf16_tflops": 2250.0}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
                   "sm_max_mhz": 1965.0}
 
@@ -357,6 +360,8 @@ def run_ours(args):
                 "peak": tensor_peak if kd["bound"] == "tensor" else peaks["hbm_gbs"],
                 "unit": kd["unit"], "frac": kd["frac"], "traffic": traffic,
                 "peak_source": f"{peak_src} ({'bf16_tflops_sustained' if kd['bound'] == 'tensor' else 'hbm_gbs'})"}
+    nom = NOMINAL["bf16_tflops"] if kd["bound"] == "tensor" else NOMINAL["hbm_gbs"]
+    roofline["nominal"] = {"peak": nom, "frac": round(kd["achieved"] / nom, 4)}
 
     result = {
         "metric": "temporal-module tokens/s (F*H'W') at F=1024",
@@ -568,13 +573,15 @@ def oracle_sample(w, positions: int):
             ("q", "k", "v", "conv_x", "conv_w", "conv_b", "gn_x", "gn_gamma", "gn_beta")}, sub
 
 
-def oracle_step(inp, sub):
+def oracle_step(inp, sub, nthreads: int = 0):
+    """The three modules of the oracle on the sample (nthreads 0 = every host core)."""
     import oracle
     oracle.dual_attn(inp["q"], inp["k"], inp["v"], sub.F, sub.N, sub.heads, sub.d, sub.n_pre,
-                     sub.n_post, sub.n_global)
-    oracle.temporal_conv(inp["conv_x"], inp["conv_w"], inp["conv_b"], sub.F, sub.N, sub.k)
+                     sub.n_post, sub.n_global, nthreads=nthreads)
+    oracle.temporal_conv(inp["conv_x"], inp["conv_w"], inp["conv_b"], sub.F, sub.N, sub.k,
+                         nthreads=nthreads)
     oracle.groupnorm_global(inp["gn_x"], inp["gn_gamma"], inp["gn_beta"], sub.F, sub.N,
-                            sub.groups, sub.eps)
+                            sub.groups, sub.eps, nthreads=nthreads)
 
 
 def calibrate_positions(w, seconds: float) -> int:
@@ -592,10 +599,17 @@ def cpu_baseline(w, seconds: float):
     t = time.perf_counter()
     oracle_step(inp, sub)
     dt = time.perf_counter() - t
+    # The same oracle on one host thread, on a smaller sample (2 positions).
+    inp1, sub1 = oracle_sample(w, min(2, w.P))
+    t = time.perf_counter()
+    oracle_step(inp1, sub1, nthreads=1)
+    dt1 = time.perf_counter() - t
     return {"value": round(sub.tokens / dt, 1), "unit": "tokens/s", "cores": oracle.max_threads(),
             "kind": "oracle", "seconds": round(dt, 2),
             "sample": f"{npos} of {w.P} positions x all {w.F} frames x {w.C} channels of "
-                      f"{w.name}, all three modules (GroupNorm statistics over the sample)"}
+                      f"{w.name}, all three modules (GroupNorm statistics over the sample)",
+            "single_thread": {"value": round(sub1.tokens / dt1, 1), "unit": "tokens/s",
+                              "sample": f"{sub1.P} positions", "seconds": round(dt1, 2)}}
 
 
 def run_reference(args):
