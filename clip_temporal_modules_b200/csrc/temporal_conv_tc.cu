@@ -56,7 +56,7 @@
 //   warp 0      TMA producer (one elected thread)
 //   warp 1      TMEM allocator + MMA issuer (one thread, even CTA of a pair)
 //   warps 2..5  epilogue; warp w reads TMEM lanes 32*(w%4) .. +31
-//   warps 6..9  (GroupNorm fusion only) normalise the landed x tiles
+//   warps 6..13 (GroupNorm fusion only) normalise the landed x tiles
 #include <atomic>
 #include <mutex>
 
@@ -71,7 +71,8 @@ constexpr int TC_SA_MAX = 6;     // A (x) stages at most
 constexpr int TC_SB_MAX = 8;     // B (w) stages at most
 constexpr int TC_NJ_MAX = 160;   // a B stage holds all k taps of one K-block
 constexpr int TC_EPI_WARPS = 4;          // one per TMEM lane quadrant
-constexpr int TC_THREADS = 64 + 32 * TC_EPI_WARPS;   // + 128 transform threads with NORM
+constexpr int TC_THREADS = 64 + 32 * TC_EPI_WARPS;   // + transform threads with NORM
+constexpr int TC_XF_WARPS = 8;           // NORM: warps normalising the landed x stages
 constexpr int TC_OUT_CHUNK = 128 * 64;   // staged output: 128 frames x 32 channels of bf16
 constexpr int TC_TMEM_COLS = 512;
 constexpr int TC_SMEM_LIMIT = 232448;   // 227 KB opt-in per CTA
@@ -184,7 +185,7 @@ static bool tc_plan(int F, int P, int C, int k, bool pair, TcPlan& pl, bool norm
 }
 
 template <bool PAIR, bool NORM>
-__global__ void __launch_bounds__(TC_THREADS + (NORM ? 128 : 0), 1)
+__global__ void __launch_bounds__(TC_THREADS + (NORM ? 32 * TC_XF_WARPS : 0), 1)
     temporal_conv_tc_kernel(const __grid_constant__ CUtensorMap tmx,
                             const __grid_constant__ CUtensorMap tmw,
                             const __grid_constant__ CUtensorMap tmy, const TcPlan pl,
@@ -224,7 +225,7 @@ __global__ void __launch_bounds__(TC_THREADS + (NORM ? 128 : 0), 1)
     }
     mbar_init(drain, 1);
     if (NORM)
-      for (int i = 0; i < pl.sa; ++i) mbar_init(a_ready + 8 * i, 4);
+      for (int i = 0; i < pl.sa; ++i) mbar_init(a_ready + 8 * i, TC_XF_WARPS);
     fence_barrier_init();
   }
   for (int c = threadIdx.x; c < pl.C; c += blockDim.x) bias_s[c] = to_f32(args.bias[c]);
@@ -433,8 +434,9 @@ __global__ void __launch_bounds__(TC_THREADS + (NORM ? 128 : 0), 1)
     if constexpr (NORM) {
       const float4* coef_s = reinterpret_cast<const float4*>(smem_raw + (sCoef - smem_u32(smem_raw)));
       uint4* stage0 = reinterpret_cast<uint4*>(smem_raw + (sA - smem_u32(smem_raw)));
-      // Thread tt always handles physical chunk pc of rows r0, r0+16, ...; all
-      // those rows share r mod 8, so the logical chunk (its 8 channels) is fixed.
+      // Thread tt always handles physical chunk pc of rows r0, r0 + 4 TC_XF_WARPS,
+      // ...; all those rows share r mod 8, so the logical chunk (its 8
+      // channels) is fixed.
       const int tt = threadIdx.x - TC_THREADS;
       const int pc = tt & 7, r0 = tt >> 3;
       const int c = pc ^ (r0 & 7);
@@ -461,7 +463,7 @@ __global__ void __launch_bounds__(TC_THREADS + (NORM ? 128 : 0), 1)
           for (int mt = 0; mt < 2; ++mt) {
             if (mt >= pl.MT) break;
             uint4* st = stage0 + (size_t)sa * (pl.a_stage / 16) + (size_t)mt * (pl.a_tile / 16);
-            for (int r = r0; r < pl.a_rows; r += 16) {
+            for (int r = r0; r < pl.a_rows; r += 4 * TC_XF_WARPS) {
               const int f = f_first[mt] + r;
               if (f < 0 || f >= pl.F) continue;
               float v[8];
@@ -621,7 +623,7 @@ static int tc_launch(const CUtensorMap& tmx, const CUtensorMap& tmw, const CUten
   }
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
-  cfg.blockDim = dim3(TC_THREADS + (NORM ? 128 : 0));
+  cfg.blockDim = dim3(TC_THREADS + (NORM ? 32 * TC_XF_WARPS : 0));
   cfg.dynamicSmemBytes = (size_t)pl.smem;
   cfg.stream = stream;
   long long grid;

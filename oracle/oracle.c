@@ -39,9 +39,21 @@ static double in_val(const void* base, int64_t idx, int dtype) {
   return (double)f;
 }
 
+#ifdef _OPENMP
+/* The process's default thread count, read before any call changes it. */
+static int all_threads(void) {
+  static int all = 0;
+  if (all == 0) all = omp_get_max_threads();
+  return all;
+}
+#endif
+
+/* nthreads > 0: that many threads for this call; 0: the process default (every
+   call sets it, so a one-thread call does not leave the next call on one thread). */
 static void set_threads(int nthreads) {
 #ifdef _OPENMP
-  if (nthreads > 0) omp_set_num_threads(nthreads);
+  const int all = all_threads();
+  omp_set_num_threads(nthreads > 0 ? nthreads : all);
 #else
   (void)nthreads;
 #endif
@@ -49,7 +61,7 @@ static void set_threads(int nthreads) {
 
 int oracle_max_threads(void) {
 #ifdef _OPENMP
-  return omp_get_max_threads();
+  return all_threads();
 #else
   return 1;
 #endif
