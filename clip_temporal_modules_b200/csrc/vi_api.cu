@@ -6,6 +6,8 @@
 #include <atomic>
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "ptx.cuh"
 #include "vi_internal.cuh"
 
@@ -435,26 +437,41 @@ int gn_shard_apply_entry(const void* x, const double* shard_stats, int W, const 
 
 }  // namespace
 
+// An NVTX range around every compute entry point, named after it, so that a
+// profiler's timeline (nsys, ncu's range filters) shows which call launched
+// which kernels.  Without a profiler attached the push/pop are no-ops.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+#define VI_RANGE() NvtxRange vi_nvtx_range_(__func__)
+
 extern "C" {
 
 int vi_dual_attn_shard(const void* q, const void* k_ext, const void* v_ext, const void* k_glob,
                        const void* v_glob, void* out, int F_loc, int N_loc, int clip0, int N,
                        int P, int heads, int d, int n_pre, int n_post, int n_global,
                        vi_stream_t stream) {
+  VI_RANGE();
   return attn_shard_entry(q, k_ext, v_ext, k_glob, v_glob, out, F_loc, N_loc, clip0, N, P, heads,
                           d, n_pre, n_post, n_global, stream);
 }
 int vi_temporal_conv_shard(const void* x_ext, const void* w, const void* b, void* y, int F_loc,
                            int P, int C, int k, vi_stream_t stream) {
+  VI_RANGE();
   return conv_shard_entry(x_ext, w, b, y, F_loc, P, C, k, stream);
 }
 int vi_groupnorm_shard_stats(const void* x, int F_loc, int P, int C, int groups, double* stats,
                              vi_stream_t stream) {
+  VI_RANGE();
   return gn_shard_stats_entry(x, F_loc, P, C, groups, stats, stream);
 }
 int vi_groupnorm_shard_apply(const void* x, const double* shard_stats, int W, const void* gamma,
                              const void* beta, void* y, int F_loc, int P, int C, int groups,
                              float eps, vi_stream_t stream) {
+  VI_RANGE();
   return gn_shard_apply_entry(x, shard_stats, W, gamma, beta, y, F_loc, P, C, groups, eps, stream);
 }
 
@@ -468,6 +485,7 @@ int vi_temporal_attention(const void* x, const void* w_qkv, const void* b_qkv, c
                           const void* b_out, void* out, void* workspace, int F, int N, int P,
                           int heads, int d, int n_pre, int n_post, int n_global,
                           vi_stream_t stream) {
+  VI_RANGE();
   return temporal_attention_entry(x, w_qkv, b_qkv, w_out, b_out, out, workspace, F, N, P, heads,
                                   d, n_pre, n_post, n_global, stream);
 }
@@ -516,31 +534,38 @@ int vi_take_device_errors(void) {
 
 int vi_dual_attn(const void* q, const void* k, const void* v, void* out, int F, int N, int P,
                  int heads, int d, int n_pre, int n_post, int n_global, vi_stream_t stream) {
+  VI_RANGE();
   return attn_entry<bf16>(q, k, v, out, F, N, P, heads, d, n_pre, n_post, n_global, stream);
 }
 int vi_dual_attn_f32(const void* q, const void* k, const void* v, void* out, int F, int N, int P,
                      int heads, int d, int n_pre, int n_post, int n_global, vi_stream_t stream) {
+  VI_RANGE();
   return attn_entry<float>(q, k, v, out, F, N, P, heads, d, n_pre, n_post, n_global, stream);
 }
 int vi_temporal_conv(const void* x, const void* w, const void* b, void* y, int F, int N, int P,
                      int C, int k, vi_stream_t stream) {
+  VI_RANGE();
   return conv_entry<bf16>(x, w, b, y, F, N, P, C, k, stream);
 }
 int vi_temporal_conv_f32(const void* x, const void* w, const void* b, void* y, int F, int N,
                          int P, int C, int k, vi_stream_t stream) {
+  VI_RANGE();
   return conv_entry<float>(x, w, b, y, F, N, P, C, k, stream);
 }
 int vi_groupnorm_conv(const void* x, const void* gamma, const void* beta, const void* w,
                       const void* b, void* y, int F, int N, int P, int C, int groups, float eps,
                       int k, vi_stream_t stream) {
+  VI_RANGE();
   return gn_conv_entry(x, gamma, beta, w, b, y, F, N, P, C, groups, eps, k, stream);
 }
 int vi_groupnorm_global(const void* x, const void* gamma, const void* beta, void* y, int F, int N,
                         int P, int C, int groups, float eps, vi_stream_t stream) {
+  VI_RANGE();
   return gn_entry<bf16>(x, gamma, beta, y, F, N, P, C, groups, eps, stream);
 }
 int vi_groupnorm_global_f32(const void* x, const void* gamma, const void* beta, void* y, int F,
                             int N, int P, int C, int groups, float eps, vi_stream_t stream) {
+  VI_RANGE();
   return gn_entry<float>(x, gamma, beta, y, F, N, P, C, groups, eps, stream);
 }
 
