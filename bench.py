@@ -375,7 +375,7 @@ def run_ours(args):
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": w.dtype,
-        "data": "synthetic (seeded SplitMix64 + Box-Muller, N(0,1) q/k/v/x, BASELINE distributions)",
+        "data": "synthetic (seeded SplitMix64 + Box-Muller; q/k/v/x N(0,1), conv w N(0,1/(kC)), GN x N(0.5,2))",
         "config": {"workload": w.name, "F": w.F, "N_clips": w.N, "P": w.P, "C": w.C,
                    "heads": w.heads, "d": w.d, "n_pre": w.n_pre, "n_post": w.n_post,
                    "n_global": w.n_global, "k": w.k, "groups": w.groups,

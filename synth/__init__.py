@@ -179,7 +179,7 @@ BY_NAME = {w.name: w for w in WORKLOADS}
 
 
 def dist(w: Workload, tensor: str):
-    """(mean, std) of each input tensor; second BASELINE parameter is a variance."""
+    """(mean, std) of each input tensor; the distributions are stated as N(mean, variance)."""
     return {
         "q": (0.0, 1.0), "k": (0.0, 1.0), "v": (0.0, 1.0),
         "conv_x": (0.0, 1.0),
