@@ -9,7 +9,7 @@ import subprocess
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-SRC = os.path.join(ROOT, "clip_temporal_modules_b200", "examples", "abi_check.c")
+SRC = os.path.join(ROOT, "tests", "abi_check.c")
 LIBDIR = os.path.join(ROOT, "clip_temporal_modules_b200")
 
 
