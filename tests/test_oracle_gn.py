@@ -89,3 +89,25 @@ def test_position_subset_equals_full_slice():
     full, _, _ = oracle.groupnorm_global(x, gamma, beta, F, N, G)
     sub, _, _ = oracle.groupnorm_global(x, gamma, beta, F, N, G, positions=[2, 0])
     np.testing.assert_array_equal(sub, full[[2, 0]])
+
+
+def test_pooled_statistics_of_equal_shards_equal_the_whole():
+    """The merge the shard calls use (mean of means; mean of var + squared
+    deviation of the shard mean) gives the statistics of the whole tensor when
+    the shards are equal in size -- checked against the oracle's GroupNorm
+    statistics of the whole tensor and of each shard."""
+    F, N, P, C, G = 64, 8, 3, 16, 4
+    x = synth.normal((P, F, C), 31, 0.5, 1.4, seed=9, dtype="f32")
+    g = np.ones(C, np.float32)
+    b = np.zeros(C, np.float32)
+    _, mean, var = oracle.groupnorm_global(x, g, b, F, N, G, want_y=False)
+    for W in (2, 4, 8):
+        Fl = F // W
+        parts = [oracle.groupnorm_global(np.ascontiguousarray(x[:, r * Fl:(r + 1) * Fl]), g, b,
+                                         Fl, N // W, G, want_y=False)[1:] for r in range(W)]
+        m = np.stack([p[0] for p in parts])
+        v = np.stack([p[1] for p in parts])
+        pooled_mean = m.mean(axis=0)
+        pooled_var = (v + (m - pooled_mean) ** 2).mean(axis=0)
+        np.testing.assert_allclose(pooled_mean, mean, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(pooled_var, var, rtol=1e-12, atol=0)
