@@ -393,6 +393,11 @@ def run_ours(args):
     result["attn_ablations"] = attn_ablations(w, d, out, stream)
     result["groupnorm_conv_fused"] = fused_gn_conv(w, d, y, z, stream)
     result["temporal_attention_module"] = attention_module(w, d, out, y, z, stream)
+    if w.dtype == "bf16" and w.F % 8 == 0 and w.N % 8 == 0:
+        try:
+            result["clip_parallel_emulated"] = clip_parallel_emulated(w, d, stream)
+        except Exception as e:       # an extra figure: never lose the headline line over it
+            result["clip_parallel_emulated"] = {"error": f"{type(e).__name__}: {e}"[:300]}
 
     if not args.no_e2e:
         result["e2e"] = run_e2e(args, w, host, dev, stream)
@@ -493,6 +498,59 @@ def attention_module(w, d, out, y, z, stream, reps=5):
     flops = 4 * 2 * w.C * w.C * w.tokens
     return {"ms": round(ms, 4), "tokens_per_s": round(w.tokens / (ms / 1e3), 1),
             "projection_tflops_total": round(flops / 1e12, 3)}
+
+
+def clip_parallel_emulated(w, d, stream, world=8, reps=5):
+    """The per-shard kernels of clip parallelism (frames sharded over `world`
+    GPUs), emulated on this GPU: each shard's neighbourhood is cut from the
+    whole tensors beforehand (what the exchange would deliver), then the shard
+    calls of every shard run back to back and are timed.  The exchange itself
+    (NCCL) is not part of this figure."""
+    import torch
+
+    from clip_temporal_modules_b200._binding import (dual_attn_shard, groupnorm_shard_apply,
+                                                     groupnorm_shard_stats, temporal_conv_shard)
+    from clip_temporal_modules_b200.clip_parallel import (ShardLayout, extended_from_full,
+                                                          global_frame_index)
+    lays = [ShardLayout(w.F, w.N, world, r) for r in range(world)]
+    gidx = global_frame_index(w.F, w.n_global)
+    kg, vg = d["k"][:, gidx].contiguous(), d["v"][:, gidx].contiguous()
+    shards = []
+    for lay in lays:
+        f0, f1 = lay.f0, lay.f0 + lay.F_loc
+        q = d["q"][:, f0:f1].contiguous()
+        shards.append({"q": q, "k": extended_from_full(d["k"], f0, f1, 8),
+                       "v": extended_from_full(d["v"], f0, f1, 8),
+                       "x": extended_from_full(d["conv_x"], f0, f1, w.k // 2),
+                       "g": d["gn_x"][:, f0:f1].contiguous(), "out": torch.empty_like(q),
+                       "y": torch.empty_like(q), "z": torch.empty_like(q)})
+
+    def run():
+        for lay, sh in zip(lays, shards):
+            dual_attn_shard(sh["q"], sh["k"], sh["v"], kg, vg, sh["out"], N_loc=lay.N_loc,
+                            clip0=lay.clip0, N=w.N, heads=w.heads, n_pre=w.n_pre,
+                            n_post=w.n_post, n_global=w.n_global)
+        for sh in shards:
+            temporal_conv_shard(sh["x"], d["conv_w"], d["conv_b"], sh["y"])
+        stats = torch.stack([groupnorm_shard_stats(sh["g"], groups=w.groups) for sh in shards])
+        for sh in shards:
+            groupnorm_shard_apply(sh["g"], stats, d["gn_gamma"], d["gn_beta"], sh["z"], eps=w.eps)
+
+    for _ in range(2):
+        run()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        run()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    del shards
+    torch.cuda.empty_cache()
+    return {"world": world, "ms_all_shards": round(ms, 4),
+            "tokens_per_s": round(w.tokens / (ms / 1e3), 1),
+            "what": f"{world} frame shards' kernels on one GPU, neighbourhoods prepared; "
+                    "exchange not included"}
 
 
 def run_e2e(args, w, host, dev, stream):
