@@ -7,7 +7,8 @@
  * parallelism and on the three temporal modules: dual-domain attention, the
  * temporal convolution, and GroupNorm.  The pages distribute the N clips of a
  * video over N GPUs and synchronise context between them; here all N clips
- * live on one GPU and each call partitions them inside one kernel grid.
+ * live on one GPU and each call partitions them inside one kernel grid (the
+ * *_shard calls at the end serve a video spread over several GPUs).
  *
  * Common conventions
  * ------------------
