@@ -21,13 +21,12 @@ Python here only marshals arguments; see _binding.py.
 """
 from ._binding import (LIB_PATH, ViError, dual_attn, dual_attn_shard,  # noqa: F401
                        groupnorm_conv, groupnorm_global, groupnorm_shard_apply,
-                       groupnorm_shard_stats, launch_count, lib, set_conv_tiles_per_job,
-                       take_device_errors, temporal_attention, temporal_conv,
-                       temporal_conv_shard)
+                       groupnorm_shard_stats, launch_count, lib, take_device_errors,
+                       temporal_attention, temporal_conv, temporal_conv_shard)
 from .host_pipeline import HostPipeline, StepShape  # noqa: F401
 
 __all__ = ["dual_attn", "temporal_conv", "groupnorm_global", "groupnorm_conv",
            "temporal_attention", "dual_attn_shard", "temporal_conv_shard",
            "groupnorm_shard_stats", "groupnorm_shard_apply", "take_device_errors",
-           "launch_count", "lib", "set_conv_tiles_per_job", "HostPipeline", "StepShape",
+           "launch_count", "lib", "HostPipeline", "StepShape",
            "ViError", "LIB_PATH"]

@@ -31,7 +31,6 @@ SIGNATURES = {
     "vi_groupnorm_conv": [_vp] * 6 + [_i] * 5 + [_f, _i, _vp],
     "vi_temporal_attention": [_vp] * 7 + [_i] * 8 + [_vp],
     "vi_selftest_wait_timeout": [_i, _vp],
-    "vi_set_conv_tiles_per_job": [_i],
     "vi_dual_attn_shard": [_vp] * 6 + [_i] * 10 + [_vp],
     "vi_temporal_conv_shard": [_vp] * 4 + [_i] * 4 + [_vp],
     "vi_groupnorm_shard_stats": [_vp] + [_i] * 4 + [_vp, _vp],
@@ -293,11 +292,48 @@ def launch_count() -> int:
     return int(lib().vi_launch_count())
 
 
-def set_conv_tiles_per_job(tiles: int) -> int:
-    """Tiles per job of the tensor-core conv (0 automatic, 1 or 2); returns the previous value."""
-    r = int(lib().vi_set_conv_tiles_per_job(int(tiles)))
-    _check("vi_set_conv_tiles_per_job", min(r, 0))
-    return r
+def conv_forced_tiles(x, w, b, out=None, *, N: int, tiles: int, stream=None):
+    """Test hook (not part of the ABI in vi.h): the bf16 tensor-core conv with
+    its tiles per job forced to 1 or 2, so that tests reach both job forms."""
+    import torch
+    if out is None:
+        out = torch.empty_like(x)
+    _dev(x, w, b, out)
+    P, F, C = x.shape
+    k = w.shape[2]
+    _shape(w, (C, C, k), "w")
+    _shape(b, (C,), "b")
+    _shape(out, x.shape, "out")
+    fn = lib().vitest_temporal_conv_tiles
+    fn.argtypes = [_vp] * 4 + [_i] * 6 + [_vp]
+    fn.restype = ctypes.c_int
+    _check("vitest_temporal_conv_tiles", fn(x.data_ptr(), w.data_ptr(), b.data_ptr(),
+                                            out.data_ptr(), F, N, P, C, k, int(tiles),
+                                            _stream_ptr(stream)))
+    return out
+
+
+def groupnorm_conv_forced_tiles(x, gamma, beta, w, b, out=None, *, N: int, groups: int,
+                                tiles: int, eps: float = 1e-5, stream=None):
+    """Test hook (not part of the ABI in vi.h): the fused GroupNorm -> conv with
+    the conv's tiles per job forced to 1 or 2."""
+    import torch
+    if out is None:
+        out = torch.empty_like(x)
+    _dev(x, gamma, beta, w, b, out)
+    P, F, C = x.shape
+    _shape(w, (C, C, w.shape[2]), "w")
+    for t, n in ((gamma, "gamma"), (beta, "beta"), (b, "b")):
+        _shape(t, (C,), n)
+    _shape(out, x.shape, "out")
+    fn = lib().vitest_groupnorm_conv_tiles
+    fn.argtypes = [_vp] * 6 + [_i] * 5 + [_f, _i, _i, _vp]
+    fn.restype = ctypes.c_int
+    _check("vitest_groupnorm_conv_tiles", fn(
+        x.data_ptr(), gamma.data_ptr(), beta.data_ptr(), w.data_ptr(), b.data_ptr(),
+        out.data_ptr(), F, N, P, C, groups, float(eps), w.shape[2], int(tiles),
+        _stream_ptr(stream)))
+    return out
 
 
 def take_device_errors() -> None:

@@ -15,13 +15,18 @@ namespace vi {
 
 static __device__ unsigned int g_device_error = 0u;
 
+// The symbol's device address, looked up once per device.  Host threads may
+// race on the first lookup; each stores the same address.
 unsigned int* device_error_word() {
-  static void* cached[64] = {nullptr};
+  static std::atomic<void*> cached[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  if (!cached[dev] && cudaGetSymbolAddress(&cached[dev], g_device_error) != cudaSuccess)
-    cached[dev] = nullptr;
-  return static_cast<unsigned int*>(cached[dev]);
+  void* p = cached[dev].load(std::memory_order_acquire);
+  if (!p) {
+    if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+    cached[dev].store(p, std::memory_order_release);
+  }
+  return static_cast<unsigned int*>(p);
 }
 
 // Kernel launchers (defined next to their kernels).
@@ -44,10 +49,12 @@ template <typename T>
 int temporal_conv_generic_launch(const T*, const T*, const T*, T*, int, int, int, int,
                                  cudaStream_t);
 int temporal_conv_bf16_tc(const bf16*, const bf16*, const bf16*, bf16*, int, int, int, int,
-                          cudaStream_t, const float* coef = nullptr);
+                          cudaStream_t, const float* coef = nullptr, int mt = 0);
+int linear_bf16_tc(const bf16*, const bf16*, const bf16*, bf16* const*, int, int, int, int, int,
+                   cudaStream_t);
 bool temporal_conv_tc_ok(int F, int P, int C, int k);
 bool temporal_conv_tc_norm_ok(int F, int P, int C, int k);
-int conv_set_tiles_per_job(int mt);
+bool linear_tc_ok(int F, int P, int C, int Cout, int n_out);
 template <typename T>
 int gn_stats_launch(const T*, const T*, const T*, int64_t, int, int, float, void*, cudaStream_t,
                     const float**);
@@ -252,7 +259,7 @@ int gn_entry(const void* x, const void* gamma, const void* beta, void* y, int F,
 
 int gn_conv_entry(const void* x, const void* gamma, const void* beta, const void* w,
                   const void* b, void* y, int F, int N, int P, int C, int groups, float eps, int k,
-                  vi_stream_t stream) {
+                  vi_stream_t stream, int mt = 0) {
   using T = bf16;
   int st = check_clips(F, N, P, C);
   if (st < 0) return st;
@@ -283,7 +290,8 @@ int gn_conv_entry(const void* x, const void* gamma, const void* beta, const void
                             static_cast<const T*>(beta), rows, C, groups, eps, scratch, s, &coef);
   if (st == VI_OK)
     st = temporal_conv_bf16_tc(static_cast<const T*>(x), static_cast<const T*>(w),
-                               static_cast<const T*>(b), static_cast<T*>(y), F, P, C, k, s, coef);
+                               static_cast<const T*>(b), static_cast<T*>(y), F, P, C, k, s, coef,
+                               mt);
   if (scratch_free(scratch, s) != cudaSuccess && st == VI_OK) st = VI_ERR_CUDA;
   return st;
 }
@@ -316,19 +324,18 @@ int temporal_attention_entry(const void* x, const void* w_qkv, const void* b_qkv
       overlaps(workspace, ws, b_qkv, 3 * C * sizeof(T)) ||
       overlaps(workspace, ws, b_out, C * sizeof(T)))
     return VI_ERR_INVALID_ARG;
-  if (!temporal_conv_tc_ok(F, P, C, 1)) return VI_ERR_UNSUPPORTED;
+  if (!temporal_conv_tc_ok(F, P, C, 1) || !linear_tc_ok(F, P, C, 3 * C, 3))
+    return VI_ERR_UNSUPPORTED;
   cudaStream_t s = as_stream(stream);
   const T* xx = static_cast<const T*>(x);
-  const T* wq = static_cast<const T*>(w_qkv);
-  const T* bq = static_cast<const T*>(b_qkv);
   T* q = static_cast<T*>(workspace);
   T* k = q + (size_t)P * F * C;
   T* v = k + (size_t)P * F * C;
   T* a = v + (size_t)P * F * C;
   T* qkv[3] = {q, k, v};
-  for (int i = 0; i < 3 && st == VI_OK; ++i)   // single-tap conv = per-frame linear layer
-    st = temporal_conv_bf16_tc(xx, wq + (size_t)i * C * C, bq + (size_t)i * C, qkv[i], F, P, C, 1,
-                               s);
+  // q, k and v from one GEMM of N = 3C over x (rows of w_qkv in q, k, v order).
+  st = linear_bf16_tc(xx, static_cast<const T*>(w_qkv), static_cast<const T*>(b_qkv), qkv, 3, F,
+                      P, C, 3 * C, s);
   if (st == VI_OK) {
     if (dual_attn_fast_ok(F, N, d, n_pre, n_post, n_global))
       st = dual_attn_bf16_fast(q, k, v, a, F, N, P, heads, n_pre, n_post, n_global, s);
@@ -517,9 +524,34 @@ int vi_selftest_wait_timeout(int limit_us, vi_stream_t stream) {
   return VI_OK;
 }
 
-int vi_set_conv_tiles_per_job(int tiles) {
-  if (tiles < 0 || tiles > 2) return VI_ERR_INVALID_ARG;
-  return conv_set_tiles_per_job(tiles);
+// Test hook, not part of the ABI in vi.h: the bf16 conv with its tiles per
+// job forced to 1 or 2, so that tests reach both job forms of the tensor-core
+// kernel.  Same checks as vi_temporal_conv; shapes the tensor-core path does
+// not take return VI_ERR_UNSUPPORTED.
+int vitest_temporal_conv_tiles(const void* x, const void* w, const void* b, void* y, int F,
+                               int N, int P, int C, int k, int tiles, vi_stream_t stream) {
+  if (tiles != 1 && tiles != 2) return VI_ERR_INVALID_ARG;
+  int st = check_clips(F, N, P, C);
+  if (st < 0) return st;
+  if (k <= 0 || k % 2 == 0 || k / 2 > F / N) return VI_ERR_INVALID_ARG;
+  if (st == kEmpty) return VI_OK;
+  if (!x || !w || !b || !y) return VI_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w) || !aligned16(b) || !aligned16(y)) return VI_ERR_ALIGNMENT;
+  const size_t bytes = (size_t)P * F * C * sizeof(bf16);
+  if (overlaps(y, bytes, x, bytes)) return VI_ERR_INVALID_ARG;
+  if (!temporal_conv_tc_ok(F, P, C, k)) return VI_ERR_UNSUPPORTED;
+  return temporal_conv_bf16_tc(static_cast<const bf16*>(x), static_cast<const bf16*>(w),
+                               static_cast<const bf16*>(b), static_cast<bf16*>(y), F, P, C, k,
+                               as_stream(stream), nullptr, tiles);
+}
+
+// Test hook, not part of the ABI in vi.h: vi_groupnorm_conv with the conv's
+// tiles per job forced to 1 or 2.
+int vitest_groupnorm_conv_tiles(const void* x, const void* gamma, const void* beta,
+                                const void* w, const void* b, void* y, int F, int N, int P, int C,
+                                int groups, float eps, int k, int tiles, vi_stream_t stream) {
+  if (tiles != 1 && tiles != 2) return VI_ERR_INVALID_ARG;
+  return gn_conv_entry(x, gamma, beta, w, b, y, F, N, P, C, groups, eps, k, stream, tiles);
 }
 
 int vi_take_device_errors(void) {

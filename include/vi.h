@@ -95,17 +95,6 @@ unsigned long long vi_launch_count(void);
 int vi_selftest_wait_timeout(int limit_us, vi_stream_t stream);
 
 /*
- * Tuning knob of the bf16 tensor-core conv (vi_temporal_conv and the
- * projections of vi_temporal_attention): how many 128-frame tiles one job of
- * a CTA covers.  0 = automatic (2 where that keeps the widest output-channel
- * slab, else 1), 1 or 2 = that form wherever its plan fits.  Both forms give
- * the same result up to fp32 summation order.  Process-wide; returns the
- * previous setting, or VI_ERR_INVALID_ARG for a value outside 0..2.  It has no
- * counterpart in the method: it exists for measurement and tests.
- */
-int vi_set_conv_tiles_per_job(int tiles);
-
-/*
  * Dual-domain temporal attention (attention-module paragraph of the source).
  *
  * For every position p, head h and clip i (frames [s, e), s = i*L, e = s+L),
@@ -185,8 +174,10 @@ int vi_groupnorm_global_f32(const void* x, const void* gamma, const void* beta, 
  *   q = x Wq^T + bq,  k = x Wk^T + bk,  v = x Wv^T + bv      (per frame)
  *   a = vi_dual_attn(q, k, v; heads, d, n_pre, n_post, n_global)
  *   out = a Wo^T + bo
- * Each stage is a separate kernel writing a bf16 tensor (the projections run
- * on the tensor-core temporal-conv kernel with a single tap).
+ * The three input projections are ONE tensor-core GEMM of N = 3C over x
+ * (the temporal-conv kernel with a single tap, its output channels split
+ * into the q, k and v tensors), then the attention kernel, then the output
+ * projection GEMM; each stage writes a bf16 tensor.
  *
  * x, out : [P][F][C], C = heads*d;  w_qkv : [3C][C] (rows Wq, Wk, Wv, PyTorch
  * Linear layout);  b_qkv : [3C];  w_out : [C][C];  b_out : [C].
@@ -238,13 +229,21 @@ int vi_groupnorm_conv(const void* x, const void* gamma, const void* beta, const 
  *                every GPU which loads the library holds until the process
  *                exits).  A call whose scratch need is larger returns
  *                VI_ERR_UNSUPPORTED before launching anything.  The need is
- *                about 64 + 16*groups + 16*C + 24*groups*B bytes, B being the
- *                number of streaming blocks (at most the SM count); on a
- *                148-SM B200 that admits, e.g., 32 groups with C up to ~58000
- *                or 256 groups with C up to ~8000.
+ *                64 + 16*groups + 16*C + 24*groups*B bytes (each term rounded
+ *                up to 64 bytes), B being the partial-sum records per group:
+ *                at most the SM count on the streaming path, and at most
+ *                8*SMs/groups + 1 on the path for rows of more than 960
+ *                16-byte vectors or 32 KB, or groups that split a 16-byte
+ *                vector (there the last term is at most 24*(8*SMs + groups)).
+ *                On a 148-SM B200 the streaming path admits, e.g., 32 groups
+ *                with C up to ~58000 or 256 groups with C up to ~8000.
  * First call   : the first call on each device looks up the array's device
  *                address with that device current (cudaGetSymbolAddress) and
- *                caches it; make that first call before any stream capture.
+ *                caches it.  It may also load the library's GPU code (CUDA
+ *                loads modules lazily), which allocates device memory.  A
+ *                caller whose running phase must not allocate should therefore
+ *                make one call during its setup, before any stream capture;
+ *                later calls allocate nothing.
  * Sharing      : every call uses the same array.  Each call clears the part
  *                that must start at zero and rewrites the rest, but calls
  *                whose work overlaps on the GPU (different streams, or several

@@ -164,14 +164,23 @@ def test_temporal_attention_workspace_bytes(L):
     assert L.vi_temporal_attention_workspace_bytes(0, 1, 1) == 0
 
 
-def test_conv_tiles_per_job_knob(L):
-    """The tuning knob takes 0..2, returns the previous value, and needs no GPU."""
-    assert L.vi_set_conv_tiles_per_job(3) == -1
-    assert L.vi_set_conv_tiles_per_job(-1) == -1
-    prev = L.vi_set_conv_tiles_per_job(1)
-    assert prev in (0, 1, 2)
-    assert L.vi_set_conv_tiles_per_job(2) == 1
-    assert L.vi_set_conv_tiles_per_job(prev) == 2
+def test_no_global_tuning_state_in_the_abi(L):
+    """Tiles per job is chosen per call: the ABI has no setter, and the test
+    hooks that force a job form take it as an argument and check it on the
+    host (no GPU here, so anything launched would have failed)."""
+    assert not hasattr(L, "vi_set_conv_tiles_per_job")
+    assert "tiles" not in open(HEADER).read()
+    conv_t = L.vitest_temporal_conv_tiles
+    conv_t.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int] * 6 + [ctypes.c_void_p]
+    gnconv_t = L.vitest_groupnorm_conv_tiles
+    gnconv_t.argtypes = [ctypes.c_void_p] * 6 + [ctypes.c_int] * 5 + [
+        ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]
+    for tiles in (0, 3, -1):
+        assert conv_t(A, B, Cp, D, 64, 4, 2, 64, 3, tiles, None) == INVALID
+        assert gnconv_t(A, B, Cp, D, A, B, 64, 4, 2, 64, 8, 1e-5, 3, tiles, None) == INVALID
+    assert conv_t(None, None, None, None, 64, 4, 0, 64, 3, 1, None) == OK     # empty
+    assert conv_t(A, B, Cp, D, 64, 4, 2, 64, 2, 1, None) == INVALID         # even k
+    assert conv_t(A + 4, B, Cp, D, 64, 4, 2, 64, 3, 2, None) == ALIGN
 
 
 def test_empty_calls_succeed_without_touching_pointers(L):

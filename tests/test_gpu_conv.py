@@ -72,8 +72,11 @@ def test_result_does_not_depend_on_clip_count(cuda_device):
 def test_one_and_two_tiles_per_job(cuda_device, w, tiles):
     """Both job forms of the tensor-core conv (one 128-frame tile per job, or
     two sharing every weight stage; odd tile counts leave a zero tile)."""
-    prev = vi.set_conv_tiles_per_job(tiles)
-    try:
-        run_case(w)
-    finally:
-        vi.set_conv_tiles_per_job(prev)
+    from clip_temporal_modules_b200._binding import conv_forced_tiles
+    x, wt, b = (synth.make(w, t) for t in ("conv_x", "conv_w", "conv_b"))
+    dx, dw, db = (to_device(a, w.dtype) for a in (x, wt, b))
+    y = conv_forced_tiles(dx, dw, db, N=w.N, tiles=tiles)
+    torch.cuda.synchronize()
+    vi.take_device_errors()
+    ref = oracle.temporal_conv(x, wt, b, w.F, w.N, w.k)
+    assert_close(from_device(y), ref, w.dtype, "conv", w.name)

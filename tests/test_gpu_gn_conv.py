@@ -90,8 +90,12 @@ def test_unsupported_channel_count_is_reported(cuda_device):
 def test_one_and_two_tiles_per_job(cuda_device, w, tiles):
     """Both job forms of the fused conv (the transform warps normalise one or
     two x boxes per stage)."""
-    prev = vi.set_conv_tiles_per_job(tiles)
-    try:
-        run_case(w)
-    finally:
-        vi.set_conv_tiles_per_job(prev)
+    from clip_temporal_modules_b200._binding import groupnorm_conv_forced_tiles
+    x, g, bt, wt, b = inputs(w)
+    dev = [to_device(a, w.dtype) for a in (x, g, bt, wt, b)]
+    y = groupnorm_conv_forced_tiles(*dev, N=w.N, groups=w.groups, eps=w.eps, tiles=tiles)
+    torch.cuda.synchronize()
+    vi.take_device_errors()
+    ref = oracle.groupnorm_conv(x, g, bt, wt, b, w.F, w.N, w.groups, w.eps, w.k,
+                                intermediate="bf16")
+    assert_close(from_device(y), ref, w.dtype, "gn", w.name)
