@@ -31,8 +31,8 @@ SIGNATURES = {
     "vi_groupnorm_conv": [_vp] * 6 + [_i] * 5 + [_f, _i, _vp],
     "vi_temporal_attention": [_vp] * 7 + [_i] * 8 + [_vp],
     "vi_selftest_wait_timeout": [_i, _vp],
-    "vi_dual_attn_shard": [_vp] * 6 + [_i] * 10 + [_vp],
-    "vi_temporal_conv_shard": [_vp] * 4 + [_i] * 4 + [_vp],
+    "vi_dual_attn_shard": [_vp] * 6 + [_i] * 11 + [_vp],
+    "vi_temporal_conv_shard": [_vp] * 4 + [_i] * 5 + [_vp],
     "vi_groupnorm_shard_stats": [_vp] + [_i] * 4 + [_vp, _vp],
     "vi_groupnorm_shard_apply": [_vp, _vp, _i, _vp, _vp, _vp] + [_i] * 4 + [_f, _vp],
     "vi_version": [],
@@ -208,11 +208,12 @@ def temporal_attention(x, w_qkv, b_qkv, w_out, b_out, out=None, workspace=None, 
 
 def dual_attn_shard(q, k_ext, v_ext, k_glob, v_glob, out=None, *, N_loc: int, clip0: int,
                     N: int, heads: int, n_pre: int = 8, n_post: int = 8, n_global: int = 16,
-                    stream=None):
+                    part: int = 0, stream=None):
     """Dual-domain attention of one shard of a video cut along frames (bf16).
 
-    q, out [P][F_loc][C]; k_ext, v_ext [P][F_loc + 16][C] (8 frames before and
-    after the shard around it); k_glob, v_glob [P][n_global][C]."""
+    q, out [P][F_loc][C]; k_ext, v_ext [P][F_loc + 16][C] (halo-padded: 8
+    frames before and after the shard around it); k_glob, v_glob
+    [P][n_global][C]; part 0 all, 1 interior blocks, 2 boundary blocks."""
     import torch
     if out is None:
         out = torch.empty_like(q)
@@ -229,12 +230,13 @@ def dual_attn_shard(q, k_ext, v_ext, k_glob, v_glob, out=None, *, N_loc: int, cl
     _check("vi_dual_attn_shard", lib().vi_dual_attn_shard(
         q.data_ptr(), k_ext.data_ptr(), v_ext.data_ptr(), k_glob.data_ptr(), v_glob.data_ptr(),
         out.data_ptr(), F_loc, N_loc, clip0, N, P, heads, C // heads, n_pre, n_post, n_global,
-        _stream_ptr(stream)))
+        int(part), _stream_ptr(stream)))
     return out
 
 
-def temporal_conv_shard(x_ext, w, b, out=None, *, stream=None):
-    """Temporal conv of one shard: x_ext [P][F_loc + 2(k/2)][C] -> [P][F_loc][C] (bf16)."""
+def temporal_conv_shard(x_ext, w, b, out=None, *, part: int = 0, stream=None):
+    """Temporal conv of one shard: x_ext [P][F_loc + 2(k/2)][C] (halo-padded)
+    -> [P][F_loc][C] (bf16); part 0 all, 1 interior blocks, 2 boundary blocks."""
     import torch
     _dev(x_ext, w, b)
     if w.dim() != 3:
@@ -249,7 +251,7 @@ def temporal_conv_shard(x_ext, w, b, out=None, *, stream=None):
     _shape(b, (C,), "b")
     _shape(out, (P, F_loc, C), "out")
     _check("vi_temporal_conv_shard", lib().vi_temporal_conv_shard(
-        x_ext.data_ptr(), w.data_ptr(), b.data_ptr(), out.data_ptr(), F_loc, P, C, k,
+        x_ext.data_ptr(), w.data_ptr(), b.data_ptr(), out.data_ptr(), F_loc, P, C, k, int(part),
         _stream_ptr(stream)))
     return out
 

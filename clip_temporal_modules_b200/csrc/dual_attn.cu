@@ -156,9 +156,12 @@ struct FaMaps {
 // a video of n_total clips (which decides the absent ends), and frame 0 of
 // the q map is row kv_off of the k/v maps (0 for a whole video on one GPU,
 // the halo width for a shard whose neighbours' frames are stacked around it).
+// The grid covers the selected clip blocks of every (position, head): blocks
+// [0, sel_lo) and [sel_hi0, sel_hi0 + n_sel - sel_lo).
 __global__ void __launch_bounds__(256) dual_attn_bf16_mma(const __grid_constant__ FaMaps maps,
-                                                          int F, int N, int heads, int nblk,
-                                                          int n_pre, int n_post, int n_global,
+                                                          int F, int N, int heads, int sel_lo,
+                                                          int sel_hi0, int n_sel, int n_pre,
+                                                          int n_post, int n_global,
                                                           float scale_log2, int kv_off, int clip0,
                                                           int n_total, unsigned int* err_word) {
   extern __shared__ uint8_t smem_raw[];
@@ -166,9 +169,10 @@ __global__ void __launch_bounds__(256) dual_attn_bf16_mma(const __grid_constant_
   const uint32_t sQ = base + FA_OFF_Q, sKW = base + FA_OFF_KW, sVW = base + FA_OFF_VW;
   const uint32_t sKG = base + FA_OFF_KG, sVG = base + FA_OFF_VG, bar = base + FA_OFF_BAR;
 
-  const int blk = blockIdx.x % nblk;
-  const int h = (blockIdx.x / nblk) % heads;
-  const int p = blockIdx.x / (nblk * heads);
+  const int sb = blockIdx.x % n_sel;
+  const int blk = sb < sel_lo ? sb : sel_hi0 + (sb - sel_lo);
+  const int h = (blockIdx.x / n_sel) % heads;
+  const int p = blockIdx.x / (n_sel * heads);
   const int f0 = blk * FA_ROWS_Q;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -343,7 +347,7 @@ int dual_attn_bf16_fast(const bf16* q, const bf16* k, const bf16* v, bf16* out, 
   unsigned int* err = device_error_word();
   if (!err) return VI_ERR_CUDA;
   dual_attn_bf16_mma<<<(unsigned)grid, 256, FA_SMEM_BYTES, stream>>>(
-      maps, F, N, heads, nblk, n_pre, n_post, n_global, scale_log2, 0, 0, N, err);
+      maps, F, N, heads, nblk, 0, nblk, n_pre, n_post, n_global, scale_log2, 0, 0, N, err);
   VI_LAUNCHED();
   return VI_OK;
 }
@@ -356,7 +360,7 @@ int dual_attn_bf16_fast(const bf16* q, const bf16* k, const bf16* v, bf16* out, 
 // hold the video's global frames.
 int dual_attn_bf16_shard(const bf16* q, const bf16* k_ext, const bf16* v_ext, const bf16* k_glob,
                          const bf16* v_glob, bf16* out, int F_loc, int N_loc, int clip0, int N,
-                         int P, int heads, int n_pre, int n_post, int n_global,
+                         int P, int heads, int n_pre, int n_post, int n_global, int part,
                          cudaStream_t stream) {
   const int C = heads * 64;
   const int F_ext = F_loc + 2 * FA_HALO;
@@ -392,14 +396,24 @@ int dual_attn_bf16_shard(const bf16* q, const bf16* k_ext, const bf16* v_ext, co
     if (dev >= 0 && dev < 64) attr_set[dev].store(true, std::memory_order_release);
   }
   const int nblk = (N_loc + FA_CLIPS - 1) / FA_CLIPS;
-  const int64_t grid = (int64_t)P * heads * nblk;
+  // Interior blocks [a, b): their k/v window (8 rows on each side of the
+  // block) lies inside the shard's own frames.  The others are the boundary.
+  const int a = nblk < 1 ? nblk : 1, b = nblk - 1 > a ? nblk - 1 : a;
+  int sel_lo = nblk, sel_hi0 = 0, n_sel = nblk;
+  if (part == VI_PART_INTERIOR) {
+    sel_lo = 0; sel_hi0 = a; n_sel = b - a;
+  } else if (part == VI_PART_BOUNDARY) {
+    sel_lo = a; sel_hi0 = b; n_sel = a + (nblk - b);
+  }
+  if (n_sel == 0) return VI_OK;              // nothing in this part
+  const int64_t grid = (int64_t)P * heads * n_sel;
   if (grid > 0x7fffffff) return VI_ERR_UNSUPPORTED;
   const float scale_log2 = 1.4426950408889634f / 8.0f;    // log2(e) / sqrt(64)
   unsigned int* err = device_error_word();
   if (!err) return VI_ERR_CUDA;
   dual_attn_bf16_mma<<<(unsigned)grid, 256, FA_SMEM_BYTES, stream>>>(
-      maps, F_loc, N_loc, heads, nblk, n_pre, n_post, n_global, scale_log2, FA_HALO, clip0, N,
-      err);
+      maps, F_loc, N_loc, heads, sel_lo, sel_hi0, n_sel, n_pre, n_post, n_global, scale_log2,
+      FA_HALO, clip0, N, err);
   VI_LAUNCHED();
   return VI_OK;
 }

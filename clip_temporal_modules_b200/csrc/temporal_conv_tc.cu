@@ -82,7 +82,9 @@ struct TcPlan {
   int n_slabs;           // Cout / NJ
   int slabs_per_out;     // slabs of one output tensor
   int n_fblk;            // ceil(F / 128)
-  long long n_tiles;     // P * n_fblk
+  int sel_lo, sel_hi0, n_sel;   // frame blocks computed per position: [0, sel_lo) and
+                                // [sel_hi0, sel_hi0 + n_sel - sel_lo) (all of them by default)
+  long long n_tiles;     // P * n_sel
   long long n_jobs;      // ceil(n_tiles / MT) * n_slabs
   int n_cb;              // C / 64
   int a_rows;            // 127 + k
@@ -169,6 +171,8 @@ static bool tc_plan(int F, int P, int C, int Cout, int n_out, int k, TcPlan& pl,
       pl.n_slabs = Cout / nj;
       pl.slabs_per_out = cpo / nj;
       pl.n_fblk = (F + TC_M - 1) / TC_M;
+      pl.sel_lo = pl.n_sel = pl.n_fblk;
+      pl.sel_hi0 = 0;
       pl.n_tiles = (long long)P * pl.n_fblk;
       pl.n_jobs = ((pl.n_tiles + mt - 1) / mt) * pl.n_slabs;
       pl.n_cb = C / TC_KB;
@@ -187,6 +191,14 @@ static bool tc_plan(int F, int P, int C, int Cout, int n_out, int k, TcPlan& pl,
     }
   }
   return false;
+}
+
+// Tile t of a launch -> its frame block and position (the launch covers the
+// plan's selected frame blocks of every position).
+__device__ __forceinline__ void tc_tile_pos(const TcPlan& pl, long long t, int& fb, int& p) {
+  const int s = (int)(t % pl.n_sel);
+  p = (int)(t / pl.n_sel);
+  fb = s < pl.sel_lo ? s : pl.sel_hi0 + (s - pl.sel_lo);
 }
 
 // The 4k MMAs of one tile and one K-block: k taps x 4 K steps of 16 channels.
@@ -329,9 +341,9 @@ __global__ void __launch_bounds__(TC_THREADS + (NORM ? 32 * TC_XF_WARPS : 0), 1)
       int frow[MT], pos[MT];
 #pragma unroll
       for (int m = 0; m < MT; ++m) {
-        const long long tile = tile0 + m;
-        frow[m] = (int)(tile % pl.n_fblk) * TC_M - halo + args.x_off;
-        pos[m] = (int)(tile / pl.n_fblk);
+        int fb;
+        tc_tile_pos(pl, tile0 + m, fb, pos[m]);
+        frow[m] = fb * TC_M - halo + args.x_off;
       }
       // Packed weights of (slab, K-block 0): k contiguous tap blocks per K-block.
       const bf16* wslab = args.wpk + (size_t)slab * pl.n_cb * (pl.b_kb / 2);
@@ -463,7 +475,11 @@ __global__ void __launch_bounds__(TC_THREADS + (NORM ? 32 * TC_XF_WARPS : 0), 1)
         const long long tile0 = (job / pl.n_slabs) * MT;
         int f_first[MT];                           // frame of row 0 of each tile's x box
 #pragma unroll
-        for (int mt = 0; mt < MT; ++mt) f_first[mt] = (int)((tile0 + mt) % pl.n_fblk) * TC_M - halo;
+        for (int mt = 0; mt < MT; ++mt) {
+          int fb, p;
+          tc_tile_pos(pl, tile0 + mt, fb, p);
+          f_first[mt] = fb * TC_M - halo;
+        }
         for (int ib = 0; ib < pl.n_cb && ok; ++ib) {
           const int cb = (ib + cb_rot) % pl.n_cb;
           float m[8], a[8], bt[8];
@@ -524,8 +540,8 @@ __global__ void __launch_bounds__(TC_THREADS + (NORM ? 32 * TC_XF_WARPS : 0), 1)
         }
         tc_fence_after();
         const long long tile = (job / pl.n_slabs) * MT + mt;
-        const int fb = (int)(tile % pl.n_fblk);
-        const int p = (int)(tile / pl.n_fblk);
+        int fb, p;
+        tc_tile_pos(pl, tile, fb, p);
         const bool tile_ok = tile < pl.n_tiles;
         const uint32_t taddr = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * pl.NJ);
         if constexpr (!NORM) {
@@ -702,7 +718,7 @@ static int tc_dispatch(const TcMaps& maps, const TcPlan& pl, const TcArgs& a, bo
 // mt: tiles per job, 0 = the default plan.
 static int tc_run(const bf16* x, int x_rows, int x_off, const bf16* w, const bf16* b,
                   bf16* const* ys, int n_out, int F, int P, int C, int Cout, int k,
-                  cudaStream_t stream, const float* coef, int mt) {
+                  cudaStream_t stream, const float* coef, int mt, int part = VI_PART_ALL) {
   TcPlan pl;
   const bool norm = coef != nullptr;
   if (mt != 0) {
@@ -718,6 +734,23 @@ static int tc_run(const bf16* x, int x_rows, int x_off, const bf16* w, const bf1
     if (k == 1 && pl.MT == 2 && !norm && tc_plan(F, P, C, Cout, n_out, k, pl2, false, 2, 2) &&
         pl2.NJ >= pl.NJ)
       pl = pl2;
+  }
+  if (part != VI_PART_ALL) {
+    // Frame blocks whose x rows (with the k/2 rows on each side) lie inside
+    // the shard are interior: [a, b).  The others are the boundary blocks.
+    const int h = k / 2;
+    const int a = pl.n_fblk < 1 ? pl.n_fblk : 1;
+    int b = (F - h) / TC_M;
+    if (b > pl.n_fblk) b = pl.n_fblk;
+    if (b < a) b = a;
+    if (part == VI_PART_INTERIOR) {
+      pl.sel_lo = 0; pl.sel_hi0 = a; pl.n_sel = b - a;
+    } else {
+      pl.sel_lo = a; pl.sel_hi0 = b; pl.n_sel = a + (pl.n_fblk - b);
+    }
+    pl.n_tiles = (long long)P * pl.n_sel;
+    pl.n_jobs = ((pl.n_tiles + pl.MT - 1) / pl.MT) * pl.n_slabs;
+    if (pl.n_sel == 0) return VI_OK;          // nothing in this part
   }
   unsigned int* err = device_error_word();
   if (!err) return VI_ERR_CUDA;
@@ -787,12 +820,13 @@ int linear_bf16_tc(const bf16* x, const bf16* w, const bf16* b, bf16* const* ys,
 // One shard of a video cut along frames: x_ext [P][F_loc + 2(k/2)][C] holds
 // the k/2 frames before the shard (zeros at the start of the video), the
 // shard's frames and the k/2 frames after it (zeros at the end); y is
-// [P][F_loc][C].
+// [P][F_loc][C].  part: every frame block, only those that read no halo row
+// (interior), or only the others (boundary).
 int temporal_conv_bf16_tc_shard(const bf16* x_ext, const bf16* w, const bf16* b, bf16* y,
-                                int F_loc, int P, int C, int k, cudaStream_t stream) {
+                                int F_loc, int P, int C, int k, int part, cudaStream_t stream) {
   bf16* ys[1] = {y};
   return tc_run(x_ext, F_loc + 2 * (k / 2), k / 2, w, b, ys, 1, F_loc, P, C, C, k, stream, nullptr,
-                0);
+                0, part);
 }
 
 }  // namespace vi

@@ -37,9 +37,9 @@ int dual_attn_bf16_fast(const bf16*, const bf16*, const bf16*, bf16*, int, int, 
                         int, int, cudaStream_t);
 bool dual_attn_fast_ok(int F, int N, int d, int n_pre, int n_post, int n_global);
 int dual_attn_bf16_shard(const bf16*, const bf16*, const bf16*, const bf16*, const bf16*, bf16*,
-                         int, int, int, int, int, int, int, int, int, cudaStream_t);
+                         int, int, int, int, int, int, int, int, int, int, cudaStream_t);
 int temporal_conv_bf16_tc_shard(const bf16*, const bf16*, const bf16*, bf16*, int, int, int, int,
-                                cudaStream_t);
+                                int, cudaStream_t);
 template <typename T>
 int gn_shard_stats(const T*, int64_t, int, int, double*, cudaStream_t);
 template <typename T>
@@ -352,8 +352,10 @@ int temporal_attention_entry(const void* x, const void* w_qkv, const void* b_qkv
 
 int attn_shard_entry(const void* q, const void* k_ext, const void* v_ext, const void* k_glob,
                      const void* v_glob, void* out, int F_loc, int N_loc, int clip0, int N, int P,
-                     int heads, int d, int n_pre, int n_post, int n_global, vi_stream_t stream) {
+                     int heads, int d, int n_pre, int n_post, int n_global, int part,
+                     vi_stream_t stream) {
   using T = bf16;
+  if (part < VI_PART_ALL || part > VI_PART_BOUNDARY) return VI_ERR_INVALID_ARG;
   if (heads <= 0 || d <= 0 || (int64_t)heads * d > 0x7fffffff) return VI_ERR_INVALID_ARG;
   const int C = heads * d;
   if (F_loc <= 0 || N_loc <= 0 || P < 0 || F_loc % N_loc != 0) return VI_ERR_INVALID_ARG;
@@ -379,12 +381,14 @@ int attn_shard_entry(const void* q, const void* k_ext, const void* v_ext, const 
   return dual_attn_bf16_shard(static_cast<const T*>(q), static_cast<const T*>(k_ext),
                               static_cast<const T*>(v_ext), static_cast<const T*>(k_glob),
                               static_cast<const T*>(v_glob), static_cast<T*>(out), F_loc, N_loc,
-                              clip0, N, P, heads, n_pre, n_post, n_global, as_stream(stream));
+                              clip0, N, P, heads, n_pre, n_post, n_global, part,
+                              as_stream(stream));
 }
 
 int conv_shard_entry(const void* x_ext, const void* w, const void* b, void* y, int F_loc, int P,
-                     int C, int k, vi_stream_t stream) {
+                     int C, int k, int part, vi_stream_t stream) {
   using T = bf16;
+  if (part < VI_PART_ALL || part > VI_PART_BOUNDARY) return VI_ERR_INVALID_ARG;
   if (F_loc <= 0 || P < 0 || C <= 0) return VI_ERR_INVALID_ARG;
   if (k <= 0 || k % 2 == 0) return VI_ERR_INVALID_ARG;
   if ((double)P * (double)(F_loc + k) * (double)C > 1.099511627776e12) return VI_ERR_UNSUPPORTED;
@@ -399,7 +403,7 @@ int conv_shard_entry(const void* x_ext, const void* w, const void* b, void* y, i
     return VI_ERR_INVALID_ARG;
   return temporal_conv_bf16_tc_shard(static_cast<const T*>(x_ext), static_cast<const T*>(w),
                                      static_cast<const T*>(b), static_cast<T*>(y), F_loc, P, C, k,
-                                     as_stream(stream));
+                                     part, as_stream(stream));
 }
 
 int gn_shard_check(int F_loc, int P, int C, int groups) {
@@ -459,16 +463,16 @@ extern "C" {
 
 int vi_dual_attn_shard(const void* q, const void* k_ext, const void* v_ext, const void* k_glob,
                        const void* v_glob, void* out, int F_loc, int N_loc, int clip0, int N,
-                       int P, int heads, int d, int n_pre, int n_post, int n_global,
+                       int P, int heads, int d, int n_pre, int n_post, int n_global, int part,
                        vi_stream_t stream) {
   VI_RANGE();
   return attn_shard_entry(q, k_ext, v_ext, k_glob, v_glob, out, F_loc, N_loc, clip0, N, P, heads,
-                          d, n_pre, n_post, n_global, stream);
+                          d, n_pre, n_post, n_global, part, stream);
 }
 int vi_temporal_conv_shard(const void* x_ext, const void* w, const void* b, void* y, int F_loc,
-                           int P, int C, int k, vi_stream_t stream) {
+                           int P, int C, int k, int part, vi_stream_t stream) {
   VI_RANGE();
-  return conv_shard_entry(x_ext, w, b, y, F_loc, P, C, k, stream);
+  return conv_shard_entry(x_ext, w, b, y, F_loc, P, C, k, part, stream);
 }
 int vi_groupnorm_shard_stats(const void* x, int F_loc, int P, int C, int groups, double* stats,
                              vi_stream_t stream) {

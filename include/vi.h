@@ -265,43 +265,66 @@ int vi_groupnorm_global_noalloc(const void* x, const void* gamma, const void* be
  * compute of that scheme; the exchange itself is the caller's (NCCL, or the
  * package's ClipParallel).  A shard holds F_loc consecutive frames of every
  * position; bf16 only.
+ *
+ * Halo-padded storage: the tensors whose neighbour frames a module reads
+ * (k and v of the attention, x of the conv) are taken as [P][F_loc + 2h][C]
+ * with the shard's frames at rows [h, h + F_loc) and h spare rows on each
+ * side.  The caller keeps its shard in that layout, and the exchange writes
+ * only the 2h halo rows of each position (zeros at the video ends), so no
+ * call copies the shard.
+ *
+ * part: which frame blocks a call computes.  VI_PART_ALL computes the whole
+ * shard.  VI_PART_INTERIOR computes only the blocks whose reads stay inside
+ * the shard's own frames (no halo row is read, so the call may run while the
+ * halo exchange is still in flight); VI_PART_BOUNDARY computes the others.
+ * INTERIOR followed by BOUNDARY gives the result of ALL.  A part with no
+ * block (e.g. INTERIOR of a shard of one block) is a valid empty call.
  */
+enum { VI_PART_ALL = 0, VI_PART_INTERIOR = 1, VI_PART_BOUNDARY = 2 };
 
 /*
  * Dual-domain attention of one shard (attention-module paragraph).
  *
  * q, out        : [P][F_loc][C], the shard's frames: clips clip0 ..
  *                 clip0 + N_loc - 1 of the video's N clips (L = F_loc / N_loc).
- * k_ext, v_ext  : [P][F_loc + 16][C]: the 8 frames before the shard, the
- *                 shard's F_loc frames, the 8 frames after it.  Rows past a
- *                 video end are masked out but are read: they must hold finite
- *                 values (zeros).
+ * k_ext, v_ext  : [P][F_loc + 16][C], halo-padded (h = 8): the 8 frames before
+ *                 the shard, the shard's F_loc frames, the 8 frames after it.
+ *                 Rows past a video end are masked out but are read: they must
+ *                 hold finite values (zeros).
  * k_glob, v_glob: [P][n_global][C]: the video's global frames
  *                 j * floor(F / n_global), j < n_global (unused if n_global == 0).
+ * part         : VI_PART_*; a block is 8 clips (128 frames), the boundary
+ *                 blocks are the first and the last.
  * Result       : exactly vi_dual_attn of the whole video, restricted to the
- *                 shard's frames.
+ *                 shard's frames (the part's blocks of them).
  * Requirements : L == 16, d == 64, n_pre, n_post <= 8, n_global <= 16
  *                 (VI_ERR_UNSUPPORTED otherwise); 0 <= clip0 <= N - N_loc;
- *                 out must not overlap any input; P == 0 is an empty call.
+ *                 part in 0..2; out must not overlap any input; P == 0 is an
+ *                 empty call.
  */
 int vi_dual_attn_shard(const void* q, const void* k_ext, const void* v_ext, const void* k_glob,
                        const void* v_glob, void* out, int F_loc, int N_loc, int clip0, int N,
-                       int P, int heads, int d, int n_pre, int n_post, int n_global,
+                       int P, int heads, int d, int n_pre, int n_post, int n_global, int part,
                        vi_stream_t stream);
 
 /*
  * Temporal conv of one shard (conv-module paragraph: each clip padded with
  * the neighbours' boundary frames).
  *
- * x_ext : [P][F_loc + 2*(k/2)][C]: k/2 frames before the shard (zeros at the
- *         start of the video), the shard's frames, k/2 frames after it (zeros
- *         at the end).   y : [P][F_loc][C].   w : [C][C][k];  b : [C].
- * Result       : vi_temporal_conv of the whole video on the shard's frames.
+ * x_ext : [P][F_loc + 2*(k/2)][C], halo-padded (h = k/2): k/2 frames before
+ *         the shard (zeros at the start of the video), the shard's frames,
+ *         k/2 frames after it (zeros at the end).   y : [P][F_loc][C].
+ *         w : [C][C][k];  b : [C].
+ * part  : VI_PART_*; a block is 128 frames; the interior blocks are those
+ *         whose frames and k/2 neighbours on each side lie in the shard.
+ * Result       : vi_temporal_conv of the whole video on the shard's frames
+ *                (the part's blocks of them).
  * Requirements : k odd; the tensor-core path (C % 64 == 0), else
- *                VI_ERR_UNSUPPORTED; y must not overlap x_ext, w or b.
+ *                VI_ERR_UNSUPPORTED; part in 0..2; y must not overlap x_ext,
+ *                w or b.
  */
 int vi_temporal_conv_shard(const void* x_ext, const void* w, const void* b, void* y, int F_loc,
-                           int P, int C, int k, vi_stream_t stream);
+                           int P, int C, int k, int part, vi_stream_t stream);
 
 /*
  * GroupNorm across shards (GroupNorm-module paragraph): every shard reduces

@@ -220,9 +220,9 @@ def test_binding_checks_shapes_before_the_call():
 
 
 def attn_shard(L, q=A, ke=B, ve=Cp, kg=D, vg=E, o=G, F_loc=64, N_loc=4, clip0=4, N=16, P=2,
-               heads=2, d=64, pre=8, post=8, glob=16):
+               heads=2, d=64, pre=8, post=8, glob=16, part=0):
     return L.vi_dual_attn_shard(q, ke, ve, kg, vg, o, F_loc, N_loc, clip0, N, P, heads, d, pre,
-                                post, glob, None)
+                                post, glob, part, None)
 
 
 @pytest.mark.parametrize("kw,expect", [
@@ -231,6 +231,8 @@ def attn_shard(L, q=A, ke=B, ve=Cp, kg=D, vg=E, o=G, F_loc=64, N_loc=4, clip0=4,
     (dict(glob=17), UNSUP), (dict(F_loc=128), UNSUP), (dict(d=32), UNSUP), (dict(P=-1), INVALID),
     (dict(q=A + 8), ALIGN), (dict(o=A), INVALID), (dict(q=None), INVALID),
     (dict(P=0, q=None, ke=None, ve=None, kg=None, vg=None, o=None), OK),
+    (dict(part=3), INVALID), (dict(part=-1), INVALID),
+    (dict(P=0, q=None, ke=None, ve=None, kg=None, vg=None, o=None, part=1), OK),
 ])
 def test_attention_shard_rejects(L, kw, expect):
     assert attn_shard(L, **kw) == expect
@@ -239,12 +241,13 @@ def test_attention_shard_rejects(L, kw, expect):
 @pytest.mark.parametrize("kw,expect", [
     (dict(k=2), INVALID), (dict(F_loc=0), INVALID), (dict(C=40), UNSUP), (dict(x=A + 8), ALIGN),
     (dict(y=A), INVALID), (dict(P=0, x=None, w=None, b=None, y=None), OK),
+    (dict(part=3), INVALID), (dict(P=0, x=None, w=None, b=None, y=None, part=2), OK),
 ])
 def test_conv_shard_rejects(L, kw, expect):
-    a = dict(x=A, w=B, b=Cp, y=D, F_loc=64, P=2, C=64, k=3)
+    a = dict(x=A, w=B, b=Cp, y=D, F_loc=64, P=2, C=64, k=3, part=0)
     a.update(kw)
     assert L.vi_temporal_conv_shard(a["x"], a["w"], a["b"], a["y"], a["F_loc"], a["P"], a["C"],
-                                    a["k"], None) == expect
+                                    a["k"], a["part"], None) == expect
 
 
 def test_groupnorm_shard_rejects(L):

@@ -122,3 +122,17 @@ def test_clock_anomaly_rules():
     assert "no reason" in bench.clock_anomaly({**ok, "sm_mhz": 1597})
     assert "hw_slowdown" in bench.clock_anomaly({**ok, "reasons": ["hw_slowdown"]})
     assert bench.clock_anomaly({**ok, "sm_mhz": None, "reasons": ["unsampled"]}) is None
+
+
+def test_tensor_peak_follows_the_timed_region():
+    """Burst figure for a short region at full clock; the sustained figure only
+    for a region of seconds whose SM clock sat well below the maximum."""
+    peaks = {"bf16_tflops": 1610.6, "bf16_tflops_sustained": 1373.6, "hbm_gbs": 6537.3}
+    full = {"sm_mhz": 1965, "sm_max_mhz": 1965, "reasons": []}
+    capped = {"sm_mhz": 1300, "sm_max_mhz": 1965, "reasons": ["sw_power_cap"]}
+    assert bench.choose_tensor_peak(peaks, 0.065, full) == (1610.6, "bf16_tflops")
+    assert bench.choose_tensor_peak(peaks, 0.065, capped) == (1610.6, "bf16_tflops")
+    assert bench.choose_tensor_peak(peaks, 5.0, full) == (1610.6, "bf16_tflops")
+    assert bench.choose_tensor_peak(peaks, 5.0, capped) == (1373.6, "bf16_tflops_sustained")
+    assert bench.choose_tensor_peak(peaks, 5.0, {"sm_mhz": None, "sm_max_mhz": None}) == \
+        (1610.6, "bf16_tflops")
