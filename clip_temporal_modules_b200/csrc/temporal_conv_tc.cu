@@ -64,8 +64,7 @@ constexpr int TC_SA_MAX = 6;     // A (x) stages at most
 constexpr int TC_SB_MAX = 8;     // B (w) stages at most
 constexpr int TC_NJ_MAX = 160;   // a B stage holds all k taps of one K-block
 constexpr int TC_EPI_WARPS = 4;          // one per TMEM lane quadrant
-constexpr int TC_THREADS = 64 + 32 * TC_EPI_WARPS;   // + transform threads with NORM
-constexpr int TC_XF_WARPS = 8;           // NORM: warps normalising the landed x stages
+constexpr int TC_THREADS = 64 + 32 * TC_EPI_WARPS;
 constexpr int TC_OUT_BUF = 32 * 128;     // one staging buffer: 32 frames x 64 channels of bf16
 constexpr int TC_TMEM_COLS = 512;
 constexpr int TC_SMEM_LIMIT = 232448;    // 227 KB opt-in per CTA
@@ -95,13 +94,15 @@ struct TcPlan {
   int b_stage;           // bytes per B stage = KS * b_kb
   int sa;                // A stages
   int sb;                // B stages
+  int hT;                // bias tables by distance to the video ends, up to hT frames:
+  int n_tab;             // (hT + 1)^2 tables of Cout floats (1 table when hT == 0)
   int wide;              // 1: the epilogue stores 64-channel chunks (else 32)
   int smem;              // dynamic shared memory bytes
 };
 
 struct TcArgs {
-  const float* coef;     // NORM: per-channel (m_c, a_c, beta_c, 0) of the GroupNorm
-  const bf16* bias;      // [Cout]
+  const float* btab;     // fp32 bias tables [n_tab][Cout] (GroupNorm-folded conv), or null
+  const bf16* bias;      // [Cout] (used when btab is null)
   const bf16* wpk;       // packed weights
   unsigned int* err;
   int x_off;             // row of output frame 0 in the x map (k/2 for a shard with halos)
@@ -118,23 +119,25 @@ struct TcMaps {
 // Ring depths.  Two tiles per job: equal x and w rings (one barrier pair per
 // stage), as deep as fit, at most 4.  One tile per job (measured on B200 at
 // F = 1024): with C <= 640 three x stages and two weight stages beat two and
-// three; at C = 1280 two x stages and as many weight stages as fit; with the
-// GroupNorm transform, three x stages.  The epilogue stages 64-channel
+// three; at C = 1280 two x stages and as many weight stages as fit.  The
+// epilogue stages 64-channel
 // chunks (two 4 KB buffers per warp) where that still leaves the widest slab
 // room, else 32-channel chunks (two 2 KB buffers per warp).
-static bool tc_plan(int F, int P, int C, int Cout, int n_out, int k, TcPlan& pl, bool norm,
+static bool tc_plan(int F, int P, int C, int Cout, int n_out, int k, TcPlan& pl, int hT,
                     int mt, int ks) {
   if (k < 1 || k % 2 == 0 || 127 + k > 256 || C % TC_KB != 0) return false;
   if (n_out < 1 || n_out > TC_MAX_OUT || Cout <= 0 || Cout % n_out != 0) return false;
   if (mt != 1 && mt != 2) return false;
-  if (ks != 1 && (ks != 2 || norm)) return false;
+  if (ks != 1 && ks != 2) return false;
+  if (hT < 0 || hT > k / 2) return false;
+  const int n_tab = (hT + 1) * (hT + 1);
   const int cpo = Cout / n_out;
   const int n_acc = mt + 1 > 2 ? mt + 1 : 2;
   const int a_rows = 127 + k;
   const int a_tile = ((a_rows * 128 + 1023) / 1024) * 1024;
   const int a_stage = ks * mt * a_tile;
-  const int base = 1024 /* align slack */ + ((4 * Cout + 63) / 64) * 64 /* bias */ +
-                   512 /* bars */ + (norm ? 16 * C : 0) /* GroupNorm coefficients */;
+  const int base = 1024 /* align slack */ + ((4 * n_tab * Cout + 63) / 64) * 64 /* bias */ +
+                   512 /* bars */;
   // Widest slab (<= 160 output channels, a multiple of 32 dividing each
   // output tensor's channels) whose all-tap weight stages leave room for at
   // least two of each ring.
@@ -150,7 +153,7 @@ static bool tc_plan(int F, int P, int C, int Cout, int n_out, int k, TcPlan& pl,
         if (n < 2) continue;
         sa = sb = n;
       } else {
-        const bool few_k = C <= 640 || norm;
+        const bool few_k = C <= 640;
         sa = few_k ? 3 : 2;
         sb = few_k ? 2 : TC_SB_MAX;
         const int sb_fit = (TC_SMEM_LIMIT - fixed - sa * a_stage) / b_stage;
@@ -185,6 +188,8 @@ static bool tc_plan(int F, int P, int C, int Cout, int n_out, int k, TcPlan& pl,
       pl.b_stage = b_stage;
       pl.sa = sa;
       pl.sb = sb;
+      pl.hT = hT;
+      pl.n_tab = n_tab;
       pl.wide = wide;
       pl.smem = fixed + sa * a_stage + sb * b_stage;
       if (pl.smem <= TC_SMEM_LIMIT) return true;
@@ -262,8 +267,8 @@ __device__ __forceinline__ void epi_stage_chunk(uint32_t stage, int lane, const 
   }
 }
 
-template <int KT, int MT, int KS, bool NORM>
-__global__ void __launch_bounds__(TC_THREADS + (NORM ? 32 * TC_XF_WARPS : 0), 1)
+template <int KT, int MT, int KS>
+__global__ void __launch_bounds__(TC_THREADS, 1)
     temporal_conv_tc_kernel(const __grid_constant__ TcMaps maps, const TcPlan pl,
                             const TcArgs args) {
   extern __shared__ uint8_t smem_raw[];
@@ -273,14 +278,12 @@ __global__ void __launch_bounds__(TC_THREADS + (NORM ? 32 * TC_XF_WARPS : 0), 1)
   const uint32_t sOut = sB + pl.sb * pl.b_stage;       // output staging, 1024-aligned
   const uint32_t out_buf = pl.wide ? TC_OUT_BUF : TC_OUT_BUF / 2;   // bytes of one staging buffer
   const uint32_t sBias = sOut + 4 * 2 * out_buf;
-  const uint32_t sBar = sBias + ((4 * pl.Cout + 63) / 64) * 64;
+  const uint32_t sBar = sBias + ((4 * pl.n_tab * pl.Cout + 63) / 64) * 64;
   // barrier block: a_full[SA] a_empty[SA] b_full[SB] b_empty[SB] acc_full[4] acc_empty[4] drain tmem_slot
   const uint32_t a_full = sBar, a_empty = a_full + 8 * TC_SA_MAX;
   const uint32_t b_full = a_empty + 8 * TC_SA_MAX, b_empty = b_full + 8 * TC_SB_MAX;
   const uint32_t acc_full = b_empty + 8 * TC_SB_MAX, acc_empty = acc_full + 32;
   const uint32_t drain = acc_empty + 32, tmem_slot = drain + 8;
-  const uint32_t a_ready = tmem_slot + 8;      // NORM: x stage normalised [SA]
-  const uint32_t sCoef = sBar + 512;           // NORM: float4 per channel
   float* bias_s = reinterpret_cast<float*>(smem_raw + (sBias - smem_u32(smem_raw)));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -294,19 +297,12 @@ __global__ void __launch_bounds__(TC_THREADS + (NORM ? 32 * TC_XF_WARPS : 0), 1)
       mbar_init(acc_empty + 8 * i, TC_EPI_WARPS);
     }
     mbar_init(drain, 1);
-    if (NORM)
-      for (int i = 0; i < pl.sa; ++i) mbar_init(a_ready + 8 * i, TC_XF_WARPS);
     fence_barrier_init();
   }
-  for (int c = threadIdx.x; c < pl.Cout; c += blockDim.x) bias_s[c] = to_f32(args.bias[c]);
-  if constexpr (NORM) {
-    float4* coef_s = reinterpret_cast<float4*>(smem_raw + (sCoef - smem_u32(smem_raw)));
-    // Channel cb*64 + 8c + e sits at slot cb*64 + 8e + c: the transform threads
-    // of one quarter-warp, which hold the 8 different c of a K-block, then
-    // read 8 consecutive slots (no bank conflict).
-    for (int ch = threadIdx.x; ch < pl.C; ch += blockDim.x)
-      coef_s[(ch & ~63) + (ch & 7) * 8 + ((ch >> 3) & 7)] =
-          reinterpret_cast<const float4*>(args.coef)[ch];
+  if (args.btab) {
+    for (int c = threadIdx.x; c < pl.n_tab * pl.Cout; c += blockDim.x) bias_s[c] = args.btab[c];
+  } else {
+    for (int c = threadIdx.x; c < pl.Cout; c += blockDim.x) bias_s[c] = to_f32(args.bias[c]);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, TC_TMEM_COLS);
@@ -415,8 +411,7 @@ __global__ void __launch_bounds__(TC_THREADS + (NORM ? 32 * TC_XF_WARPS : 0), 1)
         for (int is = 0; is < pl.n_stage && ok; ++is) {
           const int nkb = min(KS, pl.n_cb - is * KS);
           const bool last_stage = is == pl.n_stage - 1;
-          if (!mbar_wait_bounded((NORM ? a_ready : a_full) + 8 * sa, (uint32_t)pa, args.err,
-                                 VI_DEV_ERR_TMA_TIMEOUT) ||
+          if (!mbar_wait_bounded(a_full + 8 * sa, (uint32_t)pa, args.err, VI_DEV_ERR_TMA_TIMEOUT) ||
               (!uni &&
                !mbar_wait_bounded(b_full + 8 * sbi, (uint32_t)pb, args.err, VI_DEV_ERR_TMA_TIMEOUT))) {
             ok = false;
@@ -454,64 +449,6 @@ __global__ void __launch_bounds__(TC_THREADS + (NORM ? 32 * TC_XF_WARPS : 0), 1)
       umma_commit(drain);
       mbar_wait_bounded(drain, 0, args.err, VI_DEV_ERR_MMA_TIMEOUT);
     }
-  } else if (warp >= 2 + TC_EPI_WARPS) {
-    // ------------------------------------------------------------ transform (NORM)
-    // Normalise each landed x stage in place, x -> (x - m_c) a_c + beta_c,
-    // then hand it to the MMA.  Rows outside [0, F) stay zero: the conv pads
-    // the normalised sequence with zeros.  128B swizzle: the 16-byte chunk of
-    // channels [8c, 8c+8) of row r sits at chunk c ^ (r mod 8).
-    if constexpr (NORM) {
-      const float4* coef_s = reinterpret_cast<const float4*>(smem_raw + (sCoef - smem_u32(smem_raw)));
-      uint4* stage0 = reinterpret_cast<uint4*>(smem_raw + (sA - smem_u32(smem_raw)));
-      // Thread tt always handles physical chunk pc of rows r0, r0 + 4 TC_XF_WARPS,
-      // ...; all those rows share r mod 8, so the logical chunk (its 8
-      // channels) is fixed.
-      const int tt = threadIdx.x - TC_THREADS;
-      const int pc = tt & 7, r0 = tt >> 3;
-      const int c = pc ^ (r0 & 7);
-      int sa = 0, pa = 0;
-      bool ok = true;
-      for (long long job = blockIdx.x; job < pl.n_jobs && ok; job += gridDim.x) {
-        const long long tile0 = (job / pl.n_slabs) * MT;
-        int f_first[MT];                           // frame of row 0 of each tile's x box
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-          int fb, p;
-          tc_tile_pos(pl, tile0 + mt, fb, p);
-          f_first[mt] = fb * TC_M - halo;
-        }
-        for (int ib = 0; ib < pl.n_cb && ok; ++ib) {
-          const int cb = (ib + cb_rot) % pl.n_cb;
-          float m[8], a[8], bt[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float4 k4 = coef_s[cb * TC_KB + e * 8 + c];
-            m[e] = k4.x; a[e] = k4.y; bt[e] = k4.z;
-          }
-          if (!mbar_wait_bounded(a_full + 8 * sa, (uint32_t)pa, args.err, VI_DEV_ERR_TMA_TIMEOUT)) {
-            ok = false;
-            break;
-          }
-#pragma unroll
-          for (int mt = 0; mt < MT; ++mt) {
-            uint4* st = stage0 + (size_t)sa * (pl.a_stage / 16) + (size_t)mt * (pl.a_tile / 16);
-            for (int r = r0; r < pl.a_rows; r += 4 * TC_XF_WARPS) {
-              const int f = f_first[mt] + r;
-              if (f < 0 || f >= pl.F) continue;
-              float v[8];
-              unpack(st[r * 8 + pc], v);
-#pragma unroll
-              for (int e = 0; e < 8; ++e) v[e] = fmaf(v[e] - m[e], a[e], bt[e]);
-              st[r * 8 + pc] = pack(v);
-            }
-          }
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(a_ready + 8 * sa);
-          if (++sa == pl.sa) { sa = 0; pa ^= 1; }
-        }
-      }
-    }
   } else {
     // ------------------------------------------------------------ epilogue
     // Warp q owns TMEM lanes 32q .. 32q+31 (frames 32q .. of the tile) and
@@ -521,7 +458,6 @@ __global__ void __launch_bounds__(TC_THREADS + (NORM ? 32 * TC_XF_WARPS : 0), 1)
     // last chunk of a slab of 32 mod 64 channels), else 32.
     const int q = warp & 3;
     const uint32_t my_out = sOut + (uint32_t)q * 2u * out_buf;   // two staging buffers
-    const int cw = pl.wide ? 64 : 32;
     int ob = 0;                                  // staging buffer of the next chunk
     int buf = 0, pacc = 0;                       // accumulator ring, as the MMA issuer walks it
     bool ok = true;
@@ -529,7 +465,6 @@ __global__ void __launch_bounds__(TC_THREADS + (NORM ? 32 * TC_XF_WARPS : 0), 1)
       const int slab = (int)(job % pl.n_slabs);
       const int out = slab / pl.slabs_per_out;                 // output tensor of this slab
       const int ch0 = (slab - out * pl.slabs_per_out) * pl.NJ; // its first channel there
-      const float* bs = bias_s + slab * pl.NJ;
       for (int mt = 0; mt < MT; ++mt) {
         // The lanes take the (bounded) wait's outcome together.
         const bool got = __all_sync(0xffffffffu, mbar_wait_bounded(acc_full + 8 * buf, (uint32_t)pacc,
@@ -543,70 +478,49 @@ __global__ void __launch_bounds__(TC_THREADS + (NORM ? 32 * TC_XF_WARPS : 0), 1)
         int fb, p;
         tc_tile_pos(pl, tile, fb, p);
         const bool tile_ok = tile < pl.n_tiles;
+        // This row's bias table: by its distance to each video end, capped at
+        // hT (one table, the plain bias, when hT == 0).
+        const int f = fb * TC_M + 32 * q + lane;
+        const int lo = min(f, pl.hT), hi = max(min(pl.F - 1 - f, pl.hT), 0);
+        const float* bs = bias_s + (lo * (pl.hT + 1) + hi) * pl.Cout + slab * pl.NJ;
         const uint32_t taddr = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * pl.NJ);
-        if constexpr (!NORM) {
-          // The whole row of the tile (<= 160 columns) into registers first,
-          // so that the accumulator goes back to the MMA at once and the
-          // packing and stores overlap the next tiles' MMAs.
-          uint32_t r[TC_NJ_MAX / 32][32];
+        // The whole row of the tile (<= 160 columns) into registers first,
+        // so that the accumulator goes back to the MMA at once and the
+        // packing and stores overlap the next tiles' MMAs.
+        uint32_t r[TC_NJ_MAX / 32][32];
 #pragma unroll
-          for (int c = 0; c < TC_NJ_MAX / 32; ++c)
-            if (32 * c < pl.NJ) tmem_ld32(taddr + 32u * c, r[c]);
+        for (int c = 0; c < TC_NJ_MAX / 32; ++c)
+          if (32 * c < pl.NJ) tmem_ld32(taddr + 32u * c, r[c]);
 #pragma unroll
-          for (int c = 0; c < TC_NJ_MAX / 32; ++c)
-            if (32 * c < pl.NJ) tmem_wait_ld_dep(r[c]);
-          tc_fence_before();
+        for (int c = 0; c < TC_NJ_MAX / 32; ++c)
+          if (32 * c < pl.NJ) tmem_wait_ld_dep(r[c]);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(acc_empty + 8 * buf);
+        // Chunks: 64 channels (groups g, g+1) where the plan is wide and
+        // they fit, else 32 (group g).  Loops unrolled: registers indexed
+        // at compile time only.
+        bool taken = false;                   // group g went out with group g-1
+#pragma unroll
+        for (int g = 0; g < TC_NJ_MAX / 32; ++g) {
+          if (32 * g >= pl.NJ) break;
+          if (taken) { taken = false; continue; }
+          const bool w64 = g + 1 < TC_NJ_MAX / 32 && pl.wide && 32 * g + 64 <= pl.NJ;
+          const uint32_t stage = my_out + (uint32_t)ob * out_buf;
+          if (lane == 0) bulk_wait_read_le1();   // the store that last read this buffer is done
           __syncwarp();
-          if (lane == 0) mbar_arrive(acc_empty + 8 * buf);
-          // Chunks: 64 channels (groups g, g+1) where the plan is wide and
-          // they fit, else 32 (group g).  Loops unrolled: registers indexed
-          // at compile time only.
-          bool taken = false;                   // group g went out with group g-1
-#pragma unroll
-          for (int g = 0; g < TC_NJ_MAX / 32; ++g) {
-            if (32 * g >= pl.NJ) break;
-            if (taken) { taken = false; continue; }
-            const bool w64 = g + 1 < TC_NJ_MAX / 32 && pl.wide && 32 * g + 64 <= pl.NJ;
-            const uint32_t stage = my_out + (uint32_t)ob * out_buf;
-            if (lane == 0) bulk_wait_read_le1();   // the store that last read this buffer is done
-            __syncwarp();
-            if (tile_ok)
-              epi_stage_chunk(stage, lane, r[g], r[g + 1 < TC_NJ_MAX / 32 ? g + 1 : g], bs + 32 * g, w64);
-            fence_proxy_async_smem();           // the writes are visible to the TMA store
-            __syncwarp();
-            if (lane == 0 && tile_ok) {
-              // Rows past the last frame fall outside the tensor map and are dropped.
-              tma_store_3d(w64 ? &maps.y[out] : &maps.y32[out], stage, ch0 + 32 * g,
-                           fb * TC_M + 32 * q, p);
-              bulk_commit();
-            }
-            ob ^= 1;
-            taken = w64;
-          }
-        } else {
-          for (int c0 = 0; c0 < pl.NJ; c0 += cw) {
-            const bool w64 = cw == 64 && c0 + 64 <= pl.NJ;     // this chunk: 64 channels (else 32)
-            uint32_t r0[32], r1[32];
-            tmem_ld32(taddr + (uint32_t)c0, r0);
-            if (w64) tmem_ld32(taddr + (uint32_t)c0 + 32u, r1);
-            tmem_wait_ld_dep(r0);
-            if (w64) tmem_wait_ld_dep(r1);
-            const uint32_t stage = my_out + (uint32_t)ob * out_buf;
-            if (lane == 0) bulk_wait_read_le1();   // the store that last read this buffer is done
-            __syncwarp();
-            if (tile_ok) epi_stage_chunk(stage, lane, r0, r1, bs + c0, w64);
-            fence_proxy_async_smem();           // the writes are visible to the TMA store
-            __syncwarp();
-            if (lane == 0 && tile_ok) {
-              tma_store_3d(w64 ? &maps.y[out] : &maps.y32[out], stage, ch0 + c0, fb * TC_M + 32 * q, p);
-              bulk_commit();
-            }
-            ob ^= 1;
-            if (!w64 && cw == 64) break;        // the 32-channel tail was the slab's last chunk
-          }
-          tc_fence_before();
+          if (tile_ok)
+            epi_stage_chunk(stage, lane, r[g], r[g + 1 < TC_NJ_MAX / 32 ? g + 1 : g], bs + 32 * g, w64);
+          fence_proxy_async_smem();           // the writes are visible to the TMA store
           __syncwarp();
-          if (lane == 0) mbar_arrive(acc_empty + 8 * buf);
+          if (lane == 0 && tile_ok) {
+            // Rows past the last frame fall outside the tensor map and are dropped.
+            tma_store_3d(w64 ? &maps.y[out] : &maps.y32[out], stage, ch0 + 32 * g,
+                         fb * TC_M + 32 * q, p);
+            bulk_commit();
+          }
+          ob ^= 1;
+          taken = w64;
         }
         if (++buf == pl.n_acc) { buf = 0; pacc ^= 1; }
       }
@@ -623,9 +537,17 @@ __global__ void __launch_bounds__(TC_THREADS + (NORM ? 32 * TC_XF_WARPS : 0), 1)
 
 // w [C_out][C_in][k] -> [slab][cb][t][8 columns][NJ][8]: for each (slab,
 // K-block, tap) an NJ x 64 K-major block in the no-swizzle layout, the k tap
-// blocks of a (slab, K-block) contiguous.
-__global__ void temporal_conv_pack_w(const bf16* __restrict__ w, bf16* __restrict__ wpk, int C,
-                                     int Cout, int k, int NJ) {
+// blocks of a (slab, K-block) contiguous.  coef != null (GroupNorm folded
+// into the conv): each input channel's weights are scaled by its GroupNorm
+// factor a_ci first, W'[co][ci][t] = bf16(w[co][ci][t] * a_ci).
+__device__ __forceinline__ bf16 tc_folded_w(const bf16* w, const float* coef, int co, int ci,
+                                            int t, int C, int k) {
+  const bf16 v = w[((size_t)co * C + ci) * k + t];
+  return coef ? __float2bfloat16_rn(__bfloat162float(v) * coef[4 * ci + 1]) : v;
+}
+
+__global__ void temporal_conv_pack_w(const bf16* __restrict__ w, const float* __restrict__ coef,
+                                     bf16* __restrict__ wpk, int C, int Cout, int k, int NJ) {
   const long long total = (long long)Cout * C * k;
   const int n_cb = C / TC_KB;
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
@@ -637,8 +559,51 @@ __global__ void temporal_conv_pack_w(const bf16* __restrict__ w, bf16* __restric
     const int t = (int)(r % k); r /= k;
     const int cb = (int)(r % n_cb);
     const int slab = (int)(r / n_cb);
-    const int co = slab * NJ + n, ci = cb * TC_KB + col * 8 + e;
-    wpk[i] = w[((size_t)co * C + ci) * k + t];
+    wpk[i] = tc_folded_w(w, coef, slab * NJ + n, cb * TC_KB + col * 8 + e, t, C, k);
+  }
+}
+
+// Bias tables of the GroupNorm-folded conv.  With x_n = (x - m) a + beta on
+// the frames of the video and 0 outside, the conv of x_n is, per output
+// channel co and frame f,
+//   b[co] + sum_t sum_ci W[co,ci,t] x_n[f+t-h, ci]
+//     = acc + b[co] + sum_{t valid} sum_ci (W[co,ci,t] beta_ci - W'[co,ci,t] m_ci)
+// where acc = sum_t sum_ci W'[co,ci,t] x[f+t-h, ci] is what the tensor cores
+// compute from the raw x (zero outside the video) and W' = bf16(W a) are the
+// folded weights.  The mean term uses the same rounded W' as acc, so the
+// means cancel exactly and the rounding of W' only scales x - m.  A tap t is
+// valid when frame f+t-h lies in the video: with lo = min(f, h) frames
+// before f and hi = min(F-1-f, h) after it, t in [h - lo, h + hi].  One
+// block per output channel; table (lo, hi) at [(lo (h+1) + hi) Cout + co].
+__global__ void __launch_bounds__(128) temporal_conv_fold_bias(
+    const bf16* __restrict__ w, const bf16* __restrict__ b, const float* __restrict__ coef,
+    float* __restrict__ tab, int C, int Cout, int k) {
+  constexpr int MAXK = 8;
+  __shared__ double part[MAXK][4];
+  const int co = blockIdx.x, h = k / 2;
+  double acc[MAXK];
+  for (int t = 0; t < k; ++t) acc[t] = 0.0;
+  for (int ci = threadIdx.x; ci < C; ci += blockDim.x) {
+    const double m = coef[4 * ci], beta = coef[4 * ci + 2];
+    for (int t = 0; t < k; ++t) {
+      const double wv = __bfloat162float(w[((size_t)co * C + ci) * k + t]);
+      const double wf = __bfloat162float(tc_folded_w(w, coef, co, ci, t, C, k));
+      acc[t] += wv * beta - wf * m;
+    }
+  }
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int t = 0; t < k; ++t) {
+    double v = acc[t];
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (lane == 0) part[t][warp] = v;
+  }
+  __syncthreads();
+  if (threadIdx.x < (h + 1) * (h + 1)) {
+    const int lo = threadIdx.x / (h + 1), hi = threadIdx.x % (h + 1);
+    double sum = __bfloat162float(b[co]);
+    for (int t = h - lo; t <= h + hi; ++t)
+      sum += part[t][0] + part[t][1] + part[t][2] + part[t][3];
+    tab[(size_t)threadIdx.x * Cout + co] = (float)sum;
   }
 }
 
@@ -648,23 +613,26 @@ bool encode_tmap(CUtensorMap* map, const void* base, int rank, const uint64_t* d
 
 // Tiles per job of the default plan (2: every weight stage feeds two tiles).
 constexpr int TC_MT_DEFAULT = 2;
+// Largest tap count of the GroupNorm-folded conv (bias tables per distance to
+// the video ends: (k/2 + 1)^2 of them).
+constexpr int TC_FOLD_MAX_K = 7;
 
 bool temporal_conv_tc_ok(int F, int P, int C, int k) {
   TcPlan pl;
-  return F > 0 && P > 0 && tc_plan(F, P, C, C, 1, k, pl, false, 1, 1);
+  return F > 0 && P > 0 && tc_plan(F, P, C, C, 1, k, pl, 0, 1, 1);
 }
 
 bool temporal_conv_tc_norm_ok(int F, int P, int C, int k) {
   TcPlan pl;
-  return F > 0 && P > 0 && tc_plan(F, P, C, C, 1, k, pl, true, 1, 1);
+  return F > 0 && P > 0 && k <= TC_FOLD_MAX_K && tc_plan(F, P, C, C, 1, k, pl, k / 2, 1, 1);
 }
 
 bool linear_tc_ok(int F, int P, int C, int Cout, int n_out) {
   TcPlan pl;
-  return F > 0 && P > 0 && tc_plan(F, P, C, Cout, n_out, 1, pl, false, 1, 1);
+  return F > 0 && P > 0 && tc_plan(F, P, C, Cout, n_out, 1, pl, 0, 1, 1);
 }
 
-template <int KT, int MT, int KS, bool NORM>
+template <int KT, int MT, int KS>
 static int tc_launch(const TcMaps& maps, const TcPlan& pl, const TcArgs& a, cudaStream_t stream) {
   static std::mutex mu;
   static bool attr_done[64] = {false};
@@ -674,7 +642,7 @@ static int tc_launch(const TcMaps& maps, const TcPlan& pl, const TcArgs& a, cuda
     std::lock_guard<std::mutex> lock(mu);
     if (dev < 0 || dev >= 64) return VI_ERR_CUDA;
     if (!attr_done[dev]) {
-      VI_CUDA_TRY(cudaFuncSetAttribute(temporal_conv_tc_kernel<KT, MT, KS, NORM>,
+      VI_CUDA_TRY(cudaFuncSetAttribute(temporal_conv_tc_kernel<KT, MT, KS>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        TC_SMEM_LIMIT));
       attr_done[dev] = true;
@@ -682,56 +650,52 @@ static int tc_launch(const TcMaps& maps, const TcPlan& pl, const TcArgs& a, cuda
   }
   long long grid = sm_count();
   if (grid > pl.n_jobs) grid = pl.n_jobs;
-  temporal_conv_tc_kernel<KT, MT, KS, NORM>
-      <<<(unsigned)grid, TC_THREADS + (NORM ? 32 * TC_XF_WARPS : 0), (size_t)pl.smem, stream>>>(
-          maps, pl, a);
+  temporal_conv_tc_kernel<KT, MT, KS><<<(unsigned)grid, TC_THREADS, (size_t)pl.smem, stream>>>(
+      maps, pl, a);
   VI_LAUNCHED();
   return VI_OK;
 }
 
 // The kernel form of a plan: taps 3 and 1 are compiled with their loops
 // unrolled, any other odd k runs the tap loop at run time.
-static int tc_dispatch(const TcMaps& maps, const TcPlan& pl, const TcArgs& a, bool norm,
+static int tc_dispatch(const TcMaps& maps, const TcPlan& pl, const TcArgs& a,
                        cudaStream_t stream) {
   const int kt = pl.k == 3 ? 3 : pl.k == 1 ? 1 : 0;
-  if (norm) {
-    if (pl.MT == 2) return kt == 3 ? tc_launch<3, 2, 1, true>(maps, pl, a, stream)
-                                   : tc_launch<0, 2, 1, true>(maps, pl, a, stream);
-    return kt == 3 ? tc_launch<3, 1, 1, true>(maps, pl, a, stream)
-                   : tc_launch<0, 1, 1, true>(maps, pl, a, stream);
-  }
-  if (pl.KS == 2) return tc_launch<1, 2, 2, false>(maps, pl, a, stream);   // planned for k = 1, MT = 2
+  if (pl.KS == 2) return tc_launch<1, 2, 2>(maps, pl, a, stream);   // planned for k = 1, MT = 2
   switch (kt * 10 + pl.MT) {
-    case 32: return tc_launch<3, 2, 1, false>(maps, pl, a, stream);
-    case 31: return tc_launch<3, 1, 1, false>(maps, pl, a, stream);
-    case 12: return tc_launch<1, 2, 1, false>(maps, pl, a, stream);
-    case 11: return tc_launch<1, 1, 1, false>(maps, pl, a, stream);
-    case 2: return tc_launch<0, 2, 1, false>(maps, pl, a, stream);
-    default: return tc_launch<0, 1, 1, false>(maps, pl, a, stream);
+    case 32: return tc_launch<3, 2, 1>(maps, pl, a, stream);
+    case 31: return tc_launch<3, 1, 1>(maps, pl, a, stream);
+    case 12: return tc_launch<1, 2, 1>(maps, pl, a, stream);
+    case 11: return tc_launch<1, 1, 1>(maps, pl, a, stream);
+    case 2: return tc_launch<0, 2, 1>(maps, pl, a, stream);
+    default: return tc_launch<0, 1, 1>(maps, pl, a, stream);
   }
 }
 
 // One call: x [P][x_rows][C] (output frame f reads x row f + x_off + t - k/2),
 // w [Cout][C][k], b [Cout], outputs ys[0..n_out) each [P][F][Cout/n_out].
-// coef != nullptr: normalise x on the fly with the GroupNorm coefficients
-// (m_c, a_c, beta_c) before the contraction (fused GroupNorm -> conv).
+// coef != nullptr: the conv of the GroupNorm of x, with the GroupNorm's
+// per-channel coefficients (m_c, a_c, beta_c) folded into the weights and the
+// bias tables (fused GroupNorm -> conv; see temporal_conv_fold_bias).
 // mt: tiles per job, 0 = the default plan.
 static int tc_run(const bf16* x, int x_rows, int x_off, const bf16* w, const bf16* b,
                   bf16* const* ys, int n_out, int F, int P, int C, int Cout, int k,
                   cudaStream_t stream, const float* coef, int mt, int part = VI_PART_ALL) {
   TcPlan pl;
-  const bool norm = coef != nullptr;
+  const bool fold = coef != nullptr;
+  if (fold && k > TC_FOLD_MAX_K) return VI_ERR_UNSUPPORTED;
+  const int hT = fold ? k / 2 : 0;
   if (mt != 0) {
-    if (!tc_plan(F, P, C, Cout, n_out, k, pl, norm, mt, 1)) return VI_ERR_UNSUPPORTED;
+    if (!tc_plan(F, P, C, Cout, n_out, k, pl, hT, mt, 1)) return VI_ERR_UNSUPPORTED;
   } else {
-    if (!tc_plan(F, P, C, Cout, n_out, k, pl, norm, 1, 1)) return VI_ERR_UNSUPPORTED;
+    if (!tc_plan(F, P, C, Cout, n_out, k, pl, hT, 1, 1)) return VI_ERR_UNSUPPORTED;
     // Two tiles per job when that plan keeps the slab width (a narrower MMA
     // N costs more than the weight traffic it saves).
     TcPlan pl2;
-    if (tc_plan(F, P, C, Cout, n_out, k, pl2, norm, TC_MT_DEFAULT, 1) && pl2.NJ >= pl.NJ) pl = pl2;
+    if (tc_plan(F, P, C, Cout, n_out, k, pl2, hT, TC_MT_DEFAULT, 1) && pl2.NJ >= pl.NJ) pl = pl2;
     // Single tap: two K-blocks per stage where they fit at the same width, so
     // a stage still queues 16 MMAs per wait/commit.
-    if (k == 1 && pl.MT == 2 && !norm && tc_plan(F, P, C, Cout, n_out, k, pl2, false, 2, 2) &&
+    if (k == 1 && pl.MT == 2 && tc_plan(F, P, C, Cout, n_out, k, pl2, hT, 2, 2) &&
         pl2.NJ >= pl.NJ)
       pl = pl2;
   }
@@ -781,23 +745,30 @@ static int tc_run(const bf16* x, int x_rows, int x_off, const bf16* w, const bf1
                      CU_TENSOR_MAP_DATA_TYPE_BFLOAT16))
       return VI_ERR_CUDA;
   }
-  const size_t wbytes = (size_t)Cout * C * k * sizeof(bf16);
-  void* wpk = nullptr;
-  VI_CUDA_TRY(scratch_alloc(&wpk, wbytes, stream));
+  // Scratch: the packed weights, then (folded conv) the bias tables.
+  const size_t wbytes = (((size_t)Cout * C * k * sizeof(bf16)) + 255) / 256 * 256;
+  const size_t tbytes = fold ? (size_t)pl.n_tab * Cout * sizeof(float) : 0;
+  void* scratch = nullptr;
+  VI_CUDA_TRY(scratch_alloc(&scratch, wbytes + tbytes, stream));
+  bf16* wpk = static_cast<bf16*>(scratch);
+  float* tab = fold ? reinterpret_cast<float*>(static_cast<char*>(scratch) + wbytes) : nullptr;
   int st = VI_OK;
   {
     const long long total = (long long)Cout * C * k;
     int blocks = (int)((total + 255) / 256);
     if (blocks > 4 * sm_count()) blocks = 4 * sm_count();
-    temporal_conv_pack_w<<<blocks, 256, 0, stream>>>(w, static_cast<bf16*>(wpk), C, Cout, k,
-                                                     pl.NJ);
+    temporal_conv_pack_w<<<blocks, 256, 0, stream>>>(w, coef, wpk, C, Cout, k, pl.NJ);
+    if (cudaGetLastError() != cudaSuccess) st = VI_ERR_CUDA; else note_launch();
+  }
+  if (st == VI_OK && fold) {
+    temporal_conv_fold_bias<<<Cout, 128, 0, stream>>>(w, b, coef, tab, C, Cout, k);
     if (cudaGetLastError() != cudaSuccess) st = VI_ERR_CUDA; else note_launch();
   }
   if (st == VI_OK) {
-    const TcArgs a{coef, b, static_cast<const bf16*>(wpk), err, x_off};
-    st = tc_dispatch(maps, pl, a, norm, stream);
+    const TcArgs a{tab, b, wpk, err, x_off};
+    st = tc_dispatch(maps, pl, a, stream);
   }
-  if (scratch_free(wpk, stream) != cudaSuccess && st == VI_OK) st = VI_ERR_CUDA;
+  if (scratch_free(scratch, stream) != cudaSuccess && st == VI_OK) st = VI_ERR_CUDA;
   return st;
 }
 

@@ -197,17 +197,24 @@ int vi_temporal_attention(const void* x, const void* w_qkv, const void* b_qkv, c
  * GroupNorm with global statistics followed by the temporal convolution,
  * fused (bf16).  The ResNet module of the write-up normalises and then
  * convolves along frames (GroupNorm-module and conv-module paragraphs);
- *   y = vi_temporal_conv(vi_groupnorm_global(x; gamma, beta, groups, eps); w, b)
+ *   y = conv(GroupNorm(x; gamma, beta, groups, eps); w, b)
  * computed without writing the normalised tensor to memory: one statistics
- * pass over x, then the conv kernel normalises each staged x tile in shared
- * memory (bf16, round to nearest even) before the tensor-core contraction.
- * The zero padding at the video ends applies to the NORMALISED sequence.
+ * pass over x gives per-channel (m_c, a_c = gamma_c / sigma_g, beta_c); the
+ * tensor-core conv then runs on the raw x with the weights scaled per input
+ * channel, W'[co][ci][t] = bf16(w[co][ci][t] a_ci), and per-output-channel
+ * bias tables b[co] + sum over the taps inside the video of
+ * sum_ci (w beta_ci - W' m_ci), computed in fp64 from the same rounded W' (so
+ * the mean terms cancel exactly).  The zero padding at the video ends applies
+ * to the NORMALISED sequence: frames within k/2 of an end take the table of
+ * their valid taps.  The result differs from the two bf16 calls composed by
+ * bf16 rounding (of W a instead of the normalised tensor).
  *
  * x, y : [P][F][C];  gamma, beta, b : [C];  w : [C][C][k].
  * Requirements : those of vi_groupnorm_global and vi_temporal_conv; y must
  *                not overlap any input; the fused kernel also needs
- *                C % 64 == 0 (VI_ERR_UNSUPPORTED otherwise).
- * Scratch      : GroupNorm statistics and repacked w (library pool).
+ *                C % 64 == 0 and k <= 7 (VI_ERR_UNSUPPORTED otherwise).
+ * Scratch      : GroupNorm statistics, folded w and the bias tables (library
+ *                pool).
  */
 int vi_groupnorm_conv(const void* x, const void* gamma, const void* beta, const void* w,
                       const void* b, void* y, int F, int N, int P, int C, int groups, float eps,
