@@ -75,8 +75,7 @@ struct TcPlan {
   int Cout;              // output channels (all output tensors together)
   int NJ;                // output channels per job (UMMA N), multiple of 32
   int MT;                // tiles per job (1, or 2 sharing every weight stage)
-  int KS;                // K-blocks per pipeline stage (1, or 2 for single-tap convs)
-  int n_stage;           // stages per job = ceil(n_cb / KS)
+  int n_stage;           // stages per job = n_cb (a stage is one K-block)
   int n_acc;             // TMEM accumulators in the ring (MT + 1, at least 2), NJ columns each
   int n_slabs;           // Cout / NJ
   int slabs_per_out;     // slabs of one output tensor
@@ -88,10 +87,10 @@ struct TcPlan {
   int n_cb;              // C / 64
   int a_rows;            // 127 + k
   int a_tile;            // bytes of one tile's x box (a_rows x 128 B), 1024-aligned
-  int a_stage;           // bytes per A stage = KS * MT * a_tile
+  int a_stage;           // bytes per A stage = MT * a_tile
   int b_tap;             // bytes of one tap's block = NJ * 128
   int b_kb;              // weight bytes of one K-block = k * b_tap (all taps)
-  int b_stage;           // bytes per B stage = KS * b_kb
+  int b_stage;           // bytes per B stage = b_kb
   int sa;                // A stages
   int sb;                // B stages
   int hT;                // bias tables by distance to the video ends, up to hT frames:
@@ -101,8 +100,8 @@ struct TcPlan {
 };
 
 struct TcArgs {
-  const float* btab;     // fp32 bias tables [n_tab][Cout] (GroupNorm-folded conv), or null
-  const bf16* bias;      // [Cout] (used when btab is null)
+  const float* btab;     // fp32 bias tables [n_tab][Cout] in global memory (one table,
+                         // the conv's bias, unless the GroupNorm is folded in)
   const bf16* wpk;       // packed weights
   unsigned int* err;
   int x_off;             // row of output frame 0 in the x map (k/2 for a shard with halos)
@@ -124,26 +123,24 @@ struct TcMaps {
 // chunks (two 4 KB buffers per warp) where that still leaves the widest slab
 // room, else 32-channel chunks (two 2 KB buffers per warp).
 static bool tc_plan(int F, int P, int C, int Cout, int n_out, int k, TcPlan& pl, int hT,
-                    int mt, int ks) {
+                    int mt) {
   if (k < 1 || k % 2 == 0 || 127 + k > 256 || C % TC_KB != 0) return false;
   if (n_out < 1 || n_out > TC_MAX_OUT || Cout <= 0 || Cout % n_out != 0) return false;
   if (mt != 1 && mt != 2) return false;
-  if (ks != 1 && ks != 2) return false;
   if (hT < 0 || hT > k / 2) return false;
   const int n_tab = (hT + 1) * (hT + 1);
   const int cpo = Cout / n_out;
   const int n_acc = mt + 1 > 2 ? mt + 1 : 2;
   const int a_rows = 127 + k;
   const int a_tile = ((a_rows * 128 + 1023) / 1024) * 1024;
-  const int a_stage = ks * mt * a_tile;
-  const int base = 1024 /* align slack */ + ((4 * n_tab * Cout + 63) / 64) * 64 /* bias */ +
-                   512 /* bars */;
+  const int a_stage = mt * a_tile;
+  const int base = 1024 /* align slack */ + 512 /* bars */;
   // Widest slab (<= 160 output channels, a multiple of 32 dividing each
   // output tensor's channels) whose all-tap weight stages leave room for at
   // least two of each ring.
   for (int nj = TC_NJ_MAX; nj >= 32; nj -= 32) {
     if (cpo % nj != 0 || n_acc * nj > TC_TMEM_COLS) continue;
-    const int b_stage = ks * k * nj * 128;
+    const int b_stage = k * nj * 128;
     for (int wide = 1; wide >= 0; --wide) {
       const int fixed = base + 4 * 2 * (wide ? TC_OUT_BUF : TC_OUT_BUF / 2);   // output staging
       int sa, sb;
@@ -169,7 +166,6 @@ static bool tc_plan(int F, int P, int C, int Cout, int n_out, int k, TcPlan& pl,
       pl.Cout = Cout;
       pl.NJ = nj;
       pl.MT = mt;
-      pl.KS = ks;
       pl.n_acc = n_acc;
       pl.n_slabs = Cout / nj;
       pl.slabs_per_out = cpo / nj;
@@ -179,7 +175,7 @@ static bool tc_plan(int F, int P, int C, int Cout, int n_out, int k, TcPlan& pl,
       pl.n_tiles = (long long)P * pl.n_fblk;
       pl.n_jobs = ((pl.n_tiles + mt - 1) / mt) * pl.n_slabs;
       pl.n_cb = C / TC_KB;
-      pl.n_stage = (pl.n_cb + ks - 1) / ks;
+      pl.n_stage = pl.n_cb;
       pl.a_rows = a_rows;
       pl.a_tile = a_tile;
       pl.a_stage = a_stage;
@@ -267,7 +263,7 @@ __device__ __forceinline__ void epi_stage_chunk(uint32_t stage, int lane, const 
   }
 }
 
-template <int KT, int MT, int KS>
+template <int KT, int MT>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     temporal_conv_tc_kernel(const __grid_constant__ TcMaps maps, const TcPlan pl,
                             const TcArgs args) {
@@ -277,14 +273,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   const uint32_t sB = sA + pl.sa * pl.a_stage;
   const uint32_t sOut = sB + pl.sb * pl.b_stage;       // output staging, 1024-aligned
   const uint32_t out_buf = pl.wide ? TC_OUT_BUF : TC_OUT_BUF / 2;   // bytes of one staging buffer
-  const uint32_t sBias = sOut + 4 * 2 * out_buf;
-  const uint32_t sBar = sBias + ((4 * pl.n_tab * pl.Cout + 63) / 64) * 64;
+  const uint32_t sBar = sOut + 4 * 2 * out_buf;
   // barrier block: a_full[SA] a_empty[SA] b_full[SB] b_empty[SB] acc_full[4] acc_empty[4] drain tmem_slot
   const uint32_t a_full = sBar, a_empty = a_full + 8 * TC_SA_MAX;
   const uint32_t b_full = a_empty + 8 * TC_SA_MAX, b_empty = b_full + 8 * TC_SB_MAX;
   const uint32_t acc_full = b_empty + 8 * TC_SB_MAX, acc_empty = acc_full + 32;
   const uint32_t drain = acc_empty + 32, tmem_slot = drain + 8;
-  float* bias_s = reinterpret_cast<float*>(smem_raw + (sBias - smem_u32(smem_raw)));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int k = KT > 0 ? KT : pl.k;
@@ -298,11 +292,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     }
     mbar_init(drain, 1);
     fence_barrier_init();
-  }
-  if (args.btab) {
-    for (int c = threadIdx.x; c < pl.n_tab * pl.Cout; c += blockDim.x) bias_s[c] = args.btab[c];
-  } else {
-    for (int c = threadIdx.x; c < pl.Cout; c += blockDim.x) bias_s[c] = to_f32(args.bias[c]);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, TC_TMEM_COLS);
@@ -322,9 +311,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     // Lane 0 takes the ring waits and posts the expected bytes; the stage's
-    // copies are then issued by different lanes (x box j by lane j, the
-    // weights of K-block kb by lane nkb*MT + kb): one thread issuing every
-    // copy would serialise them on its issue latency.
+    // copies are then issued by different lanes (x box of tile m by lane m,
+    // the weights by lane MT): one thread issuing every copy would serialise
+    // them on its issue latency.
     int sa = 0, pa = 0, sbi = 0, pb = 0;           // ring positions as (stage, phase) counters
     bool a_used = false, b_used = false;           // first pass over a ring needs no wait
     bool ok = true;
@@ -344,35 +333,29 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       // Packed weights of (slab, K-block 0): k contiguous tap blocks per K-block.
       const bf16* wslab = args.wpk + (size_t)slab * pl.n_cb * (pl.b_kb / 2);
       for (int is = 0; is < pl.n_stage; ++is) {
-        // Stage `is` holds K-blocks kb0 .. kb0 + nkb - 1 of the job (in the
-        // CTA's rotated order); only a job's last stage can hold fewer than KS.
-        const int kb0 = is * KS;
-        const int nkb = min(KS, pl.n_cb - kb0);
+        // Stage `is` holds K-block (is + cb_rot) mod n_cb of the job.
+        const int cb = (is + cb_rot) % pl.n_cb;
         const uint32_t a_bar = a_full + 8 * sa;
         const uint32_t b_bar = uni ? a_bar : b_full + 8 * sbi;   // shared stage: one barrier
         bool go = true;
         if (lane == 0) {
           go = !a_used || mbar_wait_bounded(a_empty + 8 * sa, (uint32_t)(pa ^ 1), args.err,
                                             VI_DEV_ERR_TMA_TIMEOUT);
-          if (go) mbar_arrive_expect_tx(a_bar, (uint32_t)nkb * (a_bytes + (uni ? (uint32_t)pl.b_kb : 0u)));
+          if (go) mbar_arrive_expect_tx(a_bar, a_bytes + (uni ? (uint32_t)pl.b_kb : 0u));
           if (go && !uni) {
             go = !b_used || mbar_wait_bounded(b_empty + 8 * sbi, (uint32_t)(pb ^ 1), args.err,
                                               VI_DEV_ERR_TMA_TIMEOUT);
-            if (go) mbar_arrive_expect_tx(b_bar, (uint32_t)(nkb * pl.b_kb));
+            if (go) mbar_arrive_expect_tx(b_bar, (uint32_t)pl.b_kb);
           }
         }
         if (!__shfl_sync(0xffffffffu, go ? 1 : 0, 0)) { ok = false; break; }
-        if (lane < nkb * MT) {
-          const int kb = lane / MT, m = lane - kb * MT;
-          const int cb = (kb0 + kb + cb_rot) % pl.n_cb;
+        if (lane < MT) {
           // (a select, not a run-time array index, keeps frow/pos in registers)
           tma_load_3d(sA + sa * pl.a_stage + (uint32_t)lane * pl.a_tile, &maps.x, cb * TC_KB,
-                      m == 0 ? frow[0] : frow[MT - 1], m == 0 ? pos[0] : pos[MT - 1], a_bar);
-        } else if (lane < nkb * (MT + 1)) {
-          const int kb = lane - nkb * MT;
-          const int cb = (kb0 + kb + cb_rot) % pl.n_cb;
-          bulk_load(sB + sbi * pl.b_stage + (uint32_t)kb * pl.b_kb,
-                    wslab + (size_t)cb * (pl.b_kb / 2), (uint32_t)pl.b_kb, b_bar);
+                      lane == 0 ? frow[0] : frow[MT - 1], lane == 0 ? pos[0] : pos[MT - 1], a_bar);
+        } else if (lane == MT) {
+          bulk_load(sB + sbi * pl.b_stage, wslab + (size_t)cb * (pl.b_kb / 2), (uint32_t)pl.b_kb,
+                    b_bar);
         }
         __syncwarp();
         if (++sa == pl.sa) { sa = 0; pa ^= 1; a_used = true; }
@@ -390,7 +373,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       const uint32_t a_st16 = (uint32_t)pl.a_stage >> 4, b_st16 = (uint32_t)pl.b_stage >> 4;
       const uint32_t bt16 = (uint32_t)pl.b_tap >> 4;   // one tap's block in w
       const uint32_t bk16 = (2u * lbo_b) >> 4;          // one K step of 16 in w
-      const uint32_t bkb16 = (uint32_t)pl.b_kb >> 4;    // one K-block of w (all taps)
       const uint32_t at16 = (uint32_t)pl.a_tile >> 4;   // next tile of an x stage
       int sa = 0, pa = 0, sbi = 0, pb = 0;
       // Accumulator ring: n_acc slots of NJ columns, one per tile, in order.
@@ -409,7 +391,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           if (++slot == pl.n_acc) { slot = 0; pslot ^= 1; slot_used = true; }
         }
         for (int is = 0; is < pl.n_stage && ok; ++is) {
-          const int nkb = min(KS, pl.n_cb - is * KS);
           const bool last_stage = is == pl.n_stage - 1;
           if (!mbar_wait_bounded(a_full + 8 * sa, (uint32_t)pa, args.err, VI_DEV_ERR_TMA_TIMEOUT) ||
               (!uni &&
@@ -421,22 +402,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           const uint64_t ad_stage = ad_base + (uint64_t)(sa * a_st16);
           const uint64_t bd_stage = bd_base + (uint64_t)(sbi * b_st16);
 #pragma unroll
-          for (int kb = 0; kb < KS; ++kb) {
-            if (kb >= nkb) break;
-#pragma unroll
-            for (int m = 0; m < MT; ++m) {
-              if (is == 0 && kb == 0) {
-                // The slot must have been drained by the epilogue of its last job.
-                if (ju[m] && !mbar_wait_bounded(acc_empty + 8 * js[m], (uint32_t)(jp[m] ^ 1),
-                                                args.err, VI_DEV_ERR_MMA_TIMEOUT)) { ok = false; break; }
-                tc_fence_after();
-              }
-              tc_issue_taps<KT>(dt[m], ad_stage + (uint64_t)((kb * MT + m) * at16),
-                                bd_stage + (uint64_t)(kb * bkb16), bt16, bk16, idesc,
-                                (is > 0 || kb > 0) ? 1u : 0u, k);
-              if (last_stage && kb == nkb - 1) umma_commit(acc_full + 8 * js[m]);   // accumulator ready
+          for (int m = 0; m < MT; ++m) {
+            if (is == 0) {
+              // The slot must have been drained by the epilogue of its last job.
+              if (ju[m] && !mbar_wait_bounded(acc_empty + 8 * js[m], (uint32_t)(jp[m] ^ 1),
+                                              args.err, VI_DEV_ERR_MMA_TIMEOUT)) { ok = false; break; }
+              tc_fence_after();
             }
-            if (!ok) break;
+            tc_issue_taps<KT>(dt[m], ad_stage + (uint64_t)(m * at16), bd_stage, bt16, bk16, idesc,
+                              is > 0 ? 1u : 0u, k);
+            if (last_stage) umma_commit(acc_full + 8 * js[m]);   // accumulator ready
           }
           if (!ok) break;
           if (!uni) umma_commit(b_empty + 8 * sbi);   // frees the w stage when these MMAs finish
@@ -482,7 +457,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         // hT (one table, the plain bias, when hT == 0).
         const int f = fb * TC_M + 32 * q + lane;
         const int lo = min(f, pl.hT), hi = max(min(pl.F - 1 - f, pl.hT), 0);
-        const float* bs = bias_s + (lo * (pl.hT + 1) + hi) * pl.Cout + slab * pl.NJ;
+        // (read through L1: every warp of every CTA reads the same few KB)
+        const float* bs = args.btab + (lo * (pl.hT + 1) + hi) * pl.Cout + slab * pl.NJ;
         const uint32_t taddr = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * pl.NJ);
         // The whole row of the tile (<= 160 columns) into registers first,
         // so that the accumulator goes back to the MMA at once and the
@@ -539,7 +515,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 // K-block, tap) an NJ x 64 K-major block in the no-swizzle layout, the k tap
 // blocks of a (slab, K-block) contiguous.  coef != null (GroupNorm folded
 // into the conv): each input channel's weights are scaled by its GroupNorm
-// factor a_ci first, W'[co][ci][t] = bf16(w[co][ci][t] * a_ci).
+// factor a_ci first, W'[co][ci][t] = bf16(w[co][ci][t] * a_ci), and the bias
+// tables come from temporal_conv_fold_bias; otherwise this kernel also
+// writes the one bias table, b in fp32.
 __device__ __forceinline__ bf16 tc_folded_w(const bf16* w, const float* coef, int co, int ci,
                                             int t, int C, int k) {
   const bf16 v = w[((size_t)co * C + ci) * k + t];
@@ -547,8 +525,13 @@ __device__ __forceinline__ bf16 tc_folded_w(const bf16* w, const float* coef, in
 }
 
 __global__ void temporal_conv_pack_w(const bf16* __restrict__ w, const float* __restrict__ coef,
-                                     bf16* __restrict__ wpk, int C, int Cout, int k, int NJ) {
+                                     bf16* __restrict__ wpk, const bf16* __restrict__ b,
+                                     float* __restrict__ tab, int C, int Cout, int k, int NJ) {
   const long long total = (long long)Cout * C * k;
+  // Plain conv (no GroupNorm folded in): its one bias table is b in fp32.
+  if (!coef)
+    for (int co = blockIdx.x * blockDim.x + threadIdx.x; co < Cout; co += gridDim.x * blockDim.x)
+      tab[co] = __bfloat162float(b[co]);
   const int n_cb = C / TC_KB;
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
        i += (long long)gridDim.x * blockDim.x) {
@@ -619,20 +602,20 @@ constexpr int TC_FOLD_MAX_K = 7;
 
 bool temporal_conv_tc_ok(int F, int P, int C, int k) {
   TcPlan pl;
-  return F > 0 && P > 0 && tc_plan(F, P, C, C, 1, k, pl, 0, 1, 1);
+  return F > 0 && P > 0 && tc_plan(F, P, C, C, 1, k, pl, 0, 1);
 }
 
 bool temporal_conv_tc_norm_ok(int F, int P, int C, int k) {
   TcPlan pl;
-  return F > 0 && P > 0 && k <= TC_FOLD_MAX_K && tc_plan(F, P, C, C, 1, k, pl, k / 2, 1, 1);
+  return F > 0 && P > 0 && k <= TC_FOLD_MAX_K && tc_plan(F, P, C, C, 1, k, pl, k / 2, 1);
 }
 
 bool linear_tc_ok(int F, int P, int C, int Cout, int n_out) {
   TcPlan pl;
-  return F > 0 && P > 0 && tc_plan(F, P, C, Cout, n_out, 1, pl, 0, 1, 1);
+  return F > 0 && P > 0 && tc_plan(F, P, C, Cout, n_out, 1, pl, 0, 1);
 }
 
-template <int KT, int MT, int KS>
+template <int KT, int MT>
 static int tc_launch(const TcMaps& maps, const TcPlan& pl, const TcArgs& a, cudaStream_t stream) {
   static std::mutex mu;
   static bool attr_done[64] = {false};
@@ -642,7 +625,7 @@ static int tc_launch(const TcMaps& maps, const TcPlan& pl, const TcArgs& a, cuda
     std::lock_guard<std::mutex> lock(mu);
     if (dev < 0 || dev >= 64) return VI_ERR_CUDA;
     if (!attr_done[dev]) {
-      VI_CUDA_TRY(cudaFuncSetAttribute(temporal_conv_tc_kernel<KT, MT, KS>,
+      VI_CUDA_TRY(cudaFuncSetAttribute(temporal_conv_tc_kernel<KT, MT>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        TC_SMEM_LIMIT));
       attr_done[dev] = true;
@@ -650,7 +633,7 @@ static int tc_launch(const TcMaps& maps, const TcPlan& pl, const TcArgs& a, cuda
   }
   long long grid = sm_count();
   if (grid > pl.n_jobs) grid = pl.n_jobs;
-  temporal_conv_tc_kernel<KT, MT, KS><<<(unsigned)grid, TC_THREADS, (size_t)pl.smem, stream>>>(
+  temporal_conv_tc_kernel<KT, MT><<<(unsigned)grid, TC_THREADS, (size_t)pl.smem, stream>>>(
       maps, pl, a);
   VI_LAUNCHED();
   return VI_OK;
@@ -661,14 +644,13 @@ static int tc_launch(const TcMaps& maps, const TcPlan& pl, const TcArgs& a, cuda
 static int tc_dispatch(const TcMaps& maps, const TcPlan& pl, const TcArgs& a,
                        cudaStream_t stream) {
   const int kt = pl.k == 3 ? 3 : pl.k == 1 ? 1 : 0;
-  if (pl.KS == 2) return tc_launch<1, 2, 2>(maps, pl, a, stream);   // planned for k = 1, MT = 2
   switch (kt * 10 + pl.MT) {
-    case 32: return tc_launch<3, 2, 1>(maps, pl, a, stream);
-    case 31: return tc_launch<3, 1, 1>(maps, pl, a, stream);
-    case 12: return tc_launch<1, 2, 1>(maps, pl, a, stream);
-    case 11: return tc_launch<1, 1, 1>(maps, pl, a, stream);
-    case 2: return tc_launch<0, 2, 1>(maps, pl, a, stream);
-    default: return tc_launch<0, 1, 1>(maps, pl, a, stream);
+    case 32: return tc_launch<3, 2>(maps, pl, a, stream);
+    case 31: return tc_launch<3, 1>(maps, pl, a, stream);
+    case 12: return tc_launch<1, 2>(maps, pl, a, stream);
+    case 11: return tc_launch<1, 1>(maps, pl, a, stream);
+    case 2: return tc_launch<0, 2>(maps, pl, a, stream);
+    default: return tc_launch<0, 1>(maps, pl, a, stream);
   }
 }
 
@@ -686,18 +668,13 @@ static int tc_run(const bf16* x, int x_rows, int x_off, const bf16* w, const bf1
   if (fold && k > TC_FOLD_MAX_K) return VI_ERR_UNSUPPORTED;
   const int hT = fold ? k / 2 : 0;
   if (mt != 0) {
-    if (!tc_plan(F, P, C, Cout, n_out, k, pl, hT, mt, 1)) return VI_ERR_UNSUPPORTED;
+    if (!tc_plan(F, P, C, Cout, n_out, k, pl, hT, mt)) return VI_ERR_UNSUPPORTED;
   } else {
-    if (!tc_plan(F, P, C, Cout, n_out, k, pl, hT, 1, 1)) return VI_ERR_UNSUPPORTED;
+    if (!tc_plan(F, P, C, Cout, n_out, k, pl, hT, 1)) return VI_ERR_UNSUPPORTED;
     // Two tiles per job when that plan keeps the slab width (a narrower MMA
     // N costs more than the weight traffic it saves).
     TcPlan pl2;
-    if (tc_plan(F, P, C, Cout, n_out, k, pl2, hT, TC_MT_DEFAULT, 1) && pl2.NJ >= pl.NJ) pl = pl2;
-    // Single tap: two K-blocks per stage where they fit at the same width, so
-    // a stage still queues 16 MMAs per wait/commit.
-    if (k == 1 && pl.MT == 2 && tc_plan(F, P, C, Cout, n_out, k, pl2, hT, 2, 2) &&
-        pl2.NJ >= pl.NJ)
-      pl = pl2;
+    if (tc_plan(F, P, C, Cout, n_out, k, pl2, hT, TC_MT_DEFAULT) && pl2.NJ >= pl.NJ) pl = pl2;
   }
   if (part != VI_PART_ALL) {
     // Frame blocks whose x rows (with the k/2 rows on each side) lie inside
@@ -745,19 +722,19 @@ static int tc_run(const bf16* x, int x_rows, int x_off, const bf16* w, const bf1
                      CU_TENSOR_MAP_DATA_TYPE_BFLOAT16))
       return VI_ERR_CUDA;
   }
-  // Scratch: the packed weights, then (folded conv) the bias tables.
+  // Scratch: the packed weights, then the bias tables (fp32).
   const size_t wbytes = (((size_t)Cout * C * k * sizeof(bf16)) + 255) / 256 * 256;
-  const size_t tbytes = fold ? (size_t)pl.n_tab * Cout * sizeof(float) : 0;
+  const size_t tbytes = (size_t)pl.n_tab * Cout * sizeof(float);
   void* scratch = nullptr;
   VI_CUDA_TRY(scratch_alloc(&scratch, wbytes + tbytes, stream));
   bf16* wpk = static_cast<bf16*>(scratch);
-  float* tab = fold ? reinterpret_cast<float*>(static_cast<char*>(scratch) + wbytes) : nullptr;
+  float* tab = reinterpret_cast<float*>(static_cast<char*>(scratch) + wbytes);
   int st = VI_OK;
   {
     const long long total = (long long)Cout * C * k;
     int blocks = (int)((total + 255) / 256);
     if (blocks > 4 * sm_count()) blocks = 4 * sm_count();
-    temporal_conv_pack_w<<<blocks, 256, 0, stream>>>(w, coef, wpk, C, Cout, k, pl.NJ);
+    temporal_conv_pack_w<<<blocks, 256, 0, stream>>>(w, coef, wpk, b, tab, C, Cout, k, pl.NJ);
     if (cudaGetLastError() != cudaSuccess) st = VI_ERR_CUDA; else note_launch();
   }
   if (st == VI_OK && fold) {
@@ -765,7 +742,7 @@ static int tc_run(const bf16* x, int x_rows, int x_off, const bf16* w, const bf1
     if (cudaGetLastError() != cudaSuccess) st = VI_ERR_CUDA; else note_launch();
   }
   if (st == VI_OK) {
-    const TcArgs a{tab, b, wpk, err, x_off};
+    const TcArgs a{tab, wpk, err, x_off};
     st = tc_dispatch(maps, pl, a, stream);
   }
   if (scratch_free(scratch, stream) != cudaSuccess && st == VI_OK) st = VI_ERR_CUDA;
