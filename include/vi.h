@@ -169,7 +169,7 @@ int vi_groupnorm_global_f32(const void* x, const void* gamma, const void* beta, 
 /*
  * Temporal attention module: input projections, dual-domain attention, output
  * projection (bf16).  The attention-module paragraph redefines how the keys and
- * values are gathered ("modifying the K-V computation"); the projections
+ * values are gathered (the module changes its K/V computation); the projections
  * around it are the module's linear layers:
  *   q = x Wq^T + bq,  k = x Wk^T + bk,  v = x Wv^T + bv      (per frame)
  *   a = vi_dual_attn(q, k, v; heads, d, n_pre, n_post, n_global)

@@ -6,7 +6,9 @@ write-up), attention-module paragraph: the module's keys and values are
 gathered from the clip, its neighbours and the global frames; the linear
 projections around the attention are the module's own layers.  The oracle
 composes its pinned projection (single-tap conv) and attention functions with
-bf16 intermediates, the tensors the module's stages exchange."""
+bf16 intermediates, the tensors the module's stages exchange.  Tolerance: the
+attention's 2e-2 (the outputs are convex combinations of v projected with
+fan-in-scaled weights, sigma ~ 1)."""
 import numpy as np
 import pytest
 import torch
@@ -33,7 +35,8 @@ def run_case(w, positions=None):
                                     w.n_post, w.n_global, positions=positions)
     if positions is not None:
         got = got[positions]
-    return assert_close(got, ref, w.dtype, "gn", w.name)
+    # the attention tolerance (2e-2): module outputs have sigma ~ 1
+    return assert_close(got, ref, w.dtype, "attn", w.name)
 
 
 def W(name, F, N, P, heads, **kw):
