@@ -74,7 +74,9 @@ struct TcPlan {
   int F, P, C, k;
   int Cout;              // output channels (all output tensors together)
   int NJ;                // output channels per job (UMMA N), multiple of 32
-  int MT;                // tiles per job (1, or 2 sharing every weight stage)
+  int MT;                // tiles per job per CTA (1, or 2 sharing every weight stage)
+  int H;                 // CTAs per MMA: 1, or 2 for a CTA pair (M = 256, each holding NJ/2 weight rows)
+  int b_rows;            // weight rows per CTA = NJ / H
   int n_stage;           // stages per job = n_cb (a stage is one K-block)
   int n_acc;             // TMEM accumulators in the ring (MT + 1, at least 2), NJ columns each
   int n_slabs;           // Cout / NJ
@@ -83,12 +85,12 @@ struct TcPlan {
   int sel_lo, sel_hi0, n_sel;   // frame blocks computed per position: [0, sel_lo) and
                                 // [sel_hi0, sel_hi0 + n_sel - sel_lo) (all of them by default)
   long long n_tiles;     // P * n_sel
-  long long n_jobs;      // ceil(n_tiles / MT) * n_slabs
+  long long n_jobs;      // ceil(n_tiles / (H MT)) * n_slabs
   int n_cb;              // C / 64
   int a_rows;            // 127 + k
   int a_tile;            // bytes of one tile's x box (a_rows x 128 B), 1024-aligned
   int a_stage;           // bytes per A stage = MT * a_tile
-  int b_tap;             // bytes of one tap's block = NJ * 128
+  int b_tap;             // bytes of one tap's block = b_rows * 128
   int b_kb;              // weight bytes of one K-block = k * b_tap (all taps)
   int b_stage;           // bytes per B stage = b_kb
   int sa;                // A stages
@@ -108,9 +110,11 @@ struct TcArgs {
 };
 
 // Tensor maps of one launch: x as [P][x_rows][C], each output as
-// [P][F][Cout/n_out] with 64-channel boxes (y) and 32-channel boxes (y32).
+// [P][F][Cout/n_out] with 64-channel boxes (y) and 32-channel boxes (y32),
+// and (CTA pair) the packed weights as blocks of b_rows x 128 bytes.
 struct TcMaps {
   CUtensorMap x;
+  CUtensorMap w;
   CUtensorMap y[TC_MAX_OUT];
   CUtensorMap y32[TC_MAX_OUT];
 };
@@ -123,10 +127,12 @@ struct TcMaps {
 // chunks (two 4 KB buffers per warp) where that still leaves the widest slab
 // room, else 32-channel chunks (two 2 KB buffers per warp).
 static bool tc_plan(int F, int P, int C, int Cout, int n_out, int k, TcPlan& pl, int hT,
-                    int mt) {
+                    int mt, bool pair = false) {
   if (k < 1 || k % 2 == 0 || 127 + k > 256 || C % TC_KB != 0) return false;
   if (n_out < 1 || n_out > TC_MAX_OUT || Cout <= 0 || Cout % n_out != 0) return false;
   if (mt != 1 && mt != 2) return false;
+  if (pair && mt != 2) return false;
+  const int H = pair ? 2 : 1;
   if (hT < 0 || hT > k / 2) return false;
   const int n_tab = (hT + 1) * (hT + 1);
   const int cpo = Cout / n_out;
@@ -139,8 +145,8 @@ static bool tc_plan(int F, int P, int C, int Cout, int n_out, int k, TcPlan& pl,
   // output tensor's channels) whose all-tap weight stages leave room for at
   // least two of each ring.
   for (int nj = TC_NJ_MAX; nj >= 32; nj -= 32) {
-    if (cpo % nj != 0 || n_acc * nj > TC_TMEM_COLS) continue;
-    const int b_stage = k * nj * 128;
+    if (cpo % nj != 0 || n_acc * nj > TC_TMEM_COLS || (nj / H) % 8 != 0) continue;
+    const int b_stage = k * (nj / H) * 128;
     for (int wide = 1; wide >= 0; --wide) {
       const int fixed = base + 4 * 2 * (wide ? TC_OUT_BUF : TC_OUT_BUF / 2);   // output staging
       int sa, sb;
@@ -166,6 +172,8 @@ static bool tc_plan(int F, int P, int C, int Cout, int n_out, int k, TcPlan& pl,
       pl.Cout = Cout;
       pl.NJ = nj;
       pl.MT = mt;
+      pl.H = H;
+      pl.b_rows = nj / H;
       pl.n_acc = n_acc;
       pl.n_slabs = Cout / nj;
       pl.slabs_per_out = cpo / nj;
@@ -173,13 +181,13 @@ static bool tc_plan(int F, int P, int C, int Cout, int n_out, int k, TcPlan& pl,
       pl.sel_lo = pl.n_sel = pl.n_fblk;
       pl.sel_hi0 = 0;
       pl.n_tiles = (long long)P * pl.n_fblk;
-      pl.n_jobs = ((pl.n_tiles + mt - 1) / mt) * pl.n_slabs;
+      pl.n_jobs = ((pl.n_tiles + H * mt - 1) / (H * mt)) * pl.n_slabs;
       pl.n_cb = C / TC_KB;
       pl.n_stage = pl.n_cb;
       pl.a_rows = a_rows;
       pl.a_tile = a_tile;
       pl.a_stage = a_stage;
-      pl.b_tap = nj * 128;
+      pl.b_tap = (nj / H) * 128;
       pl.b_kb = k * pl.b_tap;
       pl.b_stage = b_stage;
       pl.sa = sa;
@@ -206,7 +214,14 @@ __device__ __forceinline__ void tc_tile_pos(const TcPlan& pl, long long t, int& 
 // Tap t reads the x tile shifted down by t rows of 128 B (8 units of 16 B);
 // K step s adds 32 B inside the swizzled x rows and two 8-column groups in w.
 // KT > 0: taps known at compile time, every offset an immediate.
-template <int KT>
+template <bool PAIR>
+__device__ __forceinline__ void tc_umma(uint32_t d_tmem, uint64_t ad, uint64_t bd, uint32_t idesc,
+                                        uint32_t acc) {
+  if constexpr (PAIR) umma_bf16_pair(d_tmem, ad, bd, idesc, acc);
+  else umma_bf16(d_tmem, ad, bd, idesc, acc);
+}
+
+template <int KT, bool PAIR>
 __device__ __forceinline__ void tc_issue_taps(uint32_t d_tmem, uint64_t ad, uint64_t bd,
                                               uint32_t bt16, uint32_t bk16, uint32_t idesc,
                                               uint32_t acc0, int k) {
@@ -215,17 +230,25 @@ __device__ __forceinline__ void tc_issue_taps(uint32_t d_tmem, uint64_t ad, uint
     for (int t = 0; t < KT; ++t) {
 #pragma unroll
       for (int s = 0; s < 4; ++s)
-        umma_bf16(d_tmem, ad + (uint64_t)(8 * t + 2 * s), bd + (uint64_t)(t * bt16 + s * bk16),
-                  idesc, (t == 0 && s == 0) ? acc0 : 1u);
+        tc_umma<PAIR>(d_tmem, ad + (uint64_t)(8 * t + 2 * s), bd + (uint64_t)(t * bt16 + s * bk16),
+                      idesc, (t == 0 && s == 0) ? acc0 : 1u);
     }
   } else {
     for (int t = 0; t < k; ++t) {
 #pragma unroll
       for (int s = 0; s < 4; ++s)
-        umma_bf16(d_tmem, ad + (uint64_t)(8 * t + 2 * s), bd + (uint64_t)(t * bt16 + s * bk16),
-                  idesc, (t == 0 && s == 0) ? acc0 : 1u);
+        tc_umma<PAIR>(d_tmem, ad + (uint64_t)(8 * t + 2 * s), bd + (uint64_t)(t * bt16 + s * bk16),
+                      idesc, (t == 0 && s == 0) ? acc0 : 1u);
     }
   }
+}
+
+// Commit: arrive on `bar` (in both CTAs of a pair) once this thread's
+// outstanding MMAs are done.
+template <bool PAIR>
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  if constexpr (PAIR) umma_commit_pair_mc(bar, 0x3);
+  else umma_commit(bar);
 }
 
 // Epilogue of one chunk of a tile row: + bias, -> bf16, into the staging
@@ -263,7 +286,25 @@ __device__ __forceinline__ void epi_stage_chunk(uint32_t stage, int lane, const 
   }
 }
 
-template <int KT, int MT>
+// Bounded wait; cluster-scope acquire in the pair form, where the barrier is
+// signalled from the other CTA (remote arrivals, commits multicast to both).
+template <bool PAIR>
+__device__ __forceinline__ bool tc_wait(uint32_t bar, uint32_t parity, unsigned int* err,
+                                        unsigned int code) {
+  if constexpr (PAIR) return mbar_wait_bounded_cluster(bar, parity, err, code);
+  else return mbar_wait_bounded(bar, parity, err, code);
+}
+
+// PAIR: a cluster of two CTAs on two SMs runs tcgen05.mma.cta_group::2 with
+// M = 256.  Each CTA holds its own MT tiles of x (A rows 0..127 of the MMA in
+// the even CTA, 128..255 in the odd one) and HALF of every weight block (N/2
+// rows each), and its own 128 accumulator lanes in TMEM.  The even CTA's
+// thread issues the MMAs; both CTAs' loads complete on the even CTA's full
+// barriers, the commits go to both CTAs' barriers, and the epilogues of both
+// arrive on the even CTA's accumulator-empty barriers.  Per SM this halves
+// the weight bytes streamed from L2 and the B operand read from shared
+// memory per MMA.
+template <int KT, int MT, bool PAIR>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     temporal_conv_tc_kernel(const __grid_constant__ TcMaps maps, const TcPlan pl,
                             const TcArgs args) {
@@ -282,29 +323,44 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int k = KT > 0 ? KT : pl.k;
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const long long cid = PAIR ? blockIdx.x / 2 : blockIdx.x;        // cluster (job walker) index
+  const long long n_cl = PAIR ? gridDim.x / 2 : gridDim.x;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < pl.sa; ++i) { mbar_init(a_full + 8 * i, 1); mbar_init(a_empty + 8 * i, 1); }
+    for (int i = 0; i < pl.sa; ++i) {
+      mbar_init(a_full + 8 * i, PAIR ? 2 : 1);       // one arrive.expect_tx per CTA
+      mbar_init(a_empty + 8 * i, 1);
+    }
     for (int i = 0; i < pl.sb; ++i) { mbar_init(b_full + 8 * i, 1); mbar_init(b_empty + 8 * i, 1); }
     for (int i = 0; i < pl.n_acc; ++i) {
       mbar_init(acc_full + 8 * i, 1);
-      mbar_init(acc_empty + 8 * i, TC_EPI_WARPS);
+      mbar_init(acc_empty + 8 * i, PAIR ? 2 * TC_EPI_WARPS : TC_EPI_WARPS);
     }
     mbar_init(drain, 1);
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, TC_TMEM_COLS);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(tmem_slot, TC_TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, TC_TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) cluster_sync();               // both CTAs' barriers are initialised
   tc_fence_after();
   uint32_t tmem_base;
   asm volatile("ld.shared.u32 %0, [%1];" : "=r"(tmem_base) : "r"(tmem_slot));
+  // The even CTA's full and accumulator-empty barriers, as cluster addresses.
+  const uint32_t lead_a_full = PAIR ? mapa_shared(a_full, 0) : a_full;
+  const uint32_t lead_acc_empty = PAIR ? mapa_shared(acc_empty, 0) : acc_empty;
 
   const int halo = k / 2;
-  const int cb_rot = (int)(blockIdx.x % pl.n_cb);
+  const int cb_rot = (int)(cid % pl.n_cb);          // the same K-block order in both CTAs
   // Equal x and w rings (the two-tile form): one barrier pair per stage covers
   // both, so a K-block costs one wait and one commit.
   const bool uni = pl.sa == pl.sb;
@@ -318,9 +374,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     bool a_used = false, b_used = false;           // first pass over a ring needs no wait
     bool ok = true;
     const uint32_t a_bytes = (uint32_t)(MT * pl.a_rows) * 128u;
-    for (long long job = blockIdx.x; job < pl.n_jobs && ok; job += gridDim.x) {
+    for (long long job = cid; job < pl.n_jobs && ok; job += n_cl) {
       const int slab = (int)(job % pl.n_slabs);
-      const long long tile0 = (job / pl.n_slabs) * MT;
+      const long long tile0 = (job / pl.n_slabs) * (pl.H * MT) + rank * MT;
       // Frame row and position of each tile of the job; p == P past the
       // last tile, which reads as zeros.
       int frow[MT], pos[MT];
@@ -330,20 +386,25 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         tc_tile_pos(pl, tile0 + m, fb, pos[m]);
         frow[m] = fb * TC_M - halo + args.x_off;
       }
-      // Packed weights of (slab, K-block 0): k contiguous tap blocks per K-block.
+      // Packed weights of (slab, K-block 0): k contiguous tap blocks per K-block
+      // (per CTA of a pair: its half).
       const bf16* wslab = args.wpk + (size_t)slab * pl.n_cb * (pl.b_kb / 2);
+      const int wblk0 = (slab * pl.n_cb * pl.H + (int)rank) * k;   // pair: block of (slab, 0, rank, 0)
       for (int is = 0; is < pl.n_stage; ++is) {
         // Stage `is` holds K-block (is + cb_rot) mod n_cb of the job.
         const int cb = (is + cb_rot) % pl.n_cb;
-        const uint32_t a_bar = a_full + 8 * sa;
+        const uint32_t a_bar = PAIR ? lead_a_full + 8 * sa : a_full + 8 * sa;
         const uint32_t b_bar = uni ? a_bar : b_full + 8 * sbi;   // shared stage: one barrier
         bool go = true;
         if (lane == 0) {
-          go = !a_used || mbar_wait_bounded(a_empty + 8 * sa, (uint32_t)(pa ^ 1), args.err,
-                                            VI_DEV_ERR_TMA_TIMEOUT);
-          if (go) mbar_arrive_expect_tx(a_bar, a_bytes + (uni ? (uint32_t)pl.b_kb : 0u));
+          go = !a_used || tc_wait<PAIR>(a_empty + 8 * sa, (uint32_t)(pa ^ 1), args.err,
+                                        VI_DEV_ERR_TMA_TIMEOUT);
+          if (go) {
+            if constexpr (PAIR) mbar_arrive_expect_tx_cluster(a_bar, a_bytes + (uint32_t)pl.b_kb);
+            else mbar_arrive_expect_tx(a_bar, a_bytes + (uni ? (uint32_t)pl.b_kb : 0u));
+          }
           if (go && !uni) {
-            go = !b_used || mbar_wait_bounded(b_empty + 8 * sbi, (uint32_t)(pb ^ 1), args.err,
+            go = !b_used || tc_wait<PAIR>(b_empty + 8 * sbi, (uint32_t)(pb ^ 1), args.err,
                                               VI_DEV_ERR_TMA_TIMEOUT);
             if (go) mbar_arrive_expect_tx(b_bar, (uint32_t)pl.b_kb);
           }
@@ -351,11 +412,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         if (!__shfl_sync(0xffffffffu, go ? 1 : 0, 0)) { ok = false; break; }
         if (lane < MT) {
           // (a select, not a run-time array index, keeps frow/pos in registers)
-          tma_load_3d(sA + sa * pl.a_stage + (uint32_t)lane * pl.a_tile, &maps.x, cb * TC_KB,
-                      lane == 0 ? frow[0] : frow[MT - 1], lane == 0 ? pos[0] : pos[MT - 1], a_bar);
+          const uint32_t dst = sA + sa * pl.a_stage + (uint32_t)lane * pl.a_tile;
+          const int fr = lane == 0 ? frow[0] : frow[MT - 1], ps = lane == 0 ? pos[0] : pos[MT - 1];
+          if constexpr (PAIR) tma_load_3d_pair(dst, &maps.x, cb * TC_KB, fr, ps, a_bar);
+          else tma_load_3d(dst, &maps.x, cb * TC_KB, fr, ps, a_bar);
         } else if (lane == MT) {
-          bulk_load(sB + sbi * pl.b_stage, wslab + (size_t)cb * (pl.b_kb / 2), (uint32_t)pl.b_kb,
-                    b_bar);
+          if constexpr (PAIR)
+            tma_load_3d_pair(sB + sbi * pl.b_stage, &maps.w, 0, 0, wblk0 + cb * pl.H * k, b_bar);
+          else
+            bulk_load(sB + sbi * pl.b_stage, wslab + (size_t)cb * (pl.b_kb / 2), (uint32_t)pl.b_kb,
+                      b_bar);
         }
         __syncwarp();
         if (++sa == pl.sa) { sa = 0; pa ^= 1; a_used = true; }
@@ -364,9 +430,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc = umma_idesc_bf16_f32(TC_M, pl.NJ);
-      const uint32_t lbo_b = (uint32_t)pl.NJ * 16u;
+    if (lane == 0 && rank == 0) {
+      const uint32_t idesc = umma_idesc_bf16_f32(TC_M * pl.H, pl.NJ);
+      const uint32_t lbo_b = (uint32_t)pl.b_rows * 16u;
       // Descriptors of stage 0; stage s adds s * stage_bytes / 16 to the start field.
       const uint64_t ad_base = umma_desc_kmajor_sw128(sA, 1024u);
       const uint64_t bd_base = umma_desc_kmajor_noswizzle(sB, lbo_b, 128u);
@@ -379,7 +445,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       int slot = 0, pslot = 0;
       bool slot_used = false;
       bool ok = true;
-      for (long long job = blockIdx.x; job < pl.n_jobs && ok; job += gridDim.x) {
+      for (long long job = cid; job < pl.n_jobs && ok; job += n_cl) {
         // This job's accumulator slots and the parity of their last release.
         int js[MT], jp[MT];
         bool ju[MT];
@@ -392,9 +458,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
         for (int is = 0; is < pl.n_stage && ok; ++is) {
           const bool last_stage = is == pl.n_stage - 1;
-          if (!mbar_wait_bounded(a_full + 8 * sa, (uint32_t)pa, args.err, VI_DEV_ERR_TMA_TIMEOUT) ||
+          if (!tc_wait<PAIR>(a_full + 8 * sa, (uint32_t)pa, args.err, VI_DEV_ERR_TMA_TIMEOUT) ||
               (!uni &&
-               !mbar_wait_bounded(b_full + 8 * sbi, (uint32_t)pb, args.err, VI_DEV_ERR_TMA_TIMEOUT))) {
+               !tc_wait<PAIR>(b_full + 8 * sbi, (uint32_t)pb, args.err, VI_DEV_ERR_TMA_TIMEOUT))) {
             ok = false;
             break;
           }
@@ -405,24 +471,24 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           for (int m = 0; m < MT; ++m) {
             if (is == 0) {
               // The slot must have been drained by the epilogue of its last job.
-              if (ju[m] && !mbar_wait_bounded(acc_empty + 8 * js[m], (uint32_t)(jp[m] ^ 1),
-                                              args.err, VI_DEV_ERR_MMA_TIMEOUT)) { ok = false; break; }
+              if (ju[m] && !tc_wait<PAIR>(acc_empty + 8 * js[m], (uint32_t)(jp[m] ^ 1),
+                                          args.err, VI_DEV_ERR_MMA_TIMEOUT)) { ok = false; break; }
               tc_fence_after();
             }
-            tc_issue_taps<KT>(dt[m], ad_stage + (uint64_t)(m * at16), bd_stage, bt16, bk16, idesc,
-                              is > 0 ? 1u : 0u, k);
-            if (last_stage) umma_commit(acc_full + 8 * js[m]);   // accumulator ready
+            tc_issue_taps<KT, PAIR>(dt[m], ad_stage + (uint64_t)(m * at16), bd_stage, bt16, bk16,
+                                    idesc, is > 0 ? 1u : 0u, k);
+            if (last_stage) tc_commit<PAIR>(acc_full + 8 * js[m]);   // accumulator ready
           }
           if (!ok) break;
-          if (!uni) umma_commit(b_empty + 8 * sbi);   // frees the w stage when these MMAs finish
-          umma_commit(a_empty + 8 * sa);              // frees the x stage (and the w stage if shared)
+          if (!uni) tc_commit<PAIR>(b_empty + 8 * sbi);   // frees the w stage when these MMAs finish
+          tc_commit<PAIR>(a_empty + 8 * sa);              // frees the x stage (and the w stage if shared)
           if (++sbi == pl.sb) { sbi = 0; pb ^= 1; }
           if (++sa == pl.sa) { sa = 0; pa ^= 1; }
         }
       }
       // Every MMA this thread issued must finish before TMEM is released.
-      umma_commit(drain);
-      mbar_wait_bounded(drain, 0, args.err, VI_DEV_ERR_MMA_TIMEOUT);
+      tc_commit<PAIR>(drain);
+      tc_wait<PAIR>(drain, 0, args.err, VI_DEV_ERR_MMA_TIMEOUT);
     }
   } else {
     // ------------------------------------------------------------ epilogue
@@ -436,20 +502,20 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     int ob = 0;                                  // staging buffer of the next chunk
     int buf = 0, pacc = 0;                       // accumulator ring, as the MMA issuer walks it
     bool ok = true;
-    for (long long job = blockIdx.x; job < pl.n_jobs && ok; job += gridDim.x) {
+    for (long long job = cid; job < pl.n_jobs && ok; job += n_cl) {
       const int slab = (int)(job % pl.n_slabs);
       const int out = slab / pl.slabs_per_out;                 // output tensor of this slab
       const int ch0 = (slab - out * pl.slabs_per_out) * pl.NJ; // its first channel there
       for (int mt = 0; mt < MT; ++mt) {
         // The lanes take the (bounded) wait's outcome together.
-        const bool got = __all_sync(0xffffffffu, mbar_wait_bounded(acc_full + 8 * buf, (uint32_t)pacc,
-                                                                    args.err, VI_DEV_ERR_MMA_TIMEOUT));
+        const bool got = __all_sync(0xffffffffu, tc_wait<PAIR>(acc_full + 8 * buf, (uint32_t)pacc,
+                                                                args.err, VI_DEV_ERR_MMA_TIMEOUT));
         if (!got) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const long long tile = (job / pl.n_slabs) * MT + mt;
+        const long long tile = (job / pl.n_slabs) * (pl.H * MT) + rank * MT + mt;
         int fb, p;
         tc_tile_pos(pl, tile, fb, p);
         const bool tile_ok = tile < pl.n_tiles;
@@ -472,7 +538,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           if (32 * c < pl.NJ) tmem_wait_ld_dep(r[c]);
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(acc_empty + 8 * buf);
+        if (lane == 0) {
+          if constexpr (PAIR) mbar_arrive_cluster(lead_acc_empty + 8 * buf);
+          else mbar_arrive(acc_empty + 8 * buf);
+        }
         // Chunks: 64 channels (groups g, g+1) where the plan is wide and
         // they fit, else 32 (group g).  Loops unrolled: registers indexed
         // at compile time only.
@@ -505,15 +574,18 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) cluster_sync();        // the pair is done with each other's memory
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, TC_TMEM_COLS);
+    if constexpr (PAIR) tmem_dealloc_pair(tmem_base, TC_TMEM_COLS);
+    else tmem_dealloc(tmem_base, TC_TMEM_COLS);
   }
 }
 
-// w [C_out][C_in][k] -> [slab][cb][t][8 columns][NJ][8]: for each (slab,
-// K-block, tap) an NJ x 64 K-major block in the no-swizzle layout, the k tap
-// blocks of a (slab, K-block) contiguous.  coef != null (GroupNorm folded
+// w [C_out][C_in][k] -> [slab][cb][h][t][8 columns][NJ/H][8]: for each (slab,
+// K-block, CTA h of a pair (H = 2) or h = 0 (H = 1), tap) an NJ/H x 64 K-major
+// block in the no-swizzle layout, the k tap blocks of a (slab, K-block, h)
+// contiguous.  coef != null (GroupNorm folded
 // into the conv): each input channel's weights are scaled by its GroupNorm
 // factor a_ci first, W'[co][ci][t] = bf16(w[co][ci][t] * a_ci), and the bias
 // tables come from temporal_conv_fold_bias; otherwise this kernel also
@@ -526,7 +598,8 @@ __device__ __forceinline__ bf16 tc_folded_w(const bf16* w, const float* coef, in
 
 __global__ void temporal_conv_pack_w(const bf16* __restrict__ w, const float* __restrict__ coef,
                                      bf16* __restrict__ wpk, const bf16* __restrict__ b,
-                                     float* __restrict__ tab, int C, int Cout, int k, int NJ) {
+                                     float* __restrict__ tab, int C, int Cout, int k, int NJ,
+                                     int H) {
   const long long total = (long long)Cout * C * k;
   // Plain conv (no GroupNorm folded in): its one bias table is b in fp32.
   if (!coef)
@@ -535,14 +608,16 @@ __global__ void temporal_conv_pack_w(const bf16* __restrict__ w, const float* __
   const int n_cb = C / TC_KB;
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
        i += (long long)gridDim.x * blockDim.x) {
+    const int R = NJ / H;
     const int e = (int)(i & 7);
     long long r = i >> 3;
-    const int n = (int)(r % NJ); r /= NJ;
+    const int n = (int)(r % R); r /= R;
     const int col = (int)(r % 8); r /= 8;
     const int t = (int)(r % k); r /= k;
+    const int h = (int)(r % H); r /= H;
     const int cb = (int)(r % n_cb);
     const int slab = (int)(r / n_cb);
-    wpk[i] = tc_folded_w(w, coef, slab * NJ + n, cb * TC_KB + col * 8 + e, t, C, k);
+    wpk[i] = tc_folded_w(w, coef, slab * NJ + h * R + n, cb * TC_KB + col * 8 + e, t, C, k);
   }
 }
 
@@ -596,6 +671,14 @@ bool encode_tmap(CUtensorMap* map, const void* base, int rank, const uint64_t* d
 
 // Tiles per job of the default plan (2: every weight stage feeds two tiles).
 constexpr int TC_MT_DEFAULT = 2;
+// The default plan runs on a CTA pair for convs of k >= 3 taps with at least
+// this many K-blocks per job, where the pair plan keeps the slab width.
+// Measured on B200 (cycles per 128-row MMA per SM, as dispatched): C = 640,
+// 10 K-blocks: 95 on a pair against 99 on one SM; C = 320, 5 K-blocks: 108
+// against 103 (the pair's accumulator hand-off, which waits for both CTAs'
+// epilogues, costs more per job than the pair saves); the single-tap GEMMs of
+// the attention module ran slower on pairs as well.
+constexpr int TC_PAIR_MIN_KBLOCKS = 10;
 // Largest tap count of the GroupNorm-folded conv (bias tables per distance to
 // the video ends: (k/2 + 1)^2 of them).
 constexpr int TC_FOLD_MAX_K = 7;
@@ -615,7 +698,7 @@ bool linear_tc_ok(int F, int P, int C, int Cout, int n_out) {
   return F > 0 && P > 0 && tc_plan(F, P, C, Cout, n_out, 1, pl, 0, 1);
 }
 
-template <int KT, int MT>
+template <int KT, int MT, bool PAIR>
 static int tc_launch(const TcMaps& maps, const TcPlan& pl, const TcArgs& a, cudaStream_t stream) {
   static std::mutex mu;
   static bool attr_done[64] = {false};
@@ -625,17 +708,41 @@ static int tc_launch(const TcMaps& maps, const TcPlan& pl, const TcArgs& a, cuda
     std::lock_guard<std::mutex> lock(mu);
     if (dev < 0 || dev >= 64) return VI_ERR_CUDA;
     if (!attr_done[dev]) {
-      VI_CUDA_TRY(cudaFuncSetAttribute(temporal_conv_tc_kernel<KT, MT>,
+      VI_CUDA_TRY(cudaFuncSetAttribute(temporal_conv_tc_kernel<KT, MT, PAIR>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        TC_SMEM_LIMIT));
       attr_done[dev] = true;
     }
   }
-  long long grid = sm_count();
-  if (grid > pl.n_jobs) grid = pl.n_jobs;
-  temporal_conv_tc_kernel<KT, MT><<<(unsigned)grid, TC_THREADS, (size_t)pl.smem, stream>>>(
-      maps, pl, a);
-  VI_LAUNCHED();
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.blockDim = dim3(TC_THREADS);
+  cfg.dynamicSmemBytes = (size_t)pl.smem;
+  cfg.stream = stream;
+  long long grid;
+  if constexpr (PAIR) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cfg.gridDim = dim3(2 * sm_count());
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, temporal_conv_tc_kernel<KT, MT, PAIR>, &cfg) !=
+            cudaSuccess ||
+        clusters < 1)
+      clusters = sm_count() / 2;
+    grid = clusters;
+    if (grid > pl.n_jobs) grid = pl.n_jobs;
+    grid *= 2;
+  } else {
+    grid = sm_count();
+    if (grid > pl.n_jobs) grid = pl.n_jobs;
+  }
+  cfg.gridDim = dim3((unsigned)grid);
+  VI_CUDA_TRY(cudaLaunchKernelEx(&cfg, temporal_conv_tc_kernel<KT, MT, PAIR>, maps, pl, a));
+  note_launch();
   return VI_OK;
 }
 
@@ -644,13 +751,20 @@ static int tc_launch(const TcMaps& maps, const TcPlan& pl, const TcArgs& a, cuda
 static int tc_dispatch(const TcMaps& maps, const TcPlan& pl, const TcArgs& a,
                        cudaStream_t stream) {
   const int kt = pl.k == 3 ? 3 : pl.k == 1 ? 1 : 0;
+  if (pl.H == 2) {                          // CTA pair, two tiles per CTA
+    switch (kt) {
+      case 3: return tc_launch<3, 2, true>(maps, pl, a, stream);
+      case 1: return tc_launch<1, 2, true>(maps, pl, a, stream);
+      default: return tc_launch<0, 2, true>(maps, pl, a, stream);
+    }
+  }
   switch (kt * 10 + pl.MT) {
-    case 32: return tc_launch<3, 2>(maps, pl, a, stream);
-    case 31: return tc_launch<3, 1>(maps, pl, a, stream);
-    case 12: return tc_launch<1, 2>(maps, pl, a, stream);
-    case 11: return tc_launch<1, 1>(maps, pl, a, stream);
-    case 2: return tc_launch<0, 2>(maps, pl, a, stream);
-    default: return tc_launch<0, 1>(maps, pl, a, stream);
+    case 32: return tc_launch<3, 2, false>(maps, pl, a, stream);
+    case 31: return tc_launch<3, 1, false>(maps, pl, a, stream);
+    case 12: return tc_launch<1, 2, false>(maps, pl, a, stream);
+    case 11: return tc_launch<1, 1, false>(maps, pl, a, stream);
+    case 2: return tc_launch<0, 2, false>(maps, pl, a, stream);
+    default: return tc_launch<0, 1, false>(maps, pl, a, stream);
   }
 }
 
@@ -659,7 +773,9 @@ static int tc_dispatch(const TcMaps& maps, const TcPlan& pl, const TcArgs& a,
 // coef != nullptr: the conv of the GroupNorm of x, with the GroupNorm's
 // per-channel coefficients (m_c, a_c, beta_c) folded into the weights and the
 // bias tables (fused GroupNorm -> conv; see temporal_conv_fold_bias).
-// mt: tiles per job, 0 = the default plan.
+// mt: tiles per job, 0 = the default plan (two tiles on one SM where that
+// keeps the slab width, else one; a CTA pair with two tiles per CTA for
+// k >= 3 convs with long jobs); 1 or 2 force that one-SM form, 4 the pair.
 static int tc_run(const bf16* x, int x_rows, int x_off, const bf16* w, const bf16* b,
                   bf16* const* ys, int n_out, int F, int P, int C, int Cout, int k,
                   cudaStream_t stream, const float* coef, int mt, int part = VI_PART_ALL) {
@@ -668,13 +784,18 @@ static int tc_run(const bf16* x, int x_rows, int x_off, const bf16* w, const bf1
   if (fold && k > TC_FOLD_MAX_K) return VI_ERR_UNSUPPORTED;
   const int hT = fold ? k / 2 : 0;
   if (mt != 0) {
-    if (!tc_plan(F, P, C, Cout, n_out, k, pl, hT, mt)) return VI_ERR_UNSUPPORTED;
+    if (!tc_plan(F, P, C, Cout, n_out, k, pl, hT, mt == 4 ? 2 : mt, mt == 4))
+      return VI_ERR_UNSUPPORTED;
   } else {
     if (!tc_plan(F, P, C, Cout, n_out, k, pl, hT, 1)) return VI_ERR_UNSUPPORTED;
     // Two tiles per job when that plan keeps the slab width (a narrower MMA
-    // N costs more than the weight traffic it saves).
+    // N costs more than the weight traffic it saves); on a CTA pair when that
+    // keeps it too and the job is long enough to pay for the pair hand-off.
     TcPlan pl2;
     if (tc_plan(F, P, C, Cout, n_out, k, pl2, hT, TC_MT_DEFAULT) && pl2.NJ >= pl.NJ) pl = pl2;
+    if (k >= 3 && C / TC_KB >= TC_PAIR_MIN_KBLOCKS &&
+        tc_plan(F, P, C, Cout, n_out, k, pl2, hT, TC_MT_DEFAULT, true) && pl2.NJ >= pl.NJ)
+      pl = pl2;
   }
   if (part != VI_PART_ALL) {
     // Frame blocks whose x rows (with the k/2 rows on each side) lie inside
@@ -734,12 +855,25 @@ static int tc_run(const bf16* x, int x_rows, int x_off, const bf16* w, const bf1
     const long long total = (long long)Cout * C * k;
     int blocks = (int)((total + 255) / 256);
     if (blocks > 4 * sm_count()) blocks = 4 * sm_count();
-    temporal_conv_pack_w<<<blocks, 256, 0, stream>>>(w, coef, wpk, b, tab, C, Cout, k, pl.NJ);
+    temporal_conv_pack_w<<<blocks, 256, 0, stream>>>(w, coef, wpk, b, tab, C, Cout, k, pl.NJ,
+                                                     pl.H);
     if (cudaGetLastError() != cudaSuccess) st = VI_ERR_CUDA; else note_launch();
   }
   if (st == VI_OK && fold) {
     temporal_conv_fold_bias<<<Cout, 128, 0, stream>>>(w, b, coef, tab, C, Cout, k);
     if (cudaGetLastError() != cudaSuccess) st = VI_ERR_CUDA; else note_launch();
+  }
+  if (st == VI_OK && pl.H == 2) {
+    // Packed weights as blocks of b_rows rows of 128 bytes: one box = the k
+    // tap blocks of one CTA's half of a (slab, K-block).
+    const uint64_t dims[3] = {64, (uint64_t)pl.b_rows, (uint64_t)Cout * C * k / (64ull * pl.b_rows)};
+    const uint64_t strides[2] = {128, (uint64_t)pl.b_rows * 128};
+    const uint32_t box[3] = {64, (uint32_t)pl.b_rows, (uint32_t)k};
+    if (!encode_tmap(&maps.w, wpk, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE,
+                     CU_TENSOR_MAP_DATA_TYPE_BFLOAT16))
+      st = VI_ERR_CUDA;
+  } else {
+    maps.w = maps.x;                          // not read by the one-SM form
   }
   if (st == VI_OK) {
     const TcArgs a{tab, wpk, err, x_off};
@@ -749,11 +883,12 @@ static int tc_run(const bf16* x, int x_rows, int x_off, const bf16* w, const bf1
   return st;
 }
 
-// mt: tiles per job, 0 for the default plan (1 or 2 force that job form; the
-// tests use it to reach both).
+// mt: 0 for the default plan; 1 or 2 tiles per job on one SM, or 4 (a CTA
+// pair, two tiles per CTA) force that job form (the tests use it to reach
+// every form).
 int temporal_conv_bf16_tc(const bf16* x, const bf16* w, const bf16* b, bf16* y, int F, int P,
                           int C, int k, cudaStream_t stream, const float* coef, int mt) {
-  if (mt < 0 || mt > 2) return VI_ERR_INVALID_ARG;
+  if (mt != 0 && mt != 1 && mt != 2 && mt != 4) return VI_ERR_INVALID_ARG;
   bf16* ys[1] = {y};
   return tc_run(x, F, 0, w, b, ys, 1, F, P, C, C, k, stream, coef, mt);
 }

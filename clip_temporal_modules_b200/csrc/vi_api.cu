@@ -528,13 +528,14 @@ int vi_selftest_wait_timeout(int limit_us, vi_stream_t stream) {
   return VI_OK;
 }
 
-// Test hook, not part of the ABI in vi.h: the bf16 conv with its tiles per
-// job forced to 1 or 2, so that tests reach both job forms of the tensor-core
-// kernel.  Same checks as vi_temporal_conv; shapes the tensor-core path does
-// not take return VI_ERR_UNSUPPORTED.
+// Test hook, not part of the ABI in vi.h: the bf16 conv with its job form
+// forced (tiles = 1 or 2 per job on one SM, or 4: two per CTA of a CTA pair),
+// so that tests reach every form of the tensor-core kernel.  Same checks as
+// vi_temporal_conv; shapes the tensor-core path does not take return
+// VI_ERR_UNSUPPORTED.
 int vitest_temporal_conv_tiles(const void* x, const void* w, const void* b, void* y, int F,
                                int N, int P, int C, int k, int tiles, vi_stream_t stream) {
-  if (tiles != 1 && tiles != 2) return VI_ERR_INVALID_ARG;
+  if (tiles != 1 && tiles != 2 && tiles != 4) return VI_ERR_INVALID_ARG;
   int st = check_clips(F, N, P, C);
   if (st < 0) return st;
   if (k <= 0 || k % 2 == 0 || k / 2 > F / N) return VI_ERR_INVALID_ARG;
@@ -550,11 +551,11 @@ int vitest_temporal_conv_tiles(const void* x, const void* w, const void* b, void
 }
 
 // Test hook, not part of the ABI in vi.h: vi_groupnorm_conv with the conv's
-// tiles per job forced to 1 or 2.
+// job form forced (tiles 1, 2 or 4, as above).
 int vitest_groupnorm_conv_tiles(const void* x, const void* gamma, const void* beta,
                                 const void* w, const void* b, void* y, int F, int N, int P, int C,
                                 int groups, float eps, int k, int tiles, vi_stream_t stream) {
-  if (tiles != 1 && tiles != 2) return VI_ERR_INVALID_ARG;
+  if (tiles != 1 && tiles != 2 && tiles != 4) return VI_ERR_INVALID_ARG;
   return gn_conv_entry(x, gamma, beta, w, b, y, F, N, P, C, groups, eps, k, stream, tiles);
 }
 

@@ -175,7 +175,7 @@ def test_no_global_tuning_state_in_the_abi(L):
     gnconv_t = L.vitest_groupnorm_conv_tiles
     gnconv_t.argtypes = [ctypes.c_void_p] * 6 + [ctypes.c_int] * 5 + [
         ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]
-    for tiles in (0, 3, -1):
+    for tiles in (0, 3, -1, 5):
         assert conv_t(A, B, Cp, D, 64, 4, 2, 64, 3, tiles, None) == INVALID
         assert gnconv_t(A, B, Cp, D, A, B, 64, 4, 2, 64, 8, 1e-5, 3, tiles, None) == INVALID
     assert conv_t(None, None, None, None, 64, 4, 0, 64, 3, 1, None) == OK     # empty

@@ -64,14 +64,15 @@ def test_result_does_not_depend_on_clip_count(cuda_device):
         assert torch.equal(y, ys[0])
 
 
-@pytest.mark.parametrize("tiles", [1, 2])
+@pytest.mark.parametrize("tiles", [1, 2, 4])
 @pytest.mark.parametrize("w", [W("bf16_F48_C64_odd_tiles", "bf16", 48, 3, 5, 64),
                                W("bf16_F200_C320_ragged", "bf16", 200, 8, 3, 320),
                                W("bf16_F24_C320_k1", "bf16", 24, 3, 3, 320, k=1)],
                          ids=lambda w: w.name)
 def test_one_and_two_tiles_per_job(cuda_device, w, tiles):
-    """Both job forms of the tensor-core conv (one 128-frame tile per job, or
-    two sharing every weight stage; odd tile counts leave a zero tile)."""
+    """Every job form of the tensor-core conv: one 128-frame tile per job, two
+    sharing every weight stage, or a CTA pair with two tiles per CTA (M = 256,
+    each CTA holding half the weight rows); odd tile counts leave zero tiles."""
     from clip_temporal_modules_b200._binding import conv_forced_tiles
     x, wt, b = (synth.make(w, t) for t in ("conv_x", "conv_w", "conv_b"))
     dx, dw, db = (to_device(a, w.dtype) for a in (x, wt, b))

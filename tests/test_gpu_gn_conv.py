@@ -86,7 +86,7 @@ def test_matches_groupnorm_then_conv_calls(cuda_device):
     assert np.all(np.abs(f - t) <= 2 * tolerance(w.dtype, ref, "gn"))
 
 
-@pytest.mark.parametrize("tiles", [1, 2])
+@pytest.mark.parametrize("tiles", [1, 2, 4])
 @pytest.mark.parametrize("w", [W("gnconv_F48_C64_G8_odd_tiles", 48, 3, 5, 64, 8),
                                W("gnconv_F200_C320_G32_ragged", 200, 8, 3, 320, 32)],
                          ids=lambda w: w.name)
