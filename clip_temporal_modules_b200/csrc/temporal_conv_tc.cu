@@ -361,9 +361,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 
   const int halo = k / 2;
   const int cb_rot = (int)(cid % pl.n_cb);          // the same K-block order in both CTAs
-  // Equal x and w rings (the two-tile form): one barrier pair per stage covers
-  // both, so a K-block costs one wait and one commit.
-  const bool uni = pl.sa == pl.sb;
+  // Two tiles per job (and every pair plan) use equal x and w rings: one
+  // barrier pair per stage covers both, so a K-block costs one wait and one
+  // commit.  One tile per job keeps separate rings.
+  constexpr bool UNI = MT == 2;
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     // Lane 0 takes the ring waits and posts the expected bytes; the stage's
@@ -394,16 +395,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         // Stage `is` holds K-block (is + cb_rot) mod n_cb of the job.
         const int cb = (is + cb_rot) % pl.n_cb;
         const uint32_t a_bar = PAIR ? lead_a_full + 8 * sa : a_full + 8 * sa;
-        const uint32_t b_bar = uni ? a_bar : b_full + 8 * sbi;   // shared stage: one barrier
+        const uint32_t b_bar = UNI ? a_bar : b_full + 8 * sbi;   // shared stage: one barrier
         bool go = true;
         if (lane == 0) {
           go = !a_used || tc_wait<PAIR>(a_empty + 8 * sa, (uint32_t)(pa ^ 1), args.err,
                                         VI_DEV_ERR_TMA_TIMEOUT);
           if (go) {
             if constexpr (PAIR) mbar_arrive_expect_tx_cluster(a_bar, a_bytes + (uint32_t)pl.b_kb);
-            else mbar_arrive_expect_tx(a_bar, a_bytes + (uni ? (uint32_t)pl.b_kb : 0u));
+            else mbar_arrive_expect_tx(a_bar, a_bytes + (UNI ? (uint32_t)pl.b_kb : 0u));
           }
-          if (go && !uni) {
+          if (go && !UNI) {
             go = !b_used || tc_wait<PAIR>(b_empty + 8 * sbi, (uint32_t)(pb ^ 1), args.err,
                                               VI_DEV_ERR_TMA_TIMEOUT);
             if (go) mbar_arrive_expect_tx(b_bar, (uint32_t)pl.b_kb);
@@ -449,41 +450,45 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         // This job's accumulator slots and the parity of their last release.
         int js[MT], jp[MT];
         bool ju[MT];
-        uint32_t dt[MT];
 #pragma unroll
         for (int m = 0; m < MT; ++m) {
           js[m] = slot; jp[m] = pslot; ju[m] = slot_used;
-          dt[m] = tmem_base + (uint32_t)(slot * pl.NJ);
           if (++slot == pl.n_acc) { slot = 0; pslot ^= 1; slot_used = true; }
         }
         for (int is = 0; is < pl.n_stage && ok; ++is) {
-          const bool last_stage = is == pl.n_stage - 1;
-          if (!tc_wait<PAIR>(a_full + 8 * sa, (uint32_t)pa, args.err, VI_DEV_ERR_TMA_TIMEOUT) ||
-              (!uni &&
-               !tc_wait<PAIR>(b_full + 8 * sbi, (uint32_t)pb, args.err, VI_DEV_ERR_TMA_TIMEOUT))) {
+          if (!tc_wait<PAIR>(a_full + 8 * sa, (uint32_t)pa, args.err, VI_DEV_ERR_TMA_TIMEOUT)) {
             ok = false;
             break;
           }
+          if constexpr (!UNI) {
+            if (!tc_wait<PAIR>(b_full + 8 * sbi, (uint32_t)pb, args.err, VI_DEV_ERR_TMA_TIMEOUT)) {
+              ok = false;
+              break;
+            }
+          }
           tc_fence_after();
           const uint64_t ad_stage = ad_base + (uint64_t)(sa * a_st16);
-          const uint64_t bd_stage = bd_base + (uint64_t)(sbi * b_st16);
+          const uint64_t bd_stage = bd_base + (uint64_t)((UNI ? sa : sbi) * b_st16);
 #pragma unroll
           for (int m = 0; m < MT; ++m) {
             if (is == 0) {
-              // The slot must have been drained by the epilogue of its last job.
-              if (ju[m] && !tc_wait<PAIR>(acc_empty + 8 * js[m], (uint32_t)(jp[m] ^ 1),
-                                          args.err, VI_DEV_ERR_MMA_TIMEOUT)) { ok = false; break; }
+              // The slot must have been drained by the epilogue of its last tile.
+              if (ju[m] && !tc_wait<PAIR>(acc_empty + 8 * js[m], (uint32_t)(jp[m] ^ 1), args.err,
+                                          VI_DEV_ERR_MMA_TIMEOUT)) { ok = false; break; }
               tc_fence_after();
             }
-            tc_issue_taps<KT, PAIR>(dt[m], ad_stage + (uint64_t)(m * at16), bd_stage, bt16, bk16,
-                                    idesc, is > 0 ? 1u : 0u, k);
-            if (last_stage) tc_commit<PAIR>(acc_full + 8 * js[m]);   // accumulator ready
+            tc_issue_taps<KT, PAIR>(tmem_base + (uint32_t)(js[m] * pl.NJ),
+                                    ad_stage + (uint64_t)(m * at16), bd_stage, bt16, bk16, idesc,
+                                    is > 0 ? 1u : 0u, k);
+            if (is == pl.n_stage - 1) tc_commit<PAIR>(acc_full + 8 * js[m]);   // accumulator ready
           }
           if (!ok) break;
-          if (!uni) tc_commit<PAIR>(b_empty + 8 * sbi);   // frees the w stage when these MMAs finish
-          tc_commit<PAIR>(a_empty + 8 * sa);              // frees the x stage (and the w stage if shared)
-          if (++sbi == pl.sb) { sbi = 0; pb ^= 1; }
+          if constexpr (!UNI) tc_commit<PAIR>(b_empty + 8 * sbi);   // frees the w stage
+          tc_commit<PAIR>(a_empty + 8 * sa);   // frees the x stage (and the w stage if shared)
           if (++sa == pl.sa) { sa = 0; pa ^= 1; }
+          if constexpr (!UNI) {
+            if (++sbi == pl.sb) { sbi = 0; pb ^= 1; }
+          }
         }
       }
       // Every MMA this thread issued must finish before TMEM is released.
