@@ -30,27 +30,28 @@
 //
 // The MMA issue loop is unrolled at compile time over the taps (k = 1 and 3),
 // the tiles of a job and the four K steps of a K-block, with every descriptor
-// offset an immediate: a single thread then issues an M = 128, N = 160 MMA
-// faster than the tensor core retires it (80 cycles), which a loop with
-// run-time trip counts and per-MMA address arithmetic did not (about 150).
+// offset an immediate, and the ring layout (one shared x/w ring for two tiles
+// per job) is known at compile time: the tensor pipe queues only about three
+// MMAs ahead of the issuing thread, so run-time tests and address arithmetic
+// between MMAs show up directly as idle pipe cycles.
 //
 // TMEM holds a ring of MT + 1 (at least 2) accumulators of NJ columns: the
-// epilogue warps (TMEM -> registers, + bias, -> bf16 -> global) drain the
-// oldest while the MMAs of the next tiles fill the others.  Every CTA walks
-// the K-blocks of a job starting at its own offset, so the CTAs do not all
-// stream the same weight block at once.
+// epilogue warps drain the oldest while the MMAs of the next tiles fill the
+// others.  Every CTA walks the K-blocks of a job starting at its own offset,
+// so the CTAs do not all stream the same weight block at once.
 //
-// The epilogue writes y through shared memory: per 32-channel chunk of an
-// accumulator the four warps write 128 rows x 64 bytes (64-byte swizzle, so
-// the 16-byte writes of eight consecutive rows hit distinct banks) into one of
-// two staging buffers, and one thread stores the chunk with a TMA tensor
-// store, which also drops the rows past the last frame.
+// Epilogue: each warp owns a TMEM lane quadrant (32 frames of the tile),
+// loads its whole row of the accumulator into registers and releases it at
+// once, then adds the bias, packs to bf16 and writes 64-channel chunks (32
+// where the plan is narrow) into its own two 128-byte-swizzled staging
+// buffers; its lane 0 stores each chunk with a TMA tensor store, which also
+// drops the rows past the last frame.
 //
 // Warp roles (192 threads, one CTA per SM, persistent over jobs):
-//   warp 0      TMA producer (one elected thread)
+//   warp 0      TMA producer: lane 0 takes the ring waits, lane m loads tile
+//               m's x box and lane MT the stage's weights
 //   warp 1      TMEM allocator + MMA issuer (one thread)
 //   warps 2..5  epilogue; warp w reads TMEM lanes 32*(w%4) .. +31
-//   warps 6..13 (GroupNorm fusion only) normalise the landed x tiles
 #include <mutex>
 
 #include "ptx.cuh"
