@@ -622,8 +622,13 @@ def clip_parallel_emulated(w, d, stream, world=8, reps=5):
         for sh in shards:
             temporal_conv_shard(sh["x"], d["conv_w"], d["conv_b"], sh["y"])
 
+    # Each shard's statistics land in its slot of the gathered [W][groups][2]
+    # tensor (what the all-gather delivers on every GPU).
+    stats = torch.empty((world, w.groups, 2), dtype=torch.float64, device=d["q"].device)
+
     def gn():
-        stats = torch.stack([groupnorm_shard_stats(sh["g"], groups=w.groups) for sh in shards])
+        for i, sh in enumerate(shards):
+            groupnorm_shard_stats(sh["g"], groups=w.groups, out=stats[i])
         for sh in shards:
             groupnorm_shard_apply(sh["g"], stats, d["gn_gamma"], d["gn_beta"], sh["z"], eps=w.eps)
 

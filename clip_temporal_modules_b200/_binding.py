@@ -256,12 +256,19 @@ def temporal_conv_shard(x_ext, w, b, out=None, *, part: int = 0, stream=None):
     return out
 
 
-def groupnorm_shard_stats(x, *, groups: int, stream=None):
-    """Per-group (mean, var) of one shard's rows: a [groups][2] float64 CUDA tensor."""
+def groupnorm_shard_stats(x, *, groups: int, out=None, stream=None):
+    """Per-group (mean, var) of one shard's rows: a [groups][2] float64 CUDA tensor
+    (`out` if given, e.g. this shard's slot of a gathered [W][groups][2] tensor)."""
     import torch
     _dev(x)
     P, F_loc, C = x.shape
-    stats = torch.empty((groups, 2), dtype=torch.float64, device=x.device)
+    if out is None:
+        stats = torch.empty((groups, 2), dtype=torch.float64, device=x.device)
+    else:
+        if not out.is_cuda or out.dtype != torch.float64 or tuple(out.shape) != (groups, 2) \
+                or not out.is_contiguous():
+            raise ValueError("out: expected a contiguous [groups][2] float64 CUDA tensor")
+        stats = out
     _check("vi_groupnorm_shard_stats", lib().vi_groupnorm_shard_stats(
         x.data_ptr(), F_loc, P, C, groups, stats.data_ptr(), _stream_ptr(stream)))
     return stats

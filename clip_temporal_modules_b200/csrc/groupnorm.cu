@@ -41,6 +41,45 @@ struct GnScratch {
   double* stats;           // [groups][2]: mu_g, var_g (kept for inspection)
 };
 
+// Where the apply pass takes its per-channel coefficients (m_c, a_c, beta_c):
+// from coef, [C][4] floats written by the statistics pass, or (shard_stats
+// != null) from W shards' per-group (mean, var) records, merged by each
+// thread for its own channels exactly as gn_merge_coef does: mean = average
+// of the means, var = average of (var_w + (mean_w - mean)^2).
+template <typename T>
+struct GnCoefSrc {
+  const float* coef;
+  const double* shard_stats;   // [W][groups][2]
+  int W, groups, cg;
+  const T* gamma;
+  const T* beta;
+  float eps;
+};
+
+template <typename T>
+__device__ __forceinline__ void gn_coef_of(const GnCoefSrc<T>& src, int c, float& m, float& a,
+                                           float& b) {
+  if (!src.shard_stats) {
+    m = src.coef[4 * c];
+    a = src.coef[4 * c + 1];
+    b = src.coef[4 * c + 2];
+    return;
+  }
+  const int g = c / src.cg;
+  double mean = 0.0;
+  for (int w = 0; w < src.W; ++w) mean += src.shard_stats[((size_t)w * src.groups + g) * 2];
+  mean /= src.W;
+  double var = 0.0;
+  for (int w = 0; w < src.W; ++w) {
+    const double dm = src.shard_stats[((size_t)w * src.groups + g) * 2] - mean;
+    var += src.shard_stats[((size_t)w * src.groups + g) * 2 + 1] + dm * dm;
+  }
+  var /= src.W;
+  m = (float)mean;
+  a = (float)((double)to_f32(src.gamma[c]) / sqrt(var + (double)src.eps));
+  b = to_f32(src.beta[c]);
+}
+
 // Merge of all partial sums by the block that finishes last.  nparts partial
 // records per group; red is the caller's shared buffer of GN_MAX_GROUPS rows.
 template <typename T>
@@ -259,7 +298,7 @@ __global__ void __launch_bounds__(1024, 1) gn_stats_ring(const T* __restrict__ x
 template <typename T>
 __global__ void __launch_bounds__(1024, 1) gn_apply_ring(const T* __restrict__ x,
                                                          T* __restrict__ y, GnRing rg,
-                                                         const float* __restrict__ coef,
+                                                         const GnCoefSrc<T> csrc,
                                                          unsigned int* err_word) {
   constexpr int V = VecOf<T>::n;
   extern __shared__ __align__(128) uint8_t smem[];
@@ -316,9 +355,8 @@ __global__ void __launch_bounds__(1024, 1) gn_apply_ring(const T* __restrict__ x
     float m[V], a[V], b[V];
 #pragma unroll
     for (int e = 0; e < V; ++e) {
-      m[e] = active ? coef[4 * (c0 + e)] : 0.f;
-      a[e] = active ? coef[4 * (c0 + e) + 1] : 0.f;
-      b[e] = active ? coef[4 * (c0 + e) + 2] : 0.f;
+      m[e] = a[e] = b[e] = 0.f;
+      if (active) gn_coef_of<T>(csrc, c0 + e, m[e], a[e], b[e]);
     }
     int kl = 0;
     for (int64_t c = blockIdx.x; c < rg.nchunks; c += gridDim.x, ++kl) {
@@ -484,7 +522,8 @@ static int gn_launch(const T* x, const T* gamma, const T* beta, T* y, int64_t ro
     gn_stats_ring<T><<<pl.blocks, pl.threads, pl.smem, stream>>>(x, pl.rg, cg, groups, s, gamma,
                                                                  beta, eps, err);
     VI_LAUNCHED();
-    gn_apply_ring<T><<<pl.blocks, pl.threads, pl.smem, stream>>>(x, y, pl.rg, s.coef, err);
+    const GnCoefSrc<T> csrc{s.coef, nullptr, 0, groups, cg, nullptr, nullptr, 0.f};
+    gn_apply_ring<T><<<pl.blocks, pl.threads, pl.smem, stream>>>(x, y, pl.rg, csrc, err);
     VI_LAUNCHED();
   } else {
     gn_stats_scalar<T><<<dim3(groups, pl.parts), 256, 0, stream>>>(x, rows, C, cg, groups, s,
@@ -505,9 +544,11 @@ static int gn_launch(const T* x, const T* gamma, const T* beta, T* y, int64_t ro
 // address, [C][4] floats (m_c, a_c, beta_c, 0).
 template <typename T>
 int gn_stats_launch(const T* x, const T* gamma, const T* beta, int64_t rows, int C, int groups,
-                    float eps, void* scratch, cudaStream_t stream, const float** coef) {
+                    float eps, void* scratch, cudaStream_t stream, const float** coef,
+                    double* stats_out) {
   const GnPlan pl = gn_plan<T>(rows, C, groups);
-  const GnScratch s = gn_carve(scratch, groups, C);
+  GnScratch s = gn_carve(scratch, groups, C);
+  if (stats_out) s.stats = stats_out;     // the last block writes (mean, var) there
   const int cg = C / groups;
   if (pl.ring) {
     unsigned int* err = device_error_word();
@@ -531,7 +572,7 @@ size_t gn_scratch_size_bf16(int64_t rows, int C, int groups) {
 }
 
 template int gn_stats_launch<bf16>(const bf16*, const bf16*, const bf16*, int64_t, int, int, float,
-                                   void*, cudaStream_t, const float**);
+                                   void*, cudaStream_t, const float**, double*);
 
 // ---------------------------------------------------------------------------
 // A video cut along frames over several GPUs (clip parallelism): each shard
@@ -539,7 +580,8 @@ template int gn_stats_launch<bf16>(const bf16*, const bf16*, const bf16*, int64_
 // (a7), and each shard normalises its rows with the merged statistics (a8).
 
 // a6 on one shard: per-group (mean, var) of the shard's rows, fp64, into
-// stats [groups][2] (device memory).
+// stats [groups][2] (device memory), written by the statistics pass's last
+// block itself.
 template <typename T>
 int gn_shard_stats(const T* x, int64_t rows, int C, int groups, double* stats,
                    cudaStream_t stream) {
@@ -549,13 +591,8 @@ int gn_shard_stats(const T* x, int64_t rows, int C, int groups, double* stats,
   const float* coef = nullptr;
   int st = cudaMemsetAsync(scratch, 0, 64, stream) == cudaSuccess ? VI_OK : VI_ERR_CUDA;
   if (st == VI_OK)
-    st = gn_stats_launch<T>(x, nullptr, nullptr, rows, C, groups, 1e-5f, scratch, stream, &coef);
-  if (st == VI_OK) {
-    const GnScratch s = gn_carve(scratch, groups, C);
-    if (cudaMemcpyAsync(stats, s.stats, sizeof(double) * 2 * groups, cudaMemcpyDeviceToDevice,
-                        stream) != cudaSuccess)
-      st = VI_ERR_CUDA;
-  }
+    st = gn_stats_launch<T>(x, nullptr, nullptr, rows, C, groups, 1e-5f, scratch, stream, &coef,
+                            stats);
   if (scratch_free(scratch, stream) != cudaSuccess && st == VI_OK) st = VI_ERR_CUDA;
   return st;
 }
@@ -589,10 +626,22 @@ __global__ void gn_merge_coef(const double* __restrict__ shard_stats, int W, int
 }
 
 // a7 + a8 on one shard: merged statistics, then y = (x - m_c) a_c + beta_c.
+// On the ring path every apply thread merges the shards' records for its own
+// channels (one launch); the scalar path merges in a kernel of its own.
 template <typename T>
 int gn_shard_apply(const T* x, const double* shard_stats, int W, const T* gamma, const T* beta,
                    T* y, int64_t rows, int C, int groups, float eps, cudaStream_t stream) {
   const GnPlan pl = gn_plan<T>(rows, C, groups);
+  if (pl.ring) {
+    unsigned int* err = device_error_word();
+    if (!err) return VI_ERR_CUDA;
+    VI_CUDA_TRY(cudaFuncSetAttribute(gn_apply_ring<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)pl.smem));
+    const GnCoefSrc<T> csrc{nullptr, shard_stats, W, groups, C / groups, gamma, beta, eps};
+    gn_apply_ring<T><<<pl.blocks, pl.threads, pl.smem, stream>>>(x, y, pl.rg, csrc, err);
+    VI_LAUNCHED();
+    return VI_OK;
+  }
   float* coef = nullptr;
   VI_CUDA_TRY(scratch_alloc(reinterpret_cast<void**>(&coef), sizeof(float) * 4 * (size_t)C,
                             stream));
@@ -600,17 +649,7 @@ int gn_shard_apply(const T* x, const double* shard_stats, int W, const T* gamma,
   gn_merge_coef<T><<<(C + 255) / 256, 256, 0, stream>>>(shard_stats, W, groups, C, gamma, beta,
                                                         eps, coef);
   if (cudaGetLastError() != cudaSuccess) st = VI_ERR_CUDA; else note_launch();
-  if (st == VI_OK && pl.ring) {
-    unsigned int* err = device_error_word();
-    if (!err) st = VI_ERR_CUDA;
-    else if (cudaFuncSetAttribute(gn_apply_ring<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)pl.smem) != cudaSuccess)
-      st = VI_ERR_CUDA;
-    if (st == VI_OK) {
-      gn_apply_ring<T><<<pl.blocks, pl.threads, pl.smem, stream>>>(x, y, pl.rg, coef, err);
-      if (cudaGetLastError() != cudaSuccess) st = VI_ERR_CUDA; else note_launch();
-    }
-  } else if (st == VI_OK) {
+  if (st == VI_OK) {
     const int64_t n = rows * C;
     int64_t blocks = (n + 255) / 256;
     if (blocks > (int64_t)sm_count() * 16) blocks = (int64_t)sm_count() * 16;

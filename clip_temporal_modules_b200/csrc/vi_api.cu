@@ -57,7 +57,7 @@ bool temporal_conv_tc_norm_ok(int F, int P, int C, int k);
 bool linear_tc_ok(int F, int P, int C, int Cout, int n_out);
 template <typename T>
 int gn_stats_launch(const T*, const T*, const T*, int64_t, int, int, float, void*, cudaStream_t,
-                    const float**);
+                    const float**, double* stats_out = nullptr);
 size_t gn_scratch_size_bf16(int64_t rows, int C, int groups);
 template <typename T>
 int groupnorm_global(const T*, const T*, const T*, T*, int64_t, int, int, float, cudaStream_t);
