@@ -115,6 +115,47 @@ def test_sharded_groupnorm_matches_one_gpu_and_oracle(cuda_device, world):
     assert_close(got, ref, w.dtype, "gn", "sharded GroupNorm")
 
 
+@pytest.mark.parametrize("C,groups", [(320, 32), (64, 32)])
+def test_shard_stats_into_gathered_slots(cuda_device, C, groups):
+    """Each shard's statistics written into its slot of one [W][groups][2]
+    tensor (what an all-gather delivers) equal the separately returned ones
+    bit for bit, and the apply pass on them matches the one-GPU call.  C=320
+    takes the ring path, whose apply threads merge the shards' records
+    themselves; C=64 with 32 groups (2 channels per group) the scalar path,
+    which merges in a kernel of its own."""
+    world = 4
+    w = synth.Workload("cp_gn_slots", "bf16", F=256, N=16, P=5, C=C, heads=C // 64, d=64,
+                       groups=groups)
+    x, g, bt = (synth.make(w, t) for t in ("gn_x", "gn_gamma", "gn_beta"))
+    dx, dg, dbt = (to_device(a, w.dtype) for a in (x, g, bt))
+    whole = vi.groupnorm_global(dx, dg, dbt, N=w.N, groups=w.groups)
+    lays = [ShardLayout(w.F, w.N, world, r) for r in range(world)]
+    shards = [dx[:, l.f0:l.f0 + l.F_loc].contiguous() for l in lays]
+    gathered = torch.full((world, w.groups, 2), float("nan"), dtype=torch.float64,
+                          device=dx.device)
+    for i, sh in enumerate(shards):
+        groupnorm_shard_stats(sh, groups=w.groups, out=gathered[i])
+    single = torch.stack([groupnorm_shard_stats(sh, groups=w.groups) for sh in shards])
+    parts = [groupnorm_shard_apply(sh, gathered, dg, dbt) for sh in shards]
+    torch.cuda.synchronize()
+    vi.take_device_errors()
+    assert torch.equal(gathered, single)
+    got = from_device(torch.cat(parts, dim=1))
+    ref, _, _ = oracle.groupnorm_global(x, g, bt, w.F, w.N, w.groups, w.eps)
+    assert np.max(np.abs(got - from_device(whole))) <= 2e-2
+    assert_close(got, ref, w.dtype, "gn", "sharded GroupNorm from gathered slots")
+
+
+def test_shard_stats_out_slot_is_checked(cuda_device):
+    x = torch.zeros((2, 16, 64), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(ValueError):
+        groupnorm_shard_stats(x, groups=32, out=torch.empty((32, 3), dtype=torch.float64,
+                                                            device="cuda"))
+    with pytest.raises(ValueError):
+        groupnorm_shard_stats(x, groups=32, out=torch.empty((32, 2), dtype=torch.float32,
+                                                            device="cuda"))
+
+
 def _single_rank_run(t, w, stream=None):
     cp = ClipParallel(w.F, w.N, heads=w.heads, groups=w.groups)
     k = w.k // 2
