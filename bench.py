@@ -399,6 +399,7 @@ def run_ours(args):
     if remeasured is not None:
         result["remeasured"] = remeasured
     result["attn_ablations"] = attn_ablations(w, d, out, y, z, stream)
+    result["attn_generic_path"] = attn_generic_path(w, d, out, stream)
     result["groupnorm_conv_fused"] = fused_gn_conv(w, d, y, z, stream)
     result["temporal_attention_module"] = attention_module(w, d, out, y, z, stream)
     if w.dtype == "bf16" and w.F % 8 == 0 and w.N % 8 == 0:
@@ -526,6 +527,33 @@ def attn_ablations(w, d, out, y, z, stream, reps=10):
             res[name] = _ablation(w, d, out, rest, stream, reps, S, a, b_, g)
     res["clocks"] = clocks.summary()
     return res
+
+
+def attn_generic_path(w, d, out, stream, reps=2):
+    """The same attention with n_pre = n_post = 16, outside the tensor-core
+    fast path (which takes n_pre, n_post <= 8, n_global <= 16, L = 16,
+    d = 64): one warp per query frame on CUDA cores.  Reported so that the
+    step's cost off the fast path is visible, not as a tuned figure."""
+    import torch
+
+    import clip_temporal_modules_b200 as vi
+    n_pre = n_post = min(16, w.F // w.N)
+
+    def attn():
+        vi.dual_attn(d["q"], d["k"], d["v"], out, N=w.N, heads=w.heads, n_pre=n_pre,
+                     n_post=n_post, n_global=w.n_global)
+    attn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        attn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    S = w.P * w.F * w.C * w.elem_bytes
+    return {"n_pre": n_pre, "n_post": n_post, "n_global": w.n_global, "ms": round(ms, 4),
+            "GB/s": round(4 * S / (ms / 1e3) / 1e9, 1), "path": "dual_attn_generic (CUDA cores)"}
 
 
 def _ablation(w, d, out, rest, stream, reps, S, a, b_, g):
