@@ -41,8 +41,9 @@
 // so the CTAs do not all stream the same weight block at once.
 //
 // Epilogue: each warp owns a TMEM lane quadrant (32 frames of the tile),
-// loads its whole row of the accumulator into registers and releases it at
-// once, then adds the bias, packs to bf16 and writes 64-channel chunks (32
+// brings its row of the accumulator into registers 32 columns at a time,
+// adds the bias and packs each group to bf16 pairs (the whole row then takes
+// 80 registers), releases the accumulator, and writes 64-channel chunks (32
 // where the plan is narrow) into its own two 128-byte-swizzled staging
 // buffers; its lane 0 stores each chunk with a TMA tensor store, which also
 // drops the rows past the last frame.
@@ -149,7 +150,7 @@ static bool tc_plan(int F, int P, int C, int Cout, int n_out, int k, TcPlan& pl,
     if (cpo % nj != 0 || n_acc * nj > TC_TMEM_COLS || (nj / H) % 8 != 0) continue;
     const int b_stage = k * (nj / H) * 128;
     for (int wide = 1; wide >= 0; --wide) {
-      const int fixed = base + 4 * 2 * (wide ? TC_OUT_BUF : TC_OUT_BUF / 2);   // output staging
+      const int fixed = base + TC_EPI_WARPS * 2 * (wide ? TC_OUT_BUF : TC_OUT_BUF / 2);   // output staging
       int sa, sb;
       if (mt == 2) {
         int n = (TC_SMEM_LIMIT - fixed) / (a_stage + b_stage);
@@ -252,38 +253,30 @@ __device__ __forceinline__ void tc_commit(uint32_t bar) {
   else umma_commit(bar);
 }
 
-// Epilogue of one chunk of a tile row: + bias, -> bf16, into the staging
-// buffer.  w64: 64 channels (lo, hi) as a 128-byte row, 16-byte chunk i at
-// i ^ (lane & 7) (128-byte swizzle); else 32 channels (lo) as a 64-byte row,
-// chunk i at i ^ ((lane >> 1) & 3) (64-byte swizzle).  Either way the eight
-// rows a quarter-warp writes at once hit distinct banks.
-__device__ __forceinline__ void epi_stage_chunk(uint32_t stage, int lane, const uint32_t (&lo)[32],
-                                                const uint32_t (&hi)[32], const float* bs, bool w64) {
-  uint32_t pk[16];
-#pragma unroll
-  for (int i = 0; i < 16; ++i)
-    pk[i] = pack2_bf16(__uint_as_float(lo[2 * i]) + bs[2 * i],
-                       __uint_as_float(lo[2 * i + 1]) + bs[2 * i + 1]);
+// Epilogue of one chunk of a tile row, already + bias and packed to bf16
+// pairs, into the staging buffer.  w64: 64 channels (lo, hi) as a 128-byte
+// row, 16-byte chunk i at i ^ (lane & 7) (128-byte swizzle); else 32
+// channels (lo) as a 64-byte row, chunk i at i ^ ((lane >> 1) & 3) (64-byte
+// swizzle).  Either way the eight rows a quarter-warp writes at once hit
+// distinct banks.
+__device__ __forceinline__ void epi_stage_chunk(uint32_t stage, int lane, const uint32_t (&lo)[16],
+                                                const uint32_t (&hi)[16], bool w64) {
   if (w64) {
     const uint32_t row = stage + (uint32_t)lane * 128u, sw = (uint32_t)(lane & 7);
 #pragma unroll
     for (int i = 0; i < 4; ++i)
       sts128(row + (((uint32_t)i ^ sw) << 4),
-             make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]));
-#pragma unroll
-    for (int i = 0; i < 16; ++i)
-      pk[i] = pack2_bf16(__uint_as_float(hi[2 * i]) + bs[32 + 2 * i],
-                         __uint_as_float(hi[2 * i + 1]) + bs[33 + 2 * i]);
+             make_uint4(lo[4 * i], lo[4 * i + 1], lo[4 * i + 2], lo[4 * i + 3]));
 #pragma unroll
     for (int i = 0; i < 4; ++i)
       sts128(row + (((uint32_t)(4 + i) ^ sw) << 4),
-             make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]));
+             make_uint4(hi[4 * i], hi[4 * i + 1], hi[4 * i + 2], hi[4 * i + 3]));
   } else {
     const uint32_t row = stage + (uint32_t)lane * 64u, sw = (uint32_t)((lane >> 1) & 3);
 #pragma unroll
     for (int i = 0; i < 4; ++i)
       sts128(row + (((uint32_t)i ^ sw) << 4),
-             make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]));
+             make_uint4(lo[4 * i], lo[4 * i + 1], lo[4 * i + 2], lo[4 * i + 3]));
   }
 }
 
@@ -315,7 +308,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   const uint32_t sB = sA + pl.sa * pl.a_stage;
   const uint32_t sOut = sB + pl.sb * pl.b_stage;       // output staging, 1024-aligned
   const uint32_t out_buf = pl.wide ? TC_OUT_BUF : TC_OUT_BUF / 2;   // bytes of one staging buffer
-  const uint32_t sBar = sOut + 4 * 2 * out_buf;
+  const uint32_t sBar = sOut + TC_EPI_WARPS * 2 * out_buf;
   // barrier block: a_full[SA] a_empty[SA] b_full[SB] b_empty[SB] acc_full[4] acc_empty[4] drain tmem_slot
   const uint32_t a_full = sBar, a_empty = a_full + 8 * TC_SA_MAX;
   const uint32_t b_full = a_empty + 8 * TC_SA_MAX, b_empty = b_full + 8 * TC_SB_MAX;
@@ -532,16 +525,33 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         // (read through L1: every warp of every CTA reads the same few KB)
         const float* bs = args.btab + (lo * (pl.hT + 1) + hi) * pl.Cout + slab * pl.NJ;
         const uint32_t taddr = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * pl.NJ);
-        // The whole row of the tile (<= 160 columns) into registers first,
-        // so that the accumulator goes back to the MMA at once and the
-        // packing and stores overlap the next tiles' MMAs.
-        uint32_t r[TC_NJ_MAX / 32][32];
+        // The tile row group by group (32 columns): TMEM -> registers, + bias,
+        // -> bf16 pairs (16 registers a group, so that the whole row fits
+        // beside the other roles' state).  The accumulator goes back to the
+        // MMA after the last group; the staging and stores of the tile
+        // overlap the next tiles' MMAs.  Loops unrolled: registers indexed at
+        // compile time only.
+        uint32_t pk[TC_NJ_MAX / 32][16];
 #pragma unroll
-        for (int c = 0; c < TC_NJ_MAX / 32; ++c)
-          if (32 * c < pl.NJ) tmem_ld32(taddr + 32u * c, r[c]);
+        for (int g = 0; g < TC_NJ_MAX / 32; ++g) {
+          if (32 * g >= pl.NJ) break;
+          uint32_t r[32];
+          tmem_ld32(taddr + 32u * g, r);
+          // (the bias tables are 128-byte aligned per 32 channels; read
+          // through L1: every warp of every CTA reads the same few KB)
+          const float4* b4 = reinterpret_cast<const float4*>(bs + 32 * g);
+          float4 bv[8];
 #pragma unroll
-        for (int c = 0; c < TC_NJ_MAX / 32; ++c)
-          if (32 * c < pl.NJ) tmem_wait_ld_dep(r[c]);
+          for (int i = 0; i < 8; ++i) bv[i] = __ldg(b4 + i);
+          tmem_wait_ld_dep(r);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            pk[g][2 * i] = pack2_bf16(__uint_as_float(r[4 * i]) + bv[i].x,
+                                      __uint_as_float(r[4 * i + 1]) + bv[i].y);
+            pk[g][2 * i + 1] = pack2_bf16(__uint_as_float(r[4 * i + 2]) + bv[i].z,
+                                          __uint_as_float(r[4 * i + 3]) + bv[i].w);
+          }
+        }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) {
@@ -561,7 +571,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           if (lane == 0) bulk_wait_read_le1();   // the store that last read this buffer is done
           __syncwarp();
           if (tile_ok)
-            epi_stage_chunk(stage, lane, r[g], r[g + 1 < TC_NJ_MAX / 32 ? g + 1 : g], bs + 32 * g, w64);
+            epi_stage_chunk(stage, lane, pk[g], pk[g + 1 < TC_NJ_MAX / 32 ? g + 1 : g], w64);
           fence_proxy_async_smem();           // the writes are visible to the TMA store
           __syncwarp();
           if (lane == 0 && tile_ok) {
