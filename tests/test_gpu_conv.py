@@ -37,6 +37,8 @@ SMALL = [
     W("bf16_F48_C64", "bf16", 48, 3, 5, 64),
     W("bf16_F200_C320_ragged", "bf16", 200, 8, 3, 320),      # frame tail of 72 rows
     W("bf16_F256_C640", "bf16", 256, 16, 2, 640),
+    W("bf16_F72_C192_slab96", "bf16", 72, 3, 3, 192),      # 96-channel slabs: 64 + 32 chunks
+    W("bf16_F64_C256_slab128", "bf16", 64, 4, 2, 256),     # 128-channel slabs
     W("bf16_F40_C136_k5", "bf16", 40, 5, 3, 136, k=5),       # channel tail, wider halo
     W("bf16_F24_C64_k1", "bf16", 24, 3, 2, 64, k=1),
     W("f32_F40_C36_k5", "f32", 40, 4, 2, 36, k=5),
