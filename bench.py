@@ -400,6 +400,7 @@ def run_ours(args):
         result["remeasured"] = remeasured
     result["attn_ablations"] = attn_ablations(w, d, out, y, z, stream)
     result["attn_generic_path"] = attn_generic_path(w, d, out, stream)
+    result["attn_halo16"] = attn_halo16(w, d, out, stream)
     result["groupnorm_conv_fused"] = fused_gn_conv(w, d, y, z, stream)
     result["temporal_attention_module"] = attention_module(w, d, out, y, z, stream)
     if w.dtype == "bf16" and w.F % 8 == 0 and w.N % 8 == 0:
@@ -530,18 +531,18 @@ def attn_ablations(w, d, out, y, z, stream, reps=10):
 
 
 def attn_generic_path(w, d, out, stream, reps=2):
-    """The same attention with n_pre = n_post = 16, outside the tensor-core
-    fast path (which takes n_pre, n_post <= 8, n_global <= 16, L = 16,
-    d = 64): one warp per query frame on CUDA cores.  Reported so that the
-    step's cost off the fast path is visible, not as a tuned figure."""
+    """The same attention with n_global = 32, outside the tensor-core fast
+    path (which takes L = 16, d = 64, n_pre, n_post <= 16, n_global <= 16):
+    one warp per query frame on CUDA cores.  Reported so that the cost off
+    the fast path is visible, not as a tuned figure."""
     import torch
 
     import clip_temporal_modules_b200 as vi
-    n_pre = n_post = min(16, w.F // w.N)
+    n_pre, n_post, n_global = w.n_pre, w.n_post, min(32, w.F)
 
     def attn():
         vi.dual_attn(d["q"], d["k"], d["v"], out, N=w.N, heads=w.heads, n_pre=n_pre,
-                     n_post=n_post, n_global=w.n_global)
+                     n_post=n_post, n_global=n_global)
     attn()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -552,8 +553,34 @@ def attn_generic_path(w, d, out, stream, reps=2):
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / reps
     S = w.P * w.F * w.C * w.elem_bytes
-    return {"n_pre": n_pre, "n_post": n_post, "n_global": w.n_global, "ms": round(ms, 4),
+    return {"n_pre": n_pre, "n_post": n_post, "n_global": n_global, "ms": round(ms, 4),
             "GB/s": round(4 * S / (ms / 1e3) / 1e9, 1), "path": "dual_attn_generic (CUDA cores)"}
+
+
+def attn_halo16(w, d, out, stream, reps=10):
+    """The attention with n_pre = n_post = 16 (a whole clip of context on each
+    side): the tensor-core kernel with its 16-row windows."""
+    import torch
+
+    import clip_temporal_modules_b200 as vi
+    n = min(16, w.F // w.N)
+
+    def attn():
+        vi.dual_attn(d["q"], d["k"], d["v"], out, N=w.N, heads=w.heads, n_pre=n, n_post=n,
+                     n_global=w.n_global)
+    for _ in range(2):
+        attn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        attn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    S = w.P * w.F * w.C * w.elem_bytes
+    return {"n_pre": n, "n_post": n, "n_global": w.n_global, "ms": round(ms, 4),
+            "GB/s": round(4 * S / (ms / 1e3) / 1e9, 1)}
 
 
 def _ablation(w, d, out, rest, stream, reps, S, a, b_, g):

@@ -127,21 +127,29 @@ int dual_attn_generic_launch(const T* q, const T* k, const T* v, T* out, int F, 
 
 constexpr int FA_CLIPS = 8;                       // clips per CTA (one per warp)
 constexpr int FA_L = 16;                          // frames per clip
-constexpr int FA_HALO = 8;                        // max n_pre / n_post
+constexpr int FA_HALO = 8;                        // halo rows of a shard's padded k/v storage
+constexpr int FA_HALO_MAX = 16;                   // max n_pre / n_post of the fast path (= L)
 constexpr int FA_NG = 16;                         // max n_global
 constexpr int FA_ROWS_Q = FA_CLIPS * FA_L;        // 128 query rows
-constexpr int FA_ROWS_W = FA_ROWS_Q + 2 * FA_HALO;  // 144 window rows
 constexpr int FA_ROW_BYTES = 128;                 // 64 bf16 channels of one head
-constexpr uint32_t FA_OFF_Q = 0;
-constexpr uint32_t FA_OFF_KW = FA_OFF_Q + FA_ROWS_Q * FA_ROW_BYTES;     // 16384
-constexpr uint32_t FA_OFF_VW = FA_OFF_KW + FA_ROWS_W * FA_ROW_BYTES;    // 34816
-constexpr uint32_t FA_OFF_KG = FA_OFF_VW + FA_ROWS_W * FA_ROW_BYTES;    // 53248
-constexpr uint32_t FA_OFF_VG = FA_OFF_KG + FA_NG * FA_ROW_BYTES;        // 55296
-constexpr uint32_t FA_OFF_BAR = FA_OFF_VG + FA_NG * FA_ROW_BYTES;       // 57344
-constexpr uint32_t FA_SMEM_BYTES = FA_OFF_BAR + 16 + 1024;  // + slack for 1024B alignment
-static_assert(FA_OFF_KW % 1024 == 0 && FA_OFF_VW % 1024 == 0 && FA_OFF_KG % 1024 == 0 &&
-                  FA_OFF_VG % 1024 == 0,
-              "128B-swizzled regions must start on 1024-byte boundaries");
+
+// Shared-memory layout of the kernel for halo width H (8: every n_pre,
+// n_post <= 8; 16: up to a whole clip): Q | K window | V window | K global |
+// V global | barrier, the swizzled regions on 1024-byte boundaries.
+template <int H>
+struct FaLayout {
+  static constexpr int ROWS_W = FA_ROWS_Q + 2 * H;      // 144 or 160 window rows
+  static constexpr uint32_t OFF_Q = 0;
+  static constexpr uint32_t OFF_KW = OFF_Q + FA_ROWS_Q * FA_ROW_BYTES;
+  static constexpr uint32_t OFF_VW = OFF_KW + ROWS_W * FA_ROW_BYTES;
+  static constexpr uint32_t OFF_KG = OFF_VW + ROWS_W * FA_ROW_BYTES;
+  static constexpr uint32_t OFF_VG = OFF_KG + FA_NG * FA_ROW_BYTES;
+  static constexpr uint32_t OFF_BAR = OFF_VG + FA_NG * FA_ROW_BYTES;
+  static constexpr uint32_t SMEM = OFF_BAR + 16 + 1024;   // + slack for 1024B alignment
+  static_assert(OFF_KW % 1024 == 0 && OFF_VW % 1024 == 0 && OFF_KG % 1024 == 0 &&
+                    OFF_VG % 1024 == 0,
+                "128B-swizzled regions must start on 1024-byte boundaries");
+};
 
 // Byte address of 16-byte chunk `chunk` of row `row` in a 128B-swizzled region.
 __device__ __forceinline__ uint32_t sw128(uint32_t region, int row, int chunk) {
@@ -158,16 +166,26 @@ struct FaMaps {
 // the halo width for a shard whose neighbours' frames are stacked around it).
 // The grid covers the selected clip blocks of every (position, head): blocks
 // [0, sel_lo) and [sel_hi0, sel_hi0 + n_sel - sel_lo).
+//
+// H: halo rows on each side of the CTA's 128 frames (the key list of a clip
+// is H window rows before it, its own 16, H after it, then the 16 global
+// frames: 2H + 32 keys, in n-tiles of 8).
+template <int H>
 __global__ void __launch_bounds__(256) dual_attn_bf16_mma(const __grid_constant__ FaMaps maps,
                                                           int F, int N, int heads, int sel_lo,
                                                           int sel_hi0, int n_sel, int n_pre,
                                                           int n_post, int n_global,
                                                           float scale_log2, int kv_off, int clip0,
                                                           int n_total, unsigned int* err_word) {
+  using Lay = FaLayout<H>;
+  constexpr int NW = 2 * H + FA_L;        // window keys of a clip
+  constexpr int NTW = NW / 8;             // their n-tiles (4 or 6)
+  constexpr int NT = NTW + FA_NG / 8;     // all n-tiles (6 or 8)
+  constexpr int KS = NT / 2;              // k-steps of P.V (3 or 4)
   extern __shared__ uint8_t smem_raw[];
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
-  const uint32_t sQ = base + FA_OFF_Q, sKW = base + FA_OFF_KW, sVW = base + FA_OFF_VW;
-  const uint32_t sKG = base + FA_OFF_KG, sVG = base + FA_OFF_VG, bar = base + FA_OFF_BAR;
+  const uint32_t sQ = base + Lay::OFF_Q, sKW = base + Lay::OFF_KW, sVW = base + Lay::OFF_VW;
+  const uint32_t sKG = base + Lay::OFF_KG, sVG = base + Lay::OFF_VG, bar = base + Lay::OFF_BAR;
 
   const int sb = blockIdx.x % n_sel;
   const int blk = sb < sel_lo ? sb : sel_hi0 + (sb - sel_lo);
@@ -182,12 +200,12 @@ __global__ void __launch_bounds__(256) dual_attn_bf16_mma(const __grid_constant_
   }
   __syncthreads();
   if (threadIdx.x == 0) {
-    const uint32_t bytes = (FA_ROWS_Q + 2 * FA_ROWS_W) * FA_ROW_BYTES +
+    const uint32_t bytes = (FA_ROWS_Q + 2 * Lay::ROWS_W) * FA_ROW_BYTES +
                            (n_global > 0 ? 2 * FA_NG * FA_ROW_BYTES : 0);
     mbar_arrive_expect_tx(bar, bytes);
     tma_load_3d(sQ, &maps.q, h * 64, f0, p, bar);
-    tma_load_3d(sKW, &maps.k, h * 64, f0 - FA_HALO + kv_off, p, bar);
-    tma_load_3d(sVW, &maps.v, h * 64, f0 - FA_HALO + kv_off, p, bar);
+    tma_load_3d(sKW, &maps.k, h * 64, f0 - H + kv_off, p, bar);
+    tma_load_3d(sVW, &maps.v, h * 64, f0 - H + kv_off, p, bar);
     if (n_global > 0) {
       tma_load_3d(sKG, &maps.kg, h * 64, 0, p, bar);
       tma_load_3d(sVG, &maps.vg, h * 64, 0, p, bar);
@@ -199,7 +217,7 @@ __global__ void __launch_bounds__(256) dual_attn_bf16_mma(const __grid_constant_
   if (clip < N) {
     const int gclip = clip0 + clip;              // index in the whole video
     const int g = lane >> 2, qd = lane & 3;
-    // ---- S = Q K^T over 48 keys (6 n-tiles of 8), 4 k-steps of 16 dims ----
+    // ---- S = Q K^T over 2H + 32 keys (NT n-tiles of 8), 4 k-steps of 16 dims ----
     uint32_t qa[4][4];
 #pragma unroll
     for (int ks = 0; ks < 4; ++ks)
@@ -209,13 +227,13 @@ __global__ void __launch_bounds__(256) dual_attn_bf16_mma(const __grid_constant_
     // would read them are skipped (their scores are masked below anyway, but
     // stale shared memory must not reach the P.V product as 0 * NaN).
     const bool has_global = n_global > 0;
-    float s[6][4];
+    float s[NT][4];
 #pragma unroll
-    for (int nt = 0; nt < 6; ++nt) {
+    for (int nt = 0; nt < NT; ++nt) {
       s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
-      if (nt >= 4 && !has_global) continue;
-      const uint32_t region = nt < 4 ? sKW : sKG;
-      const int row = nt < 4 ? warp * 16 + nt * 8 + (lane & 7) : (nt - 4) * 8 + (lane & 7);
+      if (nt >= NTW && !has_global) continue;
+      const uint32_t region = nt < NTW ? sKW : sKG;
+      const int row = nt < NTW ? warp * 16 + nt * 8 + (lane & 7) : (nt - NTW) * 8 + (lane & 7);
 #pragma unroll
       for (int kp = 0; kp < 2; ++kp) {
         uint32_t b0, b1, b2, b3;
@@ -227,15 +245,15 @@ __global__ void __launch_bounds__(256) dual_attn_bf16_mma(const __grid_constant_
     // ---- mask absent keys, softmax in log2 units ----
     float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-    for (int nt = 0; nt < 6; ++nt) {
+    for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         const int kk = nt * 8 + 2 * qd + c;     // key index in the warp's list
         bool valid;
-        if (kk < FA_HALO) valid = gclip > 0 && kk >= FA_HALO - n_pre;
-        else if (kk < FA_HALO + FA_L) valid = true;
-        else if (kk < 32) valid = gclip < n_total - 1 && kk - (FA_HALO + FA_L) < n_post;
-        else valid = kk - 32 < n_global;
+        if (kk < H) valid = gclip > 0 && kk >= H - n_pre;
+        else if (kk < H + FA_L) valid = true;
+        else if (kk < NW) valid = gclip < n_total - 1 && kk - (H + FA_L) < n_post;
+        else valid = kk - NW < n_global;
         s[nt][c] = valid ? s[nt][c] * scale_log2 : -INFINITY;
         s[nt][c + 2] = valid ? s[nt][c + 2] * scale_log2 : -INFINITY;
         mx0 = fmaxf(mx0, s[nt][c]);
@@ -248,10 +266,10 @@ __global__ void __launch_bounds__(256) dual_attn_bf16_mma(const __grid_constant_
       mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
     }
     // P in bf16 as mma A fragments: k-step ks covers keys 16ks .. 16ks+15.
-    uint32_t pa[3][4];
+    uint32_t pa[KS][4];
     float l0 = 0.f, l1 = 0.f;
 #pragma unroll
-    for (int nt = 0; nt < 6; ++nt) {
+    for (int nt = 0; nt < NT; ++nt) {
       const uint32_t lo = pack2_bf16(exp2f(s[nt][0] - mx0), exp2f(s[nt][1] - mx0));
       const uint32_t hi = pack2_bf16(exp2f(s[nt][2] - mx1), exp2f(s[nt][3] - mx1));
       l0 += __uint_as_float(lo << 16) + __uint_as_float(lo & 0xFFFF0000u);
@@ -264,15 +282,15 @@ __global__ void __launch_bounds__(256) dual_attn_bf16_mma(const __grid_constant_
       l0 += __shfl_xor_sync(0xffffffffu, l0, o);
       l1 += __shfl_xor_sync(0xffffffffu, l1, o);
     }
-    // ---- O = P V: 3 k-steps of 16 keys x 8 n-tiles of 8 dims ----
+    // ---- O = P V: KS k-steps of 16 keys x 8 n-tiles of 8 dims ----
     float o[8][4];
 #pragma unroll
     for (int nd = 0; nd < 8; ++nd) o[nd][0] = o[nd][1] = o[nd][2] = o[nd][3] = 0.f;
 #pragma unroll
-    for (int ks = 0; ks < 3; ++ks) {
-      if (ks == 2 && !has_global) continue;
-      const uint32_t region = ks < 2 ? sVW : sVG;
-      const int row = (ks < 2 ? warp * 16 + ks * 16 : 0) + (lane & 15);
+    for (int ks = 0; ks < KS; ++ks) {
+      if (ks == KS - 1 && !has_global) continue;
+      const uint32_t region = ks < KS - 1 ? sVW : sVG;
+      const int row = (ks < KS - 1 ? warp * 16 + ks * 16 : 0) + (lane & 15);
 #pragma unroll
       for (int nd = 0; nd < 8; nd += 2) {
         uint32_t b0, b1, b2, b3;
@@ -305,14 +323,31 @@ bool encode_tmap(CUtensorMap* map, const void* base, int rank, const uint64_t* d
                  const uint64_t* strides_bytes, const uint32_t* box, CUtensorMapSwizzle swz,
                  CUtensorMapDataType dt);
 
-int dual_attn_bf16_fast(const bf16* q, const bf16* k, const bf16* v, bf16* out, int F, int N,
-                        int P, int heads, int n_pre, int n_post, int n_global,
-                        cudaStream_t stream) {
+// Raise the kernel's shared-memory limit once per device and halo width.
+template <int H>
+static int fa_prepare() {
+  static std::atomic<bool> attr_set[64] = {};
+  int dev = 0;
+  VI_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64 || !attr_set[dev].load(std::memory_order_acquire)) {
+    // Idempotent, so concurrent first calls may both set it.
+    VI_CUDA_TRY(cudaFuncSetAttribute(dual_attn_bf16_mma<H>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     FaLayout<H>::SMEM));
+    if (dev >= 0 && dev < 64) attr_set[dev].store(true, std::memory_order_release);
+  }
+  return VI_OK;
+}
+
+template <int H>
+static int fa_fast_launch(const bf16* q, const bf16* k, const bf16* v, bf16* out, int F, int N,
+                          int P, int heads, int n_pre, int n_post, int n_global,
+                          cudaStream_t stream) {
   const int C = heads * 64;
   FaMaps maps;
   const uint64_t dims[3] = {(uint64_t)C, (uint64_t)F, (uint64_t)P};
   const uint64_t strides[2] = {(uint64_t)C * 2, (uint64_t)F * C * 2};
-  const uint32_t boxQ[3] = {64, FA_ROWS_Q, 1}, boxW[3] = {64, FA_ROWS_W, 1};
+  const uint32_t boxQ[3] = {64, FA_ROWS_Q, 1}, boxW[3] = {64, FaLayout<H>::ROWS_W, 1};
   const CUtensorMapDataType BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const CUtensorMapSwizzle SW = CU_TENSOR_MAP_SWIZZLE_128B;
   bool ok = encode_tmap(&maps.q, q, 3, dims, strides, boxQ, SW, BF) &&
@@ -331,25 +366,29 @@ int dual_attn_bf16_fast(const bf16* q, const bf16* k, const bf16* v, bf16* out, 
     maps.vg = maps.v;
   }
   if (!ok) return VI_ERR_CUDA;
-  static std::atomic<bool> attr_set[64] = {};
-  int dev = 0;
-  VI_CUDA_TRY(cudaGetDevice(&dev));
-  if (dev < 0 || dev >= 64 || !attr_set[dev].load(std::memory_order_acquire)) {
-    // Idempotent, so concurrent first calls may both set it.
-    VI_CUDA_TRY(cudaFuncSetAttribute(dual_attn_bf16_mma,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, FA_SMEM_BYTES));
-    if (dev >= 0 && dev < 64) attr_set[dev].store(true, std::memory_order_release);
-  }
+  int st = fa_prepare<H>();
+  if (st != VI_OK) return st;
   const int nblk = (N + FA_CLIPS - 1) / FA_CLIPS;
   const int64_t grid = (int64_t)P * heads * nblk;
   if (grid > 0x7fffffff) return VI_ERR_UNSUPPORTED;
   const float scale_log2 = 1.4426950408889634f / 8.0f;    // log2(e) / sqrt(64)
   unsigned int* err = device_error_word();
   if (!err) return VI_ERR_CUDA;
-  dual_attn_bf16_mma<<<(unsigned)grid, 256, FA_SMEM_BYTES, stream>>>(
+  dual_attn_bf16_mma<H><<<(unsigned)grid, 256, FaLayout<H>::SMEM, stream>>>(
       maps, F, N, heads, nblk, 0, nblk, n_pre, n_post, n_global, scale_log2, 0, 0, N, err);
   VI_LAUNCHED();
   return VI_OK;
+}
+
+// The whole video on one GPU: the narrower window (8 rows each side) where
+// both context sizes fit it, else the 16-row one.
+int dual_attn_bf16_fast(const bf16* q, const bf16* k, const bf16* v, bf16* out, int F, int N,
+                        int P, int heads, int n_pre, int n_post, int n_global,
+                        cudaStream_t stream) {
+  if (n_pre <= FA_HALO && n_post <= FA_HALO)
+    return fa_fast_launch<FA_HALO>(q, k, v, out, F, N, P, heads, n_pre, n_post, n_global, stream);
+  return fa_fast_launch<FA_HALO_MAX>(q, k, v, out, F, N, P, heads, n_pre, n_post, n_global,
+                                     stream);
 }
 
 // One shard of a video cut along frames (clip-parallel over several GPUs):
@@ -369,7 +408,7 @@ int dual_attn_bf16_shard(const bf16* q, const bf16* k_ext, const bf16* v_ext, co
   const uint64_t strides[2] = {(uint64_t)C * 2, (uint64_t)F_loc * C * 2};
   const uint64_t edims[3] = {(uint64_t)C, (uint64_t)F_ext, (uint64_t)P};
   const uint64_t estrides[2] = {(uint64_t)C * 2, (uint64_t)F_ext * C * 2};
-  const uint32_t boxQ[3] = {64, FA_ROWS_Q, 1}, boxW[3] = {64, FA_ROWS_W, 1};
+  const uint32_t boxQ[3] = {64, FA_ROWS_Q, 1}, boxW[3] = {64, FaLayout<FA_HALO>::ROWS_W, 1};
   const CUtensorMapDataType BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const CUtensorMapSwizzle SW = CU_TENSOR_MAP_SWIZZLE_128B;
   bool ok = encode_tmap(&maps.q, q, 3, dims, strides, boxQ, SW, BF) &&
@@ -387,14 +426,8 @@ int dual_attn_bf16_shard(const bf16* q, const bf16* k_ext, const bf16* v_ext, co
     maps.vg = maps.v;
   }
   if (!ok) return VI_ERR_CUDA;
-  static std::atomic<bool> attr_set[64] = {};
-  int dev = 0;
-  VI_CUDA_TRY(cudaGetDevice(&dev));
-  if (dev < 0 || dev >= 64 || !attr_set[dev].load(std::memory_order_acquire)) {
-    VI_CUDA_TRY(cudaFuncSetAttribute(dual_attn_bf16_mma,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, FA_SMEM_BYTES));
-    if (dev >= 0 && dev < 64) attr_set[dev].store(true, std::memory_order_release);
-  }
+  int st = fa_prepare<FA_HALO>();
+  if (st != VI_OK) return st;
   const int nblk = (N_loc + FA_CLIPS - 1) / FA_CLIPS;
   // Interior blocks [a, b): their k/v window (8 rows on each side of the
   // block) lies inside the shard's own frames.  The others are the boundary.
@@ -411,7 +444,7 @@ int dual_attn_bf16_shard(const bf16* q, const bf16* k_ext, const bf16* v_ext, co
   const float scale_log2 = 1.4426950408889634f / 8.0f;    // log2(e) / sqrt(64)
   unsigned int* err = device_error_word();
   if (!err) return VI_ERR_CUDA;
-  dual_attn_bf16_mma<<<(unsigned)grid, 256, FA_SMEM_BYTES, stream>>>(
+  dual_attn_bf16_mma<FA_HALO><<<(unsigned)grid, 256, FaLayout<FA_HALO>::SMEM, stream>>>(
       maps, F_loc, N_loc, heads, sel_lo, sel_hi0, n_sel, n_pre, n_post, n_global, scale_log2,
       FA_HALO, clip0, N, err);
   VI_LAUNCHED();
@@ -419,8 +452,13 @@ int dual_attn_bf16_shard(const bf16* q, const bf16* k_ext, const bf16* v_ext, co
 }
 
 bool dual_attn_fast_ok(int F, int N, int d, int n_pre, int n_post, int n_global) {
-  return d == 64 && F / N == FA_L && n_pre <= FA_HALO && n_post <= FA_HALO &&
+  return d == 64 && F / N == FA_L && n_pre <= FA_HALO_MAX && n_post <= FA_HALO_MAX &&
          n_global <= FA_NG;
+}
+
+// A shard's k/v storage carries FA_HALO rows of its neighbours on each side.
+bool dual_attn_shard_ok(int L, int d, int n_pre, int n_post, int n_global) {
+  return d == 64 && L == FA_L && n_pre <= FA_HALO && n_post <= FA_HALO && n_global <= FA_NG;
 }
 
 template int dual_attn_generic_launch<float>(const float*, const float*, const float*, float*,

@@ -36,6 +36,7 @@ int dual_attn_generic_launch(const T*, const T*, const T*, T*, int, int, int, in
 int dual_attn_bf16_fast(const bf16*, const bf16*, const bf16*, bf16*, int, int, int, int, int,
                         int, int, cudaStream_t);
 bool dual_attn_fast_ok(int F, int N, int d, int n_pre, int n_post, int n_global);
+bool dual_attn_shard_ok(int L, int d, int n_pre, int n_post, int n_global);
 int dual_attn_bf16_shard(const bf16*, const bf16*, const bf16*, const bf16*, const bf16*, bf16*,
                          int, int, int, int, int, int, int, int, int, int, cudaStream_t);
 int temporal_conv_bf16_tc_shard(const bf16*, const bf16*, const bf16*, bf16*, int, int, int, int,
@@ -365,7 +366,7 @@ int attn_shard_entry(const void* q, const void* k_ext, const void* v_ext, const 
   if (n_pre < 0 || n_post < 0 || n_global < 0 || n_global > N * L) return VI_ERR_INVALID_ARG;
   if (N > 1 && (n_pre > L || n_post > L)) return VI_ERR_INVALID_ARG;
   if ((double)P * (double)(F_loc + 16) * (double)C > 1.099511627776e12) return VI_ERR_UNSUPPORTED;
-  if (!dual_attn_fast_ok(L, 1, d, n_pre, n_post, n_global)) return VI_ERR_UNSUPPORTED;
+  if (!dual_attn_shard_ok(L, d, n_pre, n_post, n_global)) return VI_ERR_UNSUPPORTED;
   if (P == 0) return VI_OK;
   if (!q || !k_ext || !v_ext || !out || (n_global > 0 && (!k_glob || !v_glob)))
     return VI_ERR_INVALID_ARG;

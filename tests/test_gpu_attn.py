@@ -44,6 +44,10 @@ SMALL = [
     W("bf16_no_global", "bf16", 64, 4, 3, 1, n_global=0),
     W("bf16_one_clip", "bf16", 16, 1, 6, 2, n_global=4),
     W("bf16_no_context", "bf16", 48, 3, 2, 1, n_pre=0, n_post=0, n_global=0),
+    W("bf16_halo16", "bf16", 64, 4, 3, 2, n_pre=16, n_post=16, n_global=16),   # 16-row window
+    W("bf16_halo12_2blk_ragged", "bf16", 160, 10, 3, 2, n_pre=12, n_post=9, n_global=7),
+    W("bf16_halo_mixed", "bf16", 96, 6, 2, 1, n_pre=4, n_post=13, n_global=16),
+    W("bf16_halo16_no_global", "bf16", 48, 3, 2, 1, n_pre=16, n_post=10, n_global=0),
     W("bf16_L8_generic", "bf16", 32, 4, 4, 2),                 # L = 8: generic path
     W("bf16_L32_generic", "bf16", 64, 2, 3, 1, n_pre=16, n_post=12, n_global=20),
     W("f32_generic", "f32", 48, 3, 3, 2),
