@@ -652,23 +652,40 @@ def attention_module(w, d, out, y, z, stream, reps=5):
     ws = torch.empty(n // 2, dtype=torch.bfloat16, device=dev)
     x = d["conv_x"]
 
+    from clip_temporal_modules_b200._binding import temporal_attention_forced_form
+
     def run():
         vi.temporal_attention(x, wq, bq, wo, bo, y, ws, N=w.N, heads=w.heads, n_pre=w.n_pre,
                               n_post=w.n_post, n_global=w.n_global)
 
-    for _ in range(2):
-        run()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(reps):
-        run()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / reps
+    def run_unfused():
+        temporal_attention_forced_form(x, wq, bq, wo, bo, y, ws, N=w.N, heads=w.heads,
+                                       fused=False, n_pre=w.n_pre, n_post=w.n_post,
+                                       n_global=w.n_global)
+
+    def timed(fn):
+        for _ in range(2):
+            fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    ms = timed(run)
+    ms_unfused = timed(run_unfused)
     del ws
     flops = 4 * 2 * w.C * w.C * w.tokens
+    S = w.tokens * w.C * 2
+    # x read, q/k/v written and read back, out written (a stays on chip when
+    # the output projection is fused into the attention)
+    hbm = 8 * S
     return {"ms": round(ms, 4), "tokens_per_s": round(w.tokens / (ms / 1e3), 1),
-            "projection_tflops_total": round(flops / 1e12, 3)}
+            "projection_tflops_total": round(flops / 1e12, 3),
+            "algorithmic_gb": round(hbm / 1e9, 3),
+            "attention_then_output_gemm_ms": round(ms_unfused, 4)}
 
 
 def clip_parallel_emulated(w, d, stream, world=8, reps=5):

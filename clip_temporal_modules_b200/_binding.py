@@ -345,6 +345,37 @@ def groupnorm_conv_forced_tiles(x, gamma, beta, w, b, out=None, *, N: int, group
     return out
 
 
+def temporal_attention_forced_form(x, w_qkv, b_qkv, w_out, b_out, out=None, workspace=None, *,
+                                   N: int, heads: int, fused: bool, n_pre: int = 8,
+                                   n_post: int = 8, n_global: int = 16, stream=None):
+    """Test hook (not part of the ABI in vi.h): the attention module with its
+    form forced: the output projection fused into the attention kernel
+    (fused=True), or the attention kernel followed by the output GEMM."""
+    import torch
+    P, F, C = x.shape
+    if out is None:
+        out = torch.empty_like(x)
+    if workspace is None:
+        n = int(lib().vi_temporal_attention_workspace_bytes(F, P, C))
+        workspace = torch.empty(n // 2, dtype=torch.bfloat16, device=x.device)
+    _dev(x, w_qkv, b_qkv, w_out, b_out, out, workspace)
+    _shape(w_qkv, (3 * C, C), "w_qkv")
+    _shape(b_qkv, (3 * C,), "b_qkv")
+    _shape(w_out, (C, C), "w_out")
+    _shape(b_out, (C,), "b_out")
+    _shape(out, x.shape, "out")
+    if workspace.numel() * workspace.element_size() < 4 * P * F * C * 2:
+        raise ValueError("workspace: smaller than vi_temporal_attention_workspace_bytes")
+    fn = lib().vitest_temporal_attention_form
+    fn.argtypes = [_vp] * 7 + [_i] * 9 + [_vp]
+    fn.restype = ctypes.c_int
+    _check("vitest_temporal_attention_form", fn(
+        x.data_ptr(), w_qkv.data_ptr(), b_qkv.data_ptr(), w_out.data_ptr(), b_out.data_ptr(),
+        out.data_ptr(), workspace.data_ptr(), F, N, P, heads, C // heads, n_pre, n_post, n_global,
+        1 if fused else 0, _stream_ptr(stream)))
+    return out
+
+
 def take_device_errors() -> None:
     """Synchronise and raise if a kernel's bounded wait ran out since the last call."""
     _check("vi_take_device_errors", lib().vi_take_device_errors())

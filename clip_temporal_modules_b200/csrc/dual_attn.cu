@@ -33,6 +33,7 @@
 //   fp32, expf, and the exact key list walked in order.
 #include <atomic>
 
+#include "dual_attn_tile.cuh"
 #include "ptx.cuh"
 #include "vi_internal.cuh"
 
@@ -125,37 +126,6 @@ int dual_attn_generic_launch(const T* q, const T* k, const T* v, T* out, int F, 
 // ---------------------------------------------------------------------------
 // Fast path: TMA staging + mma.sync tensor-core tiles.
 
-constexpr int FA_CLIPS = 8;                       // clips per CTA (one per warp)
-constexpr int FA_L = 16;                          // frames per clip
-constexpr int FA_HALO = 8;                        // halo rows of a shard's padded k/v storage
-constexpr int FA_HALO_MAX = 16;                   // max n_pre / n_post of the fast path (= L)
-constexpr int FA_NG = 16;                         // max n_global
-constexpr int FA_ROWS_Q = FA_CLIPS * FA_L;        // 128 query rows
-constexpr int FA_ROW_BYTES = 128;                 // 64 bf16 channels of one head
-
-// Shared-memory layout of the kernel for halo width H (8: every n_pre,
-// n_post <= 8; 16: up to a whole clip): Q | K window | V window | K global |
-// V global | barrier, the swizzled regions on 1024-byte boundaries.
-template <int H>
-struct FaLayout {
-  static constexpr int ROWS_W = FA_ROWS_Q + 2 * H;      // 144 or 160 window rows
-  static constexpr uint32_t OFF_Q = 0;
-  static constexpr uint32_t OFF_KW = OFF_Q + FA_ROWS_Q * FA_ROW_BYTES;
-  static constexpr uint32_t OFF_VW = OFF_KW + ROWS_W * FA_ROW_BYTES;
-  static constexpr uint32_t OFF_KG = OFF_VW + ROWS_W * FA_ROW_BYTES;
-  static constexpr uint32_t OFF_VG = OFF_KG + FA_NG * FA_ROW_BYTES;
-  static constexpr uint32_t OFF_BAR = OFF_VG + FA_NG * FA_ROW_BYTES;
-  static constexpr uint32_t SMEM = OFF_BAR + 16 + 1024;   // + slack for 1024B alignment
-  static_assert(OFF_KW % 1024 == 0 && OFF_VW % 1024 == 0 && OFF_KG % 1024 == 0 &&
-                    OFF_VG % 1024 == 0,
-                "128B-swizzled regions must start on 1024-byte boundaries");
-};
-
-// Byte address of 16-byte chunk `chunk` of row `row` in a 128B-swizzled region.
-__device__ __forceinline__ uint32_t sw128(uint32_t region, int row, int chunk) {
-  return region + row * FA_ROW_BYTES + (((chunk ^ (row & 7)) & 7) << 4);
-}
-
 struct FaMaps {
   CUtensorMap q, k, v, kg, vg, o;
 };
@@ -178,10 +148,6 @@ __global__ void __launch_bounds__(256) dual_attn_bf16_mma(const __grid_constant_
                                                           float scale_log2, int kv_off, int clip0,
                                                           int n_total, unsigned int* err_word) {
   using Lay = FaLayout<H>;
-  constexpr int NW = 2 * H + FA_L;        // window keys of a clip
-  constexpr int NTW = NW / 8;             // their n-tiles (4 or 6)
-  constexpr int NT = NTW + FA_NG / 8;     // all n-tiles (6 or 8)
-  constexpr int KS = NT / 2;              // k-steps of P.V (3 or 4)
   extern __shared__ uint8_t smem_raw[];
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
   const uint32_t sQ = base + Lay::OFF_Q, sKW = base + Lay::OFF_KW, sVW = base + Lay::OFF_VW;
@@ -216,99 +182,8 @@ __global__ void __launch_bounds__(256) dual_attn_bf16_mma(const __grid_constant_
   const int clip = blk * FA_CLIPS + warp;
   if (clip < N) {
     const int gclip = clip0 + clip;              // index in the whole video
-    const int g = lane >> 2, qd = lane & 3;
-    // ---- S = Q K^T over 2H + 32 keys (NT n-tiles of 8), 4 k-steps of 16 dims ----
-    uint32_t qa[4][4];
-#pragma unroll
-    for (int ks = 0; ks < 4; ++ks)
-      ldsm_x4(sw128(sQ, warp * 16 + (lane & 15), 2 * ks + (lane >> 4)), qa[ks][0], qa[ks][1],
-              qa[ks][2], qa[ks][3]);
-    // Without global frames their K/V tiles are not loaded: the MMAs that
-    // would read them are skipped (their scores are masked below anyway, but
-    // stale shared memory must not reach the P.V product as 0 * NaN).
-    const bool has_global = n_global > 0;
-    float s[NT][4];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
-      if (nt >= NTW && !has_global) continue;
-      const uint32_t region = nt < NTW ? sKW : sKG;
-      const int row = nt < NTW ? warp * 16 + nt * 8 + (lane & 7) : (nt - NTW) * 8 + (lane & 7);
-#pragma unroll
-      for (int kp = 0; kp < 2; ++kp) {
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4(sw128(region, row, 4 * kp + (lane >> 3)), b0, b1, b2, b3);
-        mma_bf16_16816(s[nt], qa[2 * kp], b0, b1);
-        mma_bf16_16816(s[nt], qa[2 * kp + 1], b2, b3);
-      }
-    }
-    // ---- mask absent keys, softmax in log2 units ----
-    float mx0 = -INFINITY, mx1 = -INFINITY;
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        const int kk = nt * 8 + 2 * qd + c;     // key index in the warp's list
-        bool valid;
-        if (kk < H) valid = gclip > 0 && kk >= H - n_pre;
-        else if (kk < H + FA_L) valid = true;
-        else if (kk < NW) valid = gclip < n_total - 1 && kk - (H + FA_L) < n_post;
-        else valid = kk - NW < n_global;
-        s[nt][c] = valid ? s[nt][c] * scale_log2 : -INFINITY;
-        s[nt][c + 2] = valid ? s[nt][c + 2] * scale_log2 : -INFINITY;
-        mx0 = fmaxf(mx0, s[nt][c]);
-        mx1 = fmaxf(mx1, s[nt][c + 2]);
-      }
-    }
-#pragma unroll
-    for (int o = 1; o <= 2; o <<= 1) {
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
-    }
-    // P in bf16 as mma A fragments: k-step ks covers keys 16ks .. 16ks+15.
-    uint32_t pa[KS][4];
-    float l0 = 0.f, l1 = 0.f;
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      const uint32_t lo = pack2_bf16(exp2f(s[nt][0] - mx0), exp2f(s[nt][1] - mx0));
-      const uint32_t hi = pack2_bf16(exp2f(s[nt][2] - mx1), exp2f(s[nt][3] - mx1));
-      l0 += __uint_as_float(lo << 16) + __uint_as_float(lo & 0xFFFF0000u);
-      l1 += __uint_as_float(hi << 16) + __uint_as_float(hi & 0xFFFF0000u);
-      pa[nt >> 1][(nt & 1) * 2 + 0] = lo;
-      pa[nt >> 1][(nt & 1) * 2 + 1] = hi;
-    }
-#pragma unroll
-    for (int o = 1; o <= 2; o <<= 1) {
-      l0 += __shfl_xor_sync(0xffffffffu, l0, o);
-      l1 += __shfl_xor_sync(0xffffffffu, l1, o);
-    }
-    // ---- O = P V: KS k-steps of 16 keys x 8 n-tiles of 8 dims ----
-    float o[8][4];
-#pragma unroll
-    for (int nd = 0; nd < 8; ++nd) o[nd][0] = o[nd][1] = o[nd][2] = o[nd][3] = 0.f;
-#pragma unroll
-    for (int ks = 0; ks < KS; ++ks) {
-      if (ks == KS - 1 && !has_global) continue;
-      const uint32_t region = ks < KS - 1 ? sVW : sVG;
-      const int row = (ks < KS - 1 ? warp * 16 + ks * 16 : 0) + (lane & 15);
-#pragma unroll
-      for (int nd = 0; nd < 8; nd += 2) {
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4_t(sw128(region, row, nd + (lane >> 4)), b0, b1, b2, b3);
-        mma_bf16_16816(o[nd], pa[ks], b0, b1);
-        mma_bf16_16816(o[nd + 1], pa[ks], b2, b3);
-      }
-    }
-    // ---- normalise, round, write this warp's 16 rows into the Q buffer ----
-    const float inv0 = 1.f / l0, inv1 = 1.f / l1;
-    const int r0 = warp * 16 + g, r1 = r0 + 8;
-#pragma unroll
-    for (int nd = 0; nd < 8; ++nd) {
-      const uint32_t w0 = pack2_bf16(o[nd][0] * inv0, o[nd][1] * inv0);
-      const uint32_t w1 = pack2_bf16(o[nd][2] * inv1, o[nd][3] * inv1);
-      asm volatile("st.shared.b32 [%0], %1;" ::"r"(sw128(sQ, r0, nd) + 4 * qd), "r"(w0));
-      asm volatile("st.shared.b32 [%0], %1;" ::"r"(sw128(sQ, r1, nd) + 4 * qd), "r"(w1));
-    }
+    fa_attend_warp<H>(sQ, sKW, sVW, sKG, sVG, warp, lane, gclip, n_total, n_pre, n_post,
+                      n_global, scale_log2);
   }
   fence_proxy_async_smem();
   __syncthreads();

@@ -36,6 +36,10 @@ int dual_attn_generic_launch(const T*, const T*, const T*, T*, int, int, int, in
 int dual_attn_bf16_fast(const bf16*, const bf16*, const bf16*, bf16*, int, int, int, int, int,
                         int, int, cudaStream_t);
 bool dual_attn_fast_ok(int F, int N, int d, int n_pre, int n_post, int n_global);
+int dual_attn_oproj_bf16_launch(const bf16* q, const bf16* k, const bf16* v, const bf16* w_out,
+                                const bf16* b_out, bf16* out, int F, int N, int P, int heads,
+                                int n_pre, int n_post, int n_global, cudaStream_t stream);
+bool dual_attn_oproj_ok(int F, int N, int d, int heads, int n_pre, int n_post, int n_global);
 bool dual_attn_shard_ok(int L, int d, int n_pre, int n_post, int n_global);
 int dual_attn_bf16_shard(const bf16*, const bf16*, const bf16*, const bf16*, const bf16*, bf16*,
                          int, int, int, int, int, int, int, int, int, int, cudaStream_t);
@@ -297,10 +301,12 @@ int gn_conv_entry(const void* x, const void* gamma, const void* beta, const void
   return st;
 }
 
+// form: 1 = attention with the output projection fused in, 0 = attention
+// kernel then output GEMM, -1 = the fused form where its shapes allow.
 int temporal_attention_entry(const void* x, const void* w_qkv, const void* b_qkv,
                              const void* w_out, const void* b_out, void* out, void* workspace,
                              int F, int N, int P, int heads, int d, int n_pre, int n_post,
-                             int n_global, vi_stream_t stream) {
+                             int n_global, vi_stream_t stream, int form = -1) {
   using T = bf16;
   if (heads <= 0 || d <= 0 || (int64_t)heads * d > 0x7fffffff) return VI_ERR_INVALID_ARG;
   const int C = heads * d;
@@ -327,6 +333,9 @@ int temporal_attention_entry(const void* x, const void* w_qkv, const void* b_qkv
     return VI_ERR_INVALID_ARG;
   if (!temporal_conv_tc_ok(F, P, C, 1) || !linear_tc_ok(F, P, C, 3 * C, 3))
     return VI_ERR_UNSUPPORTED;
+  const bool fuse_ok = dual_attn_oproj_ok(F, N, d, heads, n_pre, n_post, n_global);
+  if (form == 1 && !fuse_ok) return VI_ERR_UNSUPPORTED;
+  const bool fused = form != 0 && fuse_ok;
   cudaStream_t s = as_stream(stream);
   const T* xx = static_cast<const T*>(x);
   T* q = static_cast<T*>(workspace);
@@ -337,12 +346,15 @@ int temporal_attention_entry(const void* x, const void* w_qkv, const void* b_qkv
   // q, k and v from one GEMM of N = 3C over x (rows of w_qkv in q, k, v order).
   st = linear_bf16_tc(xx, static_cast<const T*>(w_qkv), static_cast<const T*>(b_qkv), qkv, 3, F,
                       P, C, 3 * C, s);
-  if (st == VI_OK) {
-    if (dual_attn_fast_ok(F, N, d, n_pre, n_post, n_global))
-      st = dual_attn_bf16_fast(q, k, v, a, F, N, P, heads, n_pre, n_post, n_global, s);
-    else
-      st = dual_attn_generic_launch<T>(q, k, v, a, F, N, P, heads, d, n_pre, n_post, n_global, s);
-  }
+  if (st != VI_OK) return st;
+  if (fused)   // a stays on chip: attention and output projection in one kernel
+    return dual_attn_oproj_bf16_launch(q, k, v, static_cast<const T*>(w_out),
+                                       static_cast<const T*>(b_out), static_cast<T*>(out), F, N,
+                                       P, heads, n_pre, n_post, n_global, s);
+  if (dual_attn_fast_ok(F, N, d, n_pre, n_post, n_global))
+    st = dual_attn_bf16_fast(q, k, v, a, F, N, P, heads, n_pre, n_post, n_global, s);
+  else
+    st = dual_attn_generic_launch<T>(q, k, v, a, F, N, P, heads, d, n_pre, n_post, n_global, s);
   if (st == VI_OK)
     st = temporal_conv_bf16_tc(a, static_cast<const T*>(w_out), static_cast<const T*>(b_out),
                                static_cast<T*>(out), F, P, C, 1, s);
@@ -549,6 +561,20 @@ int vitest_temporal_conv_tiles(const void* x, const void* w, const void* b, void
   return temporal_conv_bf16_tc(static_cast<const bf16*>(x), static_cast<const bf16*>(w),
                                static_cast<const bf16*>(b), static_cast<bf16*>(y), F, P, C, k,
                                as_stream(stream), nullptr, tiles);
+}
+
+// Test hook, not part of the ABI in vi.h: vi_temporal_attention with its form
+// forced (1: the output projection fused into the attention kernel; 0: the
+// attention kernel, then the output GEMM).  Shapes the fused kernel does not
+// take return VI_ERR_UNSUPPORTED for form 1.
+int vitest_temporal_attention_form(const void* x, const void* w_qkv, const void* b_qkv,
+                                   const void* w_out, const void* b_out, void* out,
+                                   void* workspace, int F, int N, int P, int heads, int d,
+                                   int n_pre, int n_post, int n_global, int form,
+                                   vi_stream_t stream) {
+  if (form != 0 && form != 1) return VI_ERR_INVALID_ARG;
+  return temporal_attention_entry(x, w_qkv, b_qkv, w_out, b_out, out, workspace, F, N, P, heads,
+                                  d, n_pre, n_post, n_global, stream, form);
 }
 
 // Test hook, not part of the ABI in vi.h: vi_groupnorm_conv with the conv's

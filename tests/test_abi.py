@@ -178,6 +178,12 @@ def test_no_global_tuning_state_in_the_abi(L):
     for tiles in (0, 3, -1, 5):
         assert conv_t(A, B, Cp, D, 64, 4, 2, 64, 3, tiles, None) == INVALID
         assert gnconv_t(A, B, Cp, D, A, B, 64, 4, 2, 64, 8, 1e-5, 3, tiles, None) == INVALID
+    form_t = L.vitest_temporal_attention_form
+    form_t.argtypes = [ctypes.c_void_p] * 7 + [ctypes.c_int] * 9 + [ctypes.c_void_p]
+    for form in (-1, 2):
+        assert form_t(A, B, Cp, D, A, B, Cp, 64, 4, 2, 1, 64, 8, 8, 16, form, None) == INVALID
+    assert form_t(None, None, None, None, None, None, None, 64, 4, 0, 1, 64, 8, 8, 16, 1,
+                  None) == OK                                               # empty
     assert conv_t(None, None, None, None, 64, 4, 0, 64, 3, 1, None) == OK     # empty
     assert conv_t(A, B, Cp, D, 64, 4, 2, 64, 2, 1, None) == INVALID         # even k
     assert conv_t(A + 4, B, Cp, D, 64, 4, 2, 64, 3, 2, None) == ALIGN

@@ -23,11 +23,18 @@ pytestmark = pytest.mark.gpu
 NAMES = ("attn_x", "w_qkv", "b_qkv", "w_out", "b_out")
 
 
-def run_case(w, positions=None):
+def run_case(w, positions=None, fused=None):
+    """fused: None = the library's choice; True / False = that form forced."""
     x, wq, bq, wo, bo = (synth.make(w, t) for t in NAMES)
     dev = [to_device(a, w.dtype) for a in (x, wq, bq, wo, bo)]
-    out = vi.temporal_attention(*dev, N=w.N, heads=w.heads, n_pre=w.n_pre, n_post=w.n_post,
-                                n_global=w.n_global)
+    if fused is None:
+        out = vi.temporal_attention(*dev, N=w.N, heads=w.heads, n_pre=w.n_pre, n_post=w.n_post,
+                                    n_global=w.n_global)
+    else:
+        from clip_temporal_modules_b200._binding import temporal_attention_forced_form
+        out = temporal_attention_forced_form(*dev, N=w.N, heads=w.heads, fused=fused,
+                                             n_pre=w.n_pre, n_post=w.n_post,
+                                             n_global=w.n_global)
     torch.cuda.synchronize()
     vi.take_device_errors()
     got = from_device(out)
@@ -50,14 +57,55 @@ SMALL = [
 ]
 
 
+# Shapes of the fused form (attention + output projection in one kernel):
+# every head count it takes (C = 64 .. 320: one to five 32-column groups per
+# epilogue warp, 64- and 32-channel store boxes), both window widths, ragged
+# last clip blocks, one clip, no global frames, context sizes off the window.
+FUSED = [
+    W("attnmod_fused_F160_N10_P3_h2", 160, 10, 3, 2),                 # 2 blocks, 2 clips in the last
+    W("attnmod_fused_F48_N3_P5_h1_noglobal", 48, 3, 5, 1, n_global=0),
+    W("attnmod_fused_F16_N1_P7_h3_oneclip", 16, 1, 7, 3, n_global=4),
+    W("attnmod_fused_F128_N8_P3_h4", 128, 8, 3, 4),
+    W("attnmod_fused_F288_N18_P2_h5_halo16", 288, 18, 2, 5, n_pre=12, n_post=16, n_global=9),
+    W("attnmod_fused_F256_N16_P2_h5_ctx", 256, 16, 2, 5, n_pre=0, n_post=3, n_global=16),
+]
+
+
 @pytest.mark.parametrize("w", SMALL, ids=lambda w: w.name)
 def test_small_elementwise(cuda_device, w):
     run_case(w)
 
 
-def test_full_size_sampled_positions(cuda_device):
+@pytest.mark.parametrize("fused", [True, False], ids=["fused", "attn_then_gemm"])
+@pytest.mark.parametrize("w", FUSED, ids=lambda w: w.name)
+def test_both_forms_elementwise(cuda_device, w, fused):
+    run_case(w, fused=fused)
+
+
+def test_fused_form_refuses_more_than_five_heads(cuda_device):
+    """Six heads (C = 384) exceed the fused kernel's TMEM and shared-memory plan:
+    the forced fused form is refused before any launch, and the library's
+    choice runs the attention kernel and the output GEMM (checked against the
+    oracle)."""
+    from clip_temporal_modules_b200._binding import temporal_attention_forced_form
+    w = W("attnmod_F32_N2_P2_h6", 32, 2, 2, 6)
+    x, wq, bq, wo, bo = (to_device(synth.make(w, t), w.dtype) for t in NAMES)
+    n0 = vi.launch_count()
+    with pytest.raises(vi.ViError):
+        temporal_attention_forced_form(x, wq, bq, wo, bo, N=w.N, heads=w.heads, fused=True)
+    assert vi.launch_count() == n0
+    run_case(w)
+
+
+@pytest.mark.parametrize("fused", [True, False], ids=["fused", "attn_then_gemm"])
+def test_full_size_sampled_positions(cuda_device, fused):
     w = synth.BY_NAME["bf16_F1024_P2560_C320"]
-    run_case(w, positions=sample_positions(w.P, count=2))
+    run_case(w, positions=sample_positions(w.P, count=2), fused=fused)
+
+
+def test_full_size_library_choice(cuda_device):
+    w = synth.BY_NAME["bf16_F1024_P2560_C320"]
+    run_case(w, positions=sample_positions(w.P, count=1))
 
 
 def test_workspace_size_and_caller_workspace(cuda_device):
