@@ -664,8 +664,6 @@ def attention_module(w, d, out, y, z, stream, reps=5):
                                        n_global=w.n_global)
 
     def timed(fn):
-        for _ in range(2):
-            fn()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for _ in range(reps):
@@ -674,8 +672,24 @@ def attention_module(w, d, out, y, z, stream, reps=5):
         torch.cuda.synchronize()
         return e0.elapsed_time(e1) / reps
 
-    ms = timed(run)
-    ms_unfused = timed(run_unfused)
+    from clip_temporal_modules_b200._binding import dual_attn_oproj
+
+    def run_kernel():    # the fused attention + output projection kernel alone
+        dual_attn_oproj(d["q"], d["k"], d["v"], wo, bo, y, N=w.N, heads=w.heads, n_pre=w.n_pre,
+                        n_post=w.n_post, n_global=w.n_global)
+
+    for _ in range(2):
+        run()
+        run_unfused()
+        run_kernel()
+    # Three interleaved rounds of each; the median round of each.
+    fused, unfused, kern = [], [], []
+    with ClockSampler(dev.index if dev.index is not None else 0) as clocks:
+        for _ in range(3):
+            fused.append(timed(run))
+            unfused.append(timed(run_unfused))
+            kern.append(timed(run_kernel))
+    ms, ms_unfused, ms_kern = sorted(fused)[1], sorted(unfused)[1], sorted(kern)[1]
     del ws
     flops = 4 * 2 * w.C * w.C * w.tokens
     S = w.tokens * w.C * 2
@@ -685,7 +699,13 @@ def attention_module(w, d, out, y, z, stream, reps=5):
     return {"ms": round(ms, 4), "tokens_per_s": round(w.tokens / (ms / 1e3), 1),
             "projection_tflops_total": round(flops / 1e12, 3),
             "algorithmic_gb": round(hbm / 1e9, 3),
-            "attention_then_output_gemm_ms": round(ms_unfused, 4)}
+            "attention_then_output_gemm_ms": round(ms_unfused, 4),
+            "rounds_ms": [round(t, 4) for t in fused],
+            # q, k, v read and out written once (W_out comes from L2)
+            "attention_oproj_kernel": {"ms": round(ms_kern, 4),
+                                       "GB/s": round(4 * S / (ms_kern / 1e3) / 1e9, 1)},
+            "attention_then_output_gemm_rounds_ms": [round(t, 4) for t in unfused],
+            "clocks": clocks.summary()}
 
 
 def clip_parallel_emulated(w, d, stream, world=8, reps=5):

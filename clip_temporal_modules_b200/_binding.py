@@ -376,6 +376,30 @@ def temporal_attention_forced_form(x, w_qkv, b_qkv, w_out, b_out, out=None, work
     return out
 
 
+def dual_attn_oproj(q, k, v, w_out, b_out, out=None, *, N: int, heads: int, n_pre: int = 8,
+                    n_post: int = 8, n_global: int = 16, stream=None):
+    """Test hook (not part of the ABI in vi.h): the attention kernel with the
+    module's output projection fused in, out = dual_attn(q, k, v) W_out^T +
+    b_out; bf16 CUDA tensors, w_out [C][C] and b_out [C] in the Linear layout."""
+    import torch
+    if out is None:
+        out = torch.empty_like(q)
+    _dev(q, k, v, w_out, b_out, out)
+    P, F, C = q.shape
+    for t, n in ((k, "k"), (v, "v"), (out, "out")):
+        _shape(t, q.shape, n)
+    _shape(w_out, (C, C), "w_out")
+    _shape(b_out, (C,), "b_out")
+    fn = lib().vitest_dual_attn_oproj
+    fn.argtypes = [_vp] * 6 + [_i] * 8 + [_vp]
+    fn.restype = ctypes.c_int
+    _check("vitest_dual_attn_oproj", fn(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), w_out.data_ptr(), b_out.data_ptr(),
+        out.data_ptr(), F, N, P, heads, C // heads, n_pre, n_post, n_global,
+        _stream_ptr(stream)))
+    return out
+
+
 def take_device_errors() -> None:
     """Synchronise and raise if a kernel's bounded wait ran out since the last call."""
     _check("vi_take_device_errors", lib().vi_take_device_errors())

@@ -67,8 +67,9 @@ struct FoLayout {
   static constexpr uint32_t BOX = FA_ROWS_Q * FA_ROW_BYTES;     // one output box
   static constexpr int BOXES_IN_STAGE = STAGE / BOX;            // 3
   // full[3], o_full[3], w_full, m_done, acc_full, tmem_empty, staged, drain
-  // (8 bytes each), TMEM slot
-  static constexpr uint32_t SMEM = OFF_BAR + 128 + 1024;   // + slack for 1024B alignment
+  // (8 bytes each), TMEM slot; then b_out in fp32
+  static constexpr uint32_t OFF_BIAS = OFF_BAR + 128;
+  static constexpr uint32_t SMEM = OFF_BIAS + FO_C_MAX * 4 + 1024;   // + slack for alignment
   static_assert(OFF_W % 1024 == 0, "the W_out slice is 128B-swizzled");
   static_assert(BOXES_IN_STAGE >= 3 &&
                     (FO_C_MAX / 64 - BOXES_IN_STAGE) * BOX <= FO_C_MAX * FA_ROW_BYTES,
@@ -95,7 +96,7 @@ __global__ void __launch_bounds__(FO_THREADS, 1)
   using FL = FoLayout<H>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
-  const uint32_t sW = base + FL::OFF_W, bars = base + FL::OFF_BAR;
+  const uint32_t sW = base + FL::OFF_W, bars = base + FL::OFF_BAR, sBias = base + FL::OFF_BIAS;
   const uint32_t o_full0 = bars + 8 * FO_STAGES, w_full = bars + 16 * FO_STAGES;
   const uint32_t m_done = w_full + 8, acc_full = w_full + 16, tmem_empty = w_full + 24;
   const uint32_t staged = w_full + 32, drain = w_full + 40, tmem_slot = w_full + 48;
@@ -136,6 +137,9 @@ __global__ void __launch_bounds__(FO_THREADS, 1)
     tmem_alloc(tmem_slot, tmem_cols);
     tmem_relinquish();
   }
+  if ((int)threadIdx.x < C)                       // C <= FO_C_MAX = FO_THREADS
+    asm volatile("st.shared.f32 [%0], %1;" ::"r"(sBias + 4u * threadIdx.x),
+                 "f"(__bfloat162float(b_out[threadIdx.x])));
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -169,15 +173,21 @@ __global__ void __launch_bounds__(FO_THREADS, 1)
         tma_load_2d(sW + (uint32_t)NH * FA_ROW_BYTES, &maps.w, h * 64, NH, w_full);
       };
       // Block i's output, once the attention warps have staged it: one TMA
-      // store per 64 channels (frames past the end are dropped), and the
-      // staging memory back in use only after the stores have read it.
+      // store per 64 channels (frames past the end are dropped), the boxes in
+      // the W_out buffer first, each region in a bulk group of its own, so
+      // that the buffer can be refilled as soon as its boxes have been read.
+      const int n_box = C / 64, n_box_w = n_box > FL::BOXES_IN_STAGE ? n_box - FL::BOXES_IN_STAGE : 0;
       auto store_item = [&](int i) -> bool {
         if (!mbar_wait_bounded(staged, (uint32_t)(i & 1), err_word, VI_DEV_ERR_MMA_TIMEOUT))
           return false;
         int p, f0;
         item_pos(i, p, f0);
-        for (int b = 0; b < C / 64; ++b) tma_store_3d(&maps.y, box_addr(i, b), 64 * b, f0, p);
-        tma_store_commit_and_drain();
+        for (int b = n_box - n_box_w; b < n_box; ++b)
+          tma_store_3d(&maps.y, box_addr(i, b), 64 * b, f0, p);
+        bulk_commit();
+        for (int b = 0; b < n_box - n_box_w; ++b)
+          tma_store_3d(&maps.y, box_addr(i, b), 64 * b, f0, p);
+        bulk_commit();
         return true;
       };
       int n_stage = total < FO_STAGES ? total : FO_STAGES;
@@ -189,20 +199,23 @@ __global__ void __launch_bounds__(FO_THREADS, 1)
         // The MMAs of head g-1 are done: the W_out buffer and the stage of
         // head g-1 (= that of head g+2) are free -- after the stores of the
         // block's output staged there, if head g-1 was a block's last.
+        const bool edge = g % heads == 0;
         if (!mbar_wait_bounded(m_done, (uint32_t)((g - 1) & 1), err_word,
                                VI_DEV_ERR_MMA_TIMEOUT) ||
-            (g % heads == 0 && !store_item(g / heads - 1))) {
+            (edge && !store_item(g / heads - 1))) {
           ok = false;
           break;
         }
+        if (edge) bulk_wait_read_le1();        // the W_out buffer's boxes have been read
         load_w(g);
         ++n_w;
+        if (edge) bulk_wait_read_all();        // and the stage's
         if (g + 2 < total) {
           load_stage(g + 2);
           ++n_stage;
         }
       }
-      if (ok) store_item(my_items - 1);
+      if (ok && store_item(my_items - 1)) bulk_wait_read_all();
       // Every copy issued lands before the CTA may end (on an error path the
       // consumers may have stopped waiting for them).
       for (int s = 0; s < FO_STAGES && s < n_stage; ++s) {
@@ -276,34 +289,42 @@ __global__ void __launch_bounds__(FO_THREADS, 1)
                                                      VI_DEV_ERR_MMA_TIMEOUT));
       if (!ok) break;
       tc_fence_after();
-      // Group by group (32 columns): TMEM -> registers, + b_out, -> bf16
-      // pairs, -> row 32q + lane of the output boxes in the 128-byte swizzle
-      // (chunk j of row r at j ^ (r mod 8)).  The producer stores the boxes.
+      // Group by group (32 columns): TMEM -> registers (the next group's load
+      // in flight meanwhile), + b_out, -> bf16 pairs, -> row 32q + lane of the
+      // output boxes in the 128-byte swizzle (chunk j of row r at j ^ (r mod
+      // 8)).  The producer stores the boxes.  Loops unrolled: registers
+      // indexed at compile time only.
       const uint32_t taddr = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(c * NH);
       const int row = 32 * q + lane;
-      for (int gg = 0; gg < G; ++gg) {
-        uint32_t r[32];
-        tmem_ld32(taddr + 32u * gg, r);
-        // (every warp of every CTA reads the same C bf16: through L1)
-        const uint4* b8 = reinterpret_cast<const uint4*>(bias + 32 * gg);
-        uint4 bv[4];
+      uint32_t ra[32], rb[32];
+      tmem_ld32(taddr, ra);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) bv[e] = __ldg(b8 + e);
+      for (int gg = 0; gg < FO_G_MAX; ++gg) {
+        if (gg >= G) break;
+        uint32_t (&r)[32] = (gg & 1) ? rb : ra;
+        uint32_t (&rn)[32] = (gg & 1) ? ra : rb;
         tmem_wait_ld_dep(r);
+        if (gg + 1 < G) tmem_ld32(taddr + 32u * (gg + 1), rn);
         const int col = c * NH + 32 * gg;
-        const uint32_t rb = box_addr(i, col / 64) + (uint32_t)row * FA_ROW_BYTES;
+        const uint32_t rowb = box_addr(i, col / 64) + (uint32_t)row * FA_ROW_BYTES;
         const int j0 = (col % 64) / 8;           // first 16-byte chunk of the group
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
+          float bv[8];                           // (the same address in every lane)
+          asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];"
+                       : "=f"(bv[0]), "=f"(bv[1]), "=f"(bv[2]), "=f"(bv[3])
+                       : "r"(sBias + 4u * (col + 8 * e)));
+          asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];"
+                       : "=f"(bv[4]), "=f"(bv[5]), "=f"(bv[6]), "=f"(bv[7])
+                       : "r"(sBias + 4u * (col + 8 * e + 4)));
           uint32_t w[4];
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            const int t = 4 * e + u;               // bf16 pair t of the group
-            const uint32_t bw = u == 0 ? bv[e].x : u == 1 ? bv[e].y : u == 2 ? bv[e].z : bv[e].w;
-            w[u] = pack2_bf16(__uint_as_float(r[2 * t]) + __uint_as_float(bw << 16),
-                              __uint_as_float(r[2 * t + 1]) + __uint_as_float(bw & 0xFFFF0000u));
+            const int t = 8 * e + 2 * u;           // column t of the group
+            w[u] = pack2_bf16(__uint_as_float(r[t]) + bv[2 * u],
+                              __uint_as_float(r[t + 1]) + bv[2 * u + 1]);
           }
-          sts128(rb + ((uint32_t)((j0 + e) ^ (row & 7)) << 4), make_uint4(w[0], w[1], w[2], w[3]));
+          sts128(rowb + ((uint32_t)((j0 + e) ^ (row & 7)) << 4), make_uint4(w[0], w[1], w[2], w[3]));
         }
       }
       tc_fence_before();

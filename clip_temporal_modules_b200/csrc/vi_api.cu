@@ -577,6 +577,37 @@ int vitest_temporal_attention_form(const void* x, const void* w_qkv, const void*
                                   d, n_pre, n_post, n_global, stream, form);
 }
 
+// Test hook, not part of the ABI in vi.h: the attention kernel with the
+// output projection fused in, on given q, k, v (bf16 [P][F][C]):
+// out = dual_attn(q, k, v) W_out^T + b_out.  Shapes outside the fused kernel's
+// (those of the attention fast path with C <= 320) return VI_ERR_UNSUPPORTED.
+int vitest_dual_attn_oproj(const void* q, const void* k, const void* v, const void* w_out,
+                           const void* b_out, void* out, int F, int N, int P, int heads, int d,
+                           int n_pre, int n_post, int n_global, vi_stream_t stream) {
+  using T = bf16;
+  if (heads <= 0 || d <= 0 || (int64_t)heads * d > 0x7fffffff) return VI_ERR_INVALID_ARG;
+  const int C = heads * d;
+  int st = check_clips(F, N, P, C);
+  if (st < 0) return st;
+  const int L = F / N;
+  if (n_pre < 0 || n_post < 0 || n_global < 0 || n_global > F) return VI_ERR_INVALID_ARG;
+  if (N > 1 && (n_pre > L || n_post > L)) return VI_ERR_INVALID_ARG;
+  if (!dual_attn_oproj_ok(F, N, d, heads, n_pre, n_post, n_global)) return VI_ERR_UNSUPPORTED;
+  if (st == kEmpty) return VI_OK;
+  if (!q || !k || !v || !w_out || !b_out || !out) return VI_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(w_out) ||
+      !aligned16(b_out) || !aligned16(out))
+    return VI_ERR_ALIGNMENT;
+  const size_t S = (size_t)P * F * C * sizeof(T), cc = (size_t)C * C * sizeof(T);
+  if (overlaps(out, S, q, S) || overlaps(out, S, k, S) || overlaps(out, S, v, S) ||
+      overlaps(out, S, w_out, cc) || overlaps(out, S, b_out, C * sizeof(T)))
+    return VI_ERR_INVALID_ARG;
+  return dual_attn_oproj_bf16_launch(static_cast<const T*>(q), static_cast<const T*>(k),
+                                     static_cast<const T*>(v), static_cast<const T*>(w_out),
+                                     static_cast<const T*>(b_out), static_cast<T*>(out), F, N, P,
+                                     heads, n_pre, n_post, n_global, as_stream(stream));
+}
+
 // Test hook, not part of the ABI in vi.h: vi_groupnorm_conv with the conv's
 // job form forced (tiles 1, 2 or 4, as above).
 int vitest_groupnorm_conv_tiles(const void* x, const void* gamma, const void* beta,

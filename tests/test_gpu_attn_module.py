@@ -82,6 +82,38 @@ def test_both_forms_elementwise(cuda_device, w, fused):
     run_case(w, fused=fused)
 
 
+def oproj_case(w, positions=None):
+    """The fused kernel alone on q, k, v: out = bf16(a) W_out^T + b_out with a the
+    dual-domain attention, against the oracle's attention rounded to bf16 (the
+    operand the kernel hands the tensor core) and its single-tap projection."""
+    from clip_temporal_modules_b200._binding import dual_attn_oproj
+    q, k, v, wo, bo = (synth.make(w, t) for t in ("q", "k", "v", "w_out", "b_out"))
+    dq, dk, dv, dwo, dbo = (to_device(a, w.dtype) for a in (q, k, v, wo, bo))
+    out = dual_attn_oproj(dq, dk, dv, dwo, dbo, N=w.N, heads=w.heads, n_pre=w.n_pre,
+                          n_post=w.n_post, n_global=w.n_global)
+    torch.cuda.synchronize()
+    vi.take_device_errors()
+    got = from_device(out)
+    a = oracle.dual_attn(q, k, v, w.F, w.N, w.heads, w.d, w.n_pre, w.n_post, w.n_global,
+                         positions=positions)
+    a = np.ascontiguousarray(oracle.round_bf16(a), dtype=np.float32)
+    ref = oracle.temporal_conv(a, np.ascontiguousarray(wo).reshape(w.C, w.C, 1),
+                               np.ascontiguousarray(bo), w.F, w.N, 1)
+    if positions is not None:
+        got = got[positions]
+    return assert_close(got, ref, w.dtype, "attn", w.name)
+
+
+@pytest.mark.parametrize("w", FUSED, ids=lambda w: w.name)
+def test_fused_kernel_alone_elementwise(cuda_device, w):
+    oproj_case(w)
+
+
+def test_fused_kernel_alone_full_size_sampled_positions(cuda_device):
+    w = synth.BY_NAME["bf16_F1024_P2560_C320"]
+    oproj_case(w, positions=sample_positions(w.P, count=3))
+
+
 def test_fused_form_refuses_more_than_five_heads(cuda_device):
     """Six heads (C = 384) exceed the fused kernel's TMEM and shared-memory plan:
     the forced fused form is refused before any launch, and the library's
