@@ -51,3 +51,40 @@ def test_step_replays_from_a_cuda_graph(cuda_device):
         assert np.array_equal(out[n].cpu().view(torch.int16).numpy(),
                               eager[n].cpu().view(torch.int16).numpy()), n
     del g
+
+
+def test_attention_module_replays_from_a_cuda_graph(cuda_device):
+    """The attention module (q/k/v GEMM, then the attention with the output
+    projection fused in, a persistent kernel) captured with a caller-owned
+    workspace and replayed: the replays equal the eager result bit for bit."""
+    w = synth.Workload("graph_bf16_F256_P16_C320", "bf16", F=256, N=16, P=16, C=320, heads=5,
+                       d=64)
+    x, wq, bq, wo, bo = (to_device(synth.make(w, n), w.dtype)
+                         for n in ("attn_x", "w_qkv", "b_qkv", "w_out", "b_out"))
+    out = torch.empty_like(x)
+    n = int(vi.lib().vi_temporal_attention_workspace_bytes(w.F, w.P, w.C))
+    ws = torch.empty(n // 2, dtype=torch.bfloat16, device=x.device)
+
+    def step(stream):
+        vi.temporal_attention(x, wq, bq, wo, bo, out, ws, N=w.N, heads=w.heads, stream=stream)
+
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        step(s)
+    s.synchronize()
+    eager = out.clone()
+
+    g = torch.cuda.CUDAGraph()
+    n0 = vi.launch_count()
+    with torch.cuda.graph(g, stream=s):
+        step(s)
+    assert vi.launch_count() - n0 == 3           # weight pack, q/k/v GEMM, fused attention
+    out.zero_()
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    vi.take_device_errors()
+    assert np.array_equal(out.cpu().view(torch.int16).numpy(),
+                          eager.cpu().view(torch.int16).numpy())
+    del g

@@ -86,3 +86,20 @@ def test_groupnorm_beyond_2_31_elements(cuda_device):
     check(y, lambda ps: ref_all[ps], w.dtype, "gn", "GroupNorm, 2.18e9 elements")
     del dx, y
     free()
+
+
+def test_attention_module_beyond_2_31_elements(cuda_device):
+    """The attention module (q/k/v GEMM, then the attention with the output
+    projection fused in): per position, so the repeated block applies."""
+    w = BASE
+    names = ("attn_x", "w_qkv", "b_qkv", "w_out", "b_out")
+    x, wq, bq, wo, bo = (synth.make(w, t) for t in names)
+    dx = big(x, w.dtype)
+    out = vi.temporal_attention(dx, *(to_device(a, w.dtype) for a in (wq, bq, wo, bo)), N=w.N,
+                                heads=w.heads)
+    vi.take_device_errors()
+    check(out, lambda ps: oracle.temporal_attention(x, wq, bq, wo, bo, w.F, w.N, w.heads, w.d,
+                                                    positions=ps),
+          w.dtype, "attn", "attention module, 2.18e9 elements")
+    del dx, out
+    free()

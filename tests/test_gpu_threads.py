@@ -20,7 +20,8 @@ def _inputs(seed):
     w = synth.Workload("thr_bf16_F128_P8_C320", "bf16", F=128, N=8, P=8, C=320, heads=5, d=64,
                        seed=seed)
     return w, {n: to_device(synth.make(w, n), w.dtype) for n in
-               ("q", "k", "v", "conv_x", "conv_w", "conv_b", "gn_x", "gn_gamma", "gn_beta")}
+               ("q", "k", "v", "conv_x", "conv_w", "conv_b", "gn_x", "gn_gamma", "gn_beta",
+                "attn_x", "w_qkv", "b_qkv", "w_out", "b_out")}
 
 
 def _step(w, d, stream):
@@ -29,8 +30,11 @@ def _step(w, d, stream):
         y = vi.temporal_conv(d["conv_x"], d["conv_w"], d["conv_b"], N=w.N, stream=stream)
         z = vi.groupnorm_global(d["gn_x"], d["gn_gamma"], d["gn_beta"], N=w.N, groups=w.groups,
                                 stream=stream)
+        # the attention module: q/k/v GEMM, then the persistent fused kernel
+        m = vi.temporal_attention(d["attn_x"], d["w_qkv"], d["b_qkv"], d["w_out"], d["b_out"],
+                                  N=w.N, heads=w.heads, stream=stream)
     stream.synchronize()
-    return [t.cpu().view(torch.int16).numpy() for t in (a, y, z)]
+    return [t.cpu().view(torch.int16).numpy() for t in (a, y, z, m)]
 
 
 def test_concurrent_host_threads_match_serial_results(cuda_device):
@@ -56,7 +60,8 @@ def test_concurrent_host_threads_match_serial_results(cuda_device):
     assert not errors, errors
     vi.take_device_errors()
     for i in range(len(cases)):
-        # attention and GroupNorm are deterministic; the conv's summation order
-        # depends only on the grid, which is the same for every call here
+        # attention and GroupNorm are deterministic; the conv's and the
+        # module's summation orders depend only on their grids, which are the
+        # same for every call here
         for g, s in zip(got[i], serial[i]):
             assert np.array_equal(g, s)
