@@ -538,7 +538,8 @@ def attn_ablations(w, d, out, y, z, stream, reps=10):
 
 def attn_generic_path(w, d, out, stream, reps=2):
     """The same attention with n_global = 32, outside the tensor-core fast
-    path (which takes L = 16, d = 64, n_pre, n_post <= 16, n_global <= 16):
+    path (which takes d = 64, n_global <= 16, and clips of 16 frames with
+    n_pre, n_post <= 16 or of 8 with n_pre, n_post <= 8):
     one warp per query frame on CUDA cores.  Reported so that the cost off
     the fast path is visible, not as a tuned figure."""
     import torch
@@ -688,13 +689,18 @@ def attention_module(w, d, out, y, z, stream, reps=3):
         run()
         run_unfused()
         run_kernel()
-    # Three interleaved rounds of each; the median round of each.
-    fused, unfused, kern = [], [], []
-    with ClockSampler(dev.index if dev.index is not None else 0) as clocks:
+    # Three interleaved rounds of each; the median round of each.  The clock is
+    # sampled every 5 ms per round: the module draws enough power that the
+    # power cap can lower the clock within a few tens of milliseconds.
+    fused, unfused, kern, round_clocks = [], [], [], []
+    idx = dev.index if dev.index is not None else 0
+    with ClockSampler(idx) as clocks:
         for _ in range(3):
-            fused.append(timed(run))
-            unfused.append(timed(run_unfused))
-            kern.append(timed(run_kernel))
+            with ClockSampler(idx, period_s=0.005) as rc:
+                fused.append(timed(run))
+                unfused.append(timed(run_unfused))
+                kern.append(timed(run_kernel))
+            round_clocks.append(rc.summary())
     ms, ms_unfused, ms_kern = sorted(fused)[1], sorted(unfused)[1], sorted(kern)[1]
     del ws
     flops = 4 * 2 * w.C * w.C * w.tokens
@@ -711,6 +717,8 @@ def attention_module(w, d, out, y, z, stream, reps=3):
             "attention_oproj_kernel": {"ms": round(ms_kern, 4),
                                        "GB/s": round(4 * S / (ms_kern / 1e3) / 1e9, 1)},
             "attention_then_output_gemm_rounds_ms": [round(t, 4) for t in unfused],
+            "round_sm_mhz": [c.get("sm_mhz") for c in round_clocks],
+            "round_reasons": [c.get("reasons") for c in round_clocks],
             "clocks": clocks.summary()}
 
 

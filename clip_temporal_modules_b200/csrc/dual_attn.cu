@@ -13,19 +13,22 @@
 // kernel grid: a CTA owns a run of clips of one (position, head), and the
 // neighbours' frames are simply the adjacent rows of the [P][F][C] layout.
 //
-// Fast path (bf16, L = 16, d = 64, n_pre, n_post <= 8, n_global <= 16):
-//   CTA = (position p, block of 8 clips = 128 frames, head h), 8 warps.
-//   One thread issues five TMA loads (128B-swizzled, one mbarrier):
+// Fast path (bf16, d = 64, n_global <= 16; clips of L = 16 frames with
+// n_pre, n_post <= 16, or of L = 8 with n_pre, n_post <= 8):
+//   CTA = (position p, block of 128 frames, head h), 8 warps.
+//   One thread issues five TMA loads (128B-swizzled, one mbarrier), for a
+//   window of H = 8 rows each side (H = 16 where a context exceeds 8):
 //     Q   rows f0 .. f0+127                       16 KB
-//     K,V rows f0-8 .. f0+135 ("window")          18 KB each
+//     K,V rows f0-H .. f0+127+H ("window")        18 KB each (H = 8)
 //     K,V rows j*stride, j < 16 ("global")         2 KB each
 //   Rows outside [0, F) arrive as zeros and are masked out of the softmax.
-//   Warp w owns clip 8*blk + w: its 48 keys are window rows 16w .. 16w+31
-//   (C_pre | own | C_post) plus the 16 global rows.  S = Q K^T and O = P V
-//   run on tensor cores (mma.sync m16n8k16, bf16 in, fp32 accumulate: 24 +
-//   24 instructions per warp), the softmax in fp32 registers with quad
-//   shuffles; P is rounded to bf16 for the PV product and the row sums use
-//   the rounded values.  O goes back through the Q buffer and one TMA store.
+//   Warp w owns query rows 16w .. 16w+15 (one clip of 16 frames, or two of
+//   8) and window rows 16w .. 16w+2H+15 (C_pre | own | C_post of its clips)
+//   plus the 16 global rows.  S = Q K^T and O = P V run on tensor cores
+//   (mma.sync m16n8k16, bf16 in, fp32 accumulate: 24 + 24 instructions per
+//   warp at H = 8), the softmax in fp32 registers with quad shuffles; P is
+//   rounded to bf16 for the PV product and the row sums use the rounded
+//   values.  O goes back through the Q buffer and one TMA store.
 //   HBM traffic per token and head: q, k, v, out once each (4 x 128 B); the
 //   halo and global rows are re-read by neighbouring CTAs from L2.
 // Generic path (fp32 I/O, or shapes outside the fast path): one warp per
@@ -139,8 +142,9 @@ struct FaMaps {
 //
 // H: halo rows on each side of the CTA's 128 frames (the key list of a clip
 // is H window rows before it, its own 16, H after it, then the 16 global
-// frames: 2H + 32 keys, in n-tiles of 8).
-template <int H>
+// frames: 2H + 32 keys, in n-tiles of 8).  LQ: frames per clip, 16 (one clip
+// per warp) or 8 (two per warp, H = 8).
+template <int H, int LQ = FA_L>
 __global__ void __launch_bounds__(256) dual_attn_bf16_mma(const __grid_constant__ FaMaps maps,
                                                           int F, int N, int heads, int sel_lo,
                                                           int sel_hi0, int n_sel, int n_pre,
@@ -179,11 +183,12 @@ __global__ void __launch_bounds__(256) dual_attn_bf16_mma(const __grid_constant_
   }
   if (!mbar_wait_bounded(bar, 0, err_word, VI_DEV_ERR_TMA_TIMEOUT)) return;
 
-  const int clip = blk * FA_CLIPS + warp;
+  // The warp's (first) clip; clips of 8 frames come two to a warp.
+  const int clip = (blk * FA_ROWS_Q + warp * 16) / LQ;
   if (clip < N) {
     const int gclip = clip0 + clip;              // index in the whole video
-    fa_attend_warp<H>(sQ, sKW, sVW, sKG, sVG, warp, lane, gclip, n_total, n_pre, n_post,
-                      n_global, scale_log2);
+    fa_attend_warp<H, LQ>(sQ, sKW, sVW, sKG, sVG, warp, lane, gclip, n_total, n_pre, n_post,
+                          n_global, scale_log2);
   }
   fence_proxy_async_smem();
   __syncthreads();
@@ -198,15 +203,15 @@ bool encode_tmap(CUtensorMap* map, const void* base, int rank, const uint64_t* d
                  const uint64_t* strides_bytes, const uint32_t* box, CUtensorMapSwizzle swz,
                  CUtensorMapDataType dt);
 
-// Raise the kernel's shared-memory limit once per device and halo width.
-template <int H>
+// Raise the kernel's shared-memory limit once per device and kernel instance.
+template <int H, int LQ>
 static int fa_prepare() {
   static std::atomic<bool> attr_set[64] = {};
   int dev = 0;
   VI_CUDA_TRY(cudaGetDevice(&dev));
   if (dev < 0 || dev >= 64 || !attr_set[dev].load(std::memory_order_acquire)) {
     // Idempotent, so concurrent first calls may both set it.
-    VI_CUDA_TRY(cudaFuncSetAttribute(dual_attn_bf16_mma<H>,
+    VI_CUDA_TRY(cudaFuncSetAttribute(dual_attn_bf16_mma<H, LQ>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      FaLayout<H>::SMEM));
     if (dev >= 0 && dev < 64) attr_set[dev].store(true, std::memory_order_release);
@@ -214,7 +219,7 @@ static int fa_prepare() {
   return VI_OK;
 }
 
-template <int H>
+template <int H, int LQ>
 static int fa_fast_launch(const bf16* q, const bf16* k, const bf16* v, bf16* out, int F, int N,
                           int P, int heads, int n_pre, int n_post, int n_global,
                           cudaStream_t stream) {
@@ -241,29 +246,35 @@ static int fa_fast_launch(const bf16* q, const bf16* k, const bf16* v, bf16* out
     maps.vg = maps.v;
   }
   if (!ok) return VI_ERR_CUDA;
-  int st = fa_prepare<H>();
+  int st = fa_prepare<H, LQ>();
   if (st != VI_OK) return st;
-  const int nblk = (N + FA_CLIPS - 1) / FA_CLIPS;
+  const int cpb = FA_ROWS_Q / LQ;                 // clips per block of 128 frames
+  const int nblk = (N + cpb - 1) / cpb;
   const int64_t grid = (int64_t)P * heads * nblk;
   if (grid > 0x7fffffff) return VI_ERR_UNSUPPORTED;
   const float scale_log2 = 1.4426950408889634f / 8.0f;    // log2(e) / sqrt(64)
   unsigned int* err = device_error_word();
   if (!err) return VI_ERR_CUDA;
-  dual_attn_bf16_mma<H><<<(unsigned)grid, 256, FaLayout<H>::SMEM, stream>>>(
+  dual_attn_bf16_mma<H, LQ><<<(unsigned)grid, 256, FaLayout<H>::SMEM, stream>>>(
       maps, F, N, heads, nblk, 0, nblk, n_pre, n_post, n_global, scale_log2, 0, 0, N, err);
   VI_LAUNCHED();
   return VI_OK;
 }
 
-// The whole video on one GPU: the narrower window (8 rows each side) where
-// both context sizes fit it, else the 16-row one.
+// The whole video on one GPU.  Clips of 16 frames: the narrower window (8
+// rows each side) where both context sizes fit it, else the 16-row one; clips
+// of 8 frames: the 8-row window, two clips per warp.
 int dual_attn_bf16_fast(const bf16* q, const bf16* k, const bf16* v, bf16* out, int F, int N,
                         int P, int heads, int n_pre, int n_post, int n_global,
                         cudaStream_t stream) {
+  if (F / N == 8)
+    return fa_fast_launch<FA_HALO, 8>(q, k, v, out, F, N, P, heads, n_pre, n_post, n_global,
+                                      stream);
   if (n_pre <= FA_HALO && n_post <= FA_HALO)
-    return fa_fast_launch<FA_HALO>(q, k, v, out, F, N, P, heads, n_pre, n_post, n_global, stream);
-  return fa_fast_launch<FA_HALO_MAX>(q, k, v, out, F, N, P, heads, n_pre, n_post, n_global,
-                                     stream);
+    return fa_fast_launch<FA_HALO, FA_L>(q, k, v, out, F, N, P, heads, n_pre, n_post, n_global,
+                                         stream);
+  return fa_fast_launch<FA_HALO_MAX, FA_L>(q, k, v, out, F, N, P, heads, n_pre, n_post, n_global,
+                                           stream);
 }
 
 // One shard of a video cut along frames (clip-parallel over several GPUs):
@@ -301,7 +312,7 @@ int dual_attn_bf16_shard(const bf16* q, const bf16* k_ext, const bf16* v_ext, co
     maps.vg = maps.v;
   }
   if (!ok) return VI_ERR_CUDA;
-  int st = fa_prepare<FA_HALO>();
+  int st = fa_prepare<FA_HALO, FA_L>();
   if (st != VI_OK) return st;
   const int nblk = (N_loc + FA_CLIPS - 1) / FA_CLIPS;
   // Interior blocks [a, b): their k/v window (8 rows on each side of the
@@ -319,16 +330,19 @@ int dual_attn_bf16_shard(const bf16* q, const bf16* k_ext, const bf16* v_ext, co
   const float scale_log2 = 1.4426950408889634f / 8.0f;    // log2(e) / sqrt(64)
   unsigned int* err = device_error_word();
   if (!err) return VI_ERR_CUDA;
-  dual_attn_bf16_mma<FA_HALO><<<(unsigned)grid, 256, FaLayout<FA_HALO>::SMEM, stream>>>(
+  dual_attn_bf16_mma<FA_HALO, FA_L><<<(unsigned)grid, 256, FaLayout<FA_HALO>::SMEM, stream>>>(
       maps, F_loc, N_loc, heads, sel_lo, sel_hi0, n_sel, n_pre, n_post, n_global, scale_log2,
       FA_HALO, clip0, N, err);
   VI_LAUNCHED();
   return VI_OK;
 }
 
+// Clips of 16 frames with up to 16 context frames on each side, or of 8 with
+// up to 8; at most 16 global frames; d = 64.
 bool dual_attn_fast_ok(int F, int N, int d, int n_pre, int n_post, int n_global) {
-  return d == 64 && F / N == FA_L && n_pre <= FA_HALO_MAX && n_post <= FA_HALO_MAX &&
-         n_global <= FA_NG;
+  const int L = F / N;
+  const int ctx = L == FA_L ? FA_HALO_MAX : L == 8 ? FA_HALO : -1;
+  return d == 64 && ctx >= 0 && n_pre <= ctx && n_post <= ctx && n_global <= FA_NG;
 }
 
 // A shard's k/v storage carries FA_HALO rows of its neighbours on each side.

@@ -12,10 +12,11 @@
 // The attention kernel followed by the output GEMM writes a to HBM and reads
 // it back: 2 x 2 bytes per channel and token on top of q, k, v and out.  Here
 // a never leaves the SM.
-//   Work item = (position p, block of 8 clips = 128 frames), every head.  One
+//   Work item = (position p, block of 128 frames), every head.  One
 //   persistent CTA per SM walks its items; 10 warps:
-//     warps 0-7  the attention (warp w: clip 8*blk + w, the same per-warp code
-//                as the attention kernel), then the block's epilogue;
+//     warps 0-7  the attention (warp w: frames 16w .. 16w+15 of the block, one
+//                clip of 16 frames or two of 8, the same per-warp code as
+//                the attention kernel), then the block's epilogue;
 //     warp 8     TMA producer: per head, its stage (Q, K/V window, K/V global)
 //                into a ring of 3 stages that runs on across blocks, and the
 //                columns 64h .. 64h+63 of W_out (C rows x 128 bytes) into one
@@ -83,11 +84,11 @@ struct FoMaps {
   CUtensorMap y;                 // out [P][F][C]: box of 64 channels x 128 frames
 };
 
-// Persistent: CTA c walks the blocks (position p, 8 clips) c, c + grid, ...
-// of the video (N clips of L = 16 frames, P positions); global head g of the
-// CTA is head g % heads of its block g / heads, staged in stage g % 3.
+// Persistent: CTA c walks the blocks (position p, 128 frames) c, c + grid,
+// ... of the video (N clips of LQ = 16 or 8 frames, P positions); global head
+// g of the CTA is head g % heads of its block g / heads, staged in stage g % 3.
 // tmem_cols: a power of two >= C.
-template <int H>
+template <int H, int LQ>
 __global__ void __launch_bounds__(FO_THREADS, 1)
     dual_attn_oproj_bf16(const __grid_constant__ FoMaps maps, const bf16* __restrict__ b_out,
                          int N, int P, int heads, int n_pre, int n_post, int n_global,
@@ -101,7 +102,8 @@ __global__ void __launch_bounds__(FO_THREADS, 1)
   const uint32_t m_done = w_full + 8, acc_full = w_full + 16, tmem_empty = w_full + 24;
   const uint32_t staged = w_full + 32, drain = w_full + 40, tmem_slot = w_full + 48;
   const int C = heads * 64, NH = C / 2;           // NH: N of one MMA, columns of one warp
-  const int nblk = (N + FA_CLIPS - 1) / FA_CLIPS;
+  const int cpb = FA_ROWS_Q / LQ;                 // clips per block
+  const int nblk = (N + cpb - 1) / cpb;
   const long long n_items = (long long)P * nblk;
   const int my_items = (int)((n_items - blockIdx.x + gridDim.x - 1) / gridDim.x);
   const int total = my_items * heads;             // this CTA's heads, all blocks
@@ -261,13 +263,12 @@ __global__ void __launch_bounds__(FO_THREADS, 1)
     // ------------------------------------------------------------ attention
     const int q = warp & 3, c = warp >> 2;   // epilogue: TMEM lane quarter, column half
     const int G = NH / 32;                   // 32-column groups of this warp (<= FO_G_MAX)
-    const bf16* bias = b_out + c * NH;
     bool ok = true;
     int g = 0;
     for (int i = 0; i < my_items && ok; ++i) {
       int p, f0;
       item_pos(i, p, f0);
-      const int clip = f0 / FA_L + warp;
+      const int clip = (f0 + 16 * warp) / LQ;  // the warp's (first) clip
       for (int h = 0; h < heads; ++h, ++g) {
         const int s = g % FO_STAGES;
         const uint32_t st = base + (uint32_t)s * Lay::STAGE;
@@ -276,7 +277,7 @@ __global__ void __launch_bounds__(FO_THREADS, 1)
                                                        err_word, VI_DEV_ERR_TMA_TIMEOUT));
         if (!ok) break;
         if (clip < N)
-          fa_attend_warp<H>(st + Lay::OFF_Q, st + Lay::OFF_KW, st + Lay::OFF_VW,
+          fa_attend_warp<H, LQ>(st + Lay::OFF_Q, st + Lay::OFF_KW, st + Lay::OFF_VW,
                             st + Lay::OFF_KG, st + Lay::OFF_VG, warp, lane, clip, N, n_pre,
                             n_post, n_global, scale_log2);
         fence_proxy_async_smem();            // O_h is visible to the tensor core
@@ -348,13 +349,13 @@ bool encode_tmap(CUtensorMap* map, const void* base, int rank, const uint64_t* d
                  const uint64_t* strides_bytes, const uint32_t* box, CUtensorMapSwizzle swz,
                  CUtensorMapDataType dt);
 
-template <int H>
+template <int H, int LQ>
 static int fo_prepare() {
   static std::atomic<bool> attr_set[64] = {};
   int dev = 0;
   VI_CUDA_TRY(cudaGetDevice(&dev));
   if (dev < 0 || dev >= 64 || !attr_set[dev].load(std::memory_order_acquire)) {
-    VI_CUDA_TRY(cudaFuncSetAttribute(dual_attn_oproj_bf16<H>,
+    VI_CUDA_TRY(cudaFuncSetAttribute(dual_attn_oproj_bf16<H, LQ>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      FoLayout<H>::SMEM));
     if (dev >= 0 && dev < 64) attr_set[dev].store(true, std::memory_order_release);
@@ -362,7 +363,7 @@ static int fo_prepare() {
   return VI_OK;
 }
 
-template <int H>
+template <int H, int LQ>
 static int fo_launch(const bf16* q, const bf16* k, const bf16* v, const bf16* w_out,
                      const bf16* b_out, bf16* out, int F, int N, int P, int heads, int n_pre,
                      int n_post, int n_global, cudaStream_t stream) {
@@ -396,9 +397,10 @@ static int fo_launch(const bf16* q, const bf16* k, const bf16* v, const bf16* w_
     maps.vg = maps.v;
   }
   if (!ok) return VI_ERR_CUDA;
-  int st = fo_prepare<H>();
+  int st = fo_prepare<H, LQ>();
   if (st != VI_OK) return st;
-  const int nblk = (N + FA_CLIPS - 1) / FA_CLIPS;
+  const int cpb = FA_ROWS_Q / LQ;
+  const int nblk = (N + cpb - 1) / cpb;
   const int64_t n_items = (int64_t)P * nblk;
   const int sms = sm_count();
   if (sms <= 0) return VI_ERR_CUDA;
@@ -411,26 +413,31 @@ static int fo_launch(const bf16* q, const bf16* k, const bf16* v, const bf16* w_
   const float scale_log2 = 1.4426950408889634f / 8.0f;    // log2(e) / sqrt(64)
   unsigned int* err = device_error_word();
   if (!err) return VI_ERR_CUDA;
-  dual_attn_oproj_bf16<H><<<(unsigned)grid, FO_THREADS, FoLayout<H>::SMEM, stream>>>(
+  dual_attn_oproj_bf16<H, LQ><<<(unsigned)grid, FO_THREADS, FoLayout<H>::SMEM, stream>>>(
       maps, b_out, N, P, heads, n_pre, n_post, n_global, scale_log2, tmem_cols, err);
   VI_LAUNCHED();
   return VI_OK;
 }
 
+bool dual_attn_fast_ok(int F, int N, int d, int n_pre, int n_post, int n_global);
+
 // The attention fast path's shapes with at most FO_C_MAX channels.
 bool dual_attn_oproj_ok(int F, int N, int d, int heads, int n_pre, int n_post, int n_global) {
-  return d == 64 && heads >= 1 && heads * 64 <= FO_C_MAX && F / N == FA_L &&
-         n_pre <= FA_HALO_MAX && n_post <= FA_HALO_MAX && n_global <= FA_NG;
+  return heads >= 1 && heads * 64 <= FO_C_MAX &&
+         dual_attn_fast_ok(F, N, d, n_pre, n_post, n_global);
 }
 
 int dual_attn_oproj_bf16_launch(const bf16* q, const bf16* k, const bf16* v, const bf16* w_out,
                                 const bf16* b_out, bf16* out, int F, int N, int P, int heads,
                                 int n_pre, int n_post, int n_global, cudaStream_t stream) {
+  if (F / N == 8)
+    return fo_launch<FA_HALO, 8>(q, k, v, w_out, b_out, out, F, N, P, heads, n_pre, n_post,
+                                 n_global, stream);
   if (n_pre <= FA_HALO && n_post <= FA_HALO)
-    return fo_launch<FA_HALO>(q, k, v, w_out, b_out, out, F, N, P, heads, n_pre, n_post,
-                              n_global, stream);
-  return fo_launch<FA_HALO_MAX>(q, k, v, w_out, b_out, out, F, N, P, heads, n_pre, n_post,
-                                n_global, stream);
+    return fo_launch<FA_HALO, FA_L>(q, k, v, w_out, b_out, out, F, N, P, heads, n_pre, n_post,
+                                    n_global, stream);
+  return fo_launch<FA_HALO_MAX, FA_L>(q, k, v, w_out, b_out, out, F, N, P, heads, n_pre, n_post,
+                                      n_global, stream);
 }
 
 }  // namespace vi

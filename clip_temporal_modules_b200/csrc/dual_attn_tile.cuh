@@ -47,19 +47,23 @@ __device__ __forceinline__ uint32_t sw128(uint32_t region, int row, int chunk) {
   return region + row * FA_ROW_BYTES + (((chunk ^ (row & 7)) & 7) << 4);
 }
 
-// Warp `warp` of the block computes clip `gclip` (its index in the whole
-// video of n_total clips): the 16 query rows 16*warp .. 16*warp+15 of the Q
-// tile, its 2H + 16 window keys (window rows 16*warp .. 16*warp + 2H + 15:
-// C_pre | own | C_post) and the 16 global keys, and writes its 16 rows of O
-// (bf16, normalised) over the same rows of the Q tile, in the tile's 128-byte
-// swizzle.
+// Warp `warp` of the block computes the 16 query rows 16*warp .. 16*warp+15
+// of the Q tile against the 2H + 16 window rows 16*warp .. 16*warp + 2H + 15
+// and the 16 global keys, and writes its 16 rows of O (bf16, normalised) over
+// the same rows of the Q tile, in the tile's 128-byte swizzle.
+//   LQ = 16 (clips of 16 frames): the rows are clip `gclip` (its index in the
+//   whole video of n_total clips), its window keys C_pre | own | C_post.
+//   LQ = 8 (clips of 8 frames, H = 8): rows 0-7 are clip gclip and rows 8-15
+//   clip gclip + 1; their windows (8 | 8 | 8 keys) are window rows 0-23 and
+//   8-31 of the warp's 32.  In the mma.sync accumulator layout a thread holds
+//   rows g and g + 8, one of each clip, so each takes its own clip's mask.
 //   S = Q K^T and O = P V on tensor cores (mma.sync m16n8k16, bf16 in, fp32
 //   accumulate), the softmax in fp32 registers with quad shuffles in log2
 //   units (scale_log2 = log2(e)/sqrt(d)); P is rounded to bf16 for the P V
 //   product and the row sums use the rounded values.  Keys outside the clip's
 //   list (absent ends, n_pre / n_post below H, n_global below 16) are masked
 //   to -inf.  Without global frames their tiles are not read at all.
-template <int H>
+template <int H, int LQ = FA_L>
 __device__ __forceinline__ void fa_attend_warp(uint32_t sQ, uint32_t sKW, uint32_t sVW,
                                                uint32_t sKG, uint32_t sVG, int warp, int lane,
                                                int gclip, int n_total, int n_pre, int n_post,
@@ -68,6 +72,7 @@ __device__ __forceinline__ void fa_attend_warp(uint32_t sQ, uint32_t sKW, uint32
   constexpr int NTW = NW / 8;             // their n-tiles (4 or 6)
   constexpr int NT = NTW + FA_NG / 8;     // all n-tiles (6 or 8)
   constexpr int KS = NT / 2;              // k-steps of P.V (3 or 4)
+  static_assert(LQ == FA_L || (LQ == 8 && H == 8), "clips of 16 frames, or of 8 with H = 8");
   const int g = lane >> 2, qd = lane & 3;
   // ---- S = Q K^T over 2H + 32 keys (NT n-tiles of 8), 4 k-steps of 16 dims ----
   uint32_t qa[4][4];
@@ -101,13 +106,32 @@ __device__ __forceinline__ void fa_attend_warp(uint32_t sQ, uint32_t sKW, uint32
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
       const int kk = nt * 8 + 2 * qd + c;     // key index in the warp's list
-      bool valid;
-      if (kk < H) valid = gclip > 0 && kk >= H - n_pre;
-      else if (kk < H + FA_L) valid = true;
-      else if (kk < NW) valid = gclip < n_total - 1 && kk - (H + FA_L) < n_post;
-      else valid = kk - NW < n_global;
-      s[nt][c] = valid ? s[nt][c] * scale_log2 : -INFINITY;
-      s[nt][c + 2] = valid ? s[nt][c + 2] * scale_log2 : -INFINITY;
+      bool v0, v1;                            // for rows g and g + 8
+      if (kk >= NW) {
+        v0 = v1 = kk - NW < n_global;
+      } else if constexpr (LQ == FA_L) {
+        if (kk < H) v0 = gclip > 0 && kk >= H - n_pre;
+        else if (kk < H + FA_L) v0 = true;
+        else v0 = gclip < n_total - 1 && kk - (H + FA_L) < n_post;
+        v1 = v0;
+      } else {
+        // clip gclip + hr sees window keys 8hr .. 8hr + 23 as pre | own | post
+        // (a clip past the video's last has no rows in the output: its own
+        // keys keep its softmax finite)
+        bool v[2];
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr) {
+          const int gc = gclip + hr, kl = kk - 8 * hr;
+          if (kl < 0 || kl >= 24) v[hr] = false;
+          else if (kl < 8) v[hr] = gc > 0 && kl >= 8 - n_pre;
+          else if (kl < 16) v[hr] = true;
+          else v[hr] = gc < n_total - 1 && kl - 16 < n_post;
+        }
+        v0 = v[0];
+        v1 = v[1];
+      }
+      s[nt][c] = v0 ? s[nt][c] * scale_log2 : -INFINITY;
+      s[nt][c + 2] = v1 ? s[nt][c + 2] * scale_log2 : -INFINITY;
       mx0 = fmaxf(mx0, s[nt][c]);
       mx1 = fmaxf(mx1, s[nt][c + 2]);
     }

@@ -48,8 +48,18 @@ SMALL = [
     W("bf16_halo12_2blk_ragged", "bf16", 160, 10, 3, 2, n_pre=12, n_post=9, n_global=7),
     W("bf16_halo_mixed", "bf16", 96, 6, 2, 1, n_pre=4, n_post=13, n_global=16),
     W("bf16_halo16_no_global", "bf16", 48, 3, 2, 1, n_pre=16, n_post=10, n_global=0),
-    W("bf16_L8_generic", "bf16", 32, 4, 4, 2),                 # L = 8: generic path
+    # clips of 8 frames on the fast path: two clips per warp, each its own mask
+    W("bf16_L8_1blk_ragged", "bf16", 40, 5, 5, 2),             # warps (0,1) (2,3) (4,-)
+    W("bf16_L8_2blk_ragged", "bf16", 200, 25, 3, 3),           # 16 + 9 clips
+    W("bf16_L8_two_clips", "bf16", 16, 2, 4, 1, n_global=2),
+    W("bf16_L8_one_clip", "bf16", 8, 1, 6, 2, n_global=4),
+    W("bf16_L8_short_ctx", "bf16", 64, 8, 4, 2, n_pre=3, n_post=5, n_global=7),
+    W("bf16_L8_one_sided", "bf16", 96, 12, 3, 1, n_pre=0, n_post=8, n_global=0),
+    W("bf16_L8_pre_only", "bf16", 48, 6, 2, 1, n_pre=8, n_post=1, n_global=16),
+    # shapes outside the fast path: the generic kernel
+    W("bf16_L4_generic", "bf16", 32, 8, 4, 2, n_pre=4, n_post=4),
     W("bf16_L32_generic", "bf16", 64, 2, 3, 1, n_pre=16, n_post=12, n_global=20),
+    W("bf16_L8_global20_generic", "bf16", 64, 8, 2, 1, n_global=20),
     W("f32_generic", "f32", 48, 3, 3, 2),
     W("f32_L16_short", "f32", 64, 4, 2, 1, n_pre=2, n_post=0, n_global=5),
 ]
@@ -63,6 +73,12 @@ def test_small_elementwise(cuda_device, w):
 @pytest.mark.parametrize("w", synth.WORKLOADS[1:], ids=lambda w: w.name)
 def test_full_size_sampled_positions(cuda_device, w):
     run_case(w, positions=sample_positions(w.P))
+
+
+def test_clips_of_8_frames_at_size(cuda_device):
+    """F = 1024 in 128 clips of 8 frames (the fast path, two clips per warp)."""
+    w = W("bf16_F1024_N128_P64_C320_L8", "bf16", 1024, 128, 64, 5)
+    run_case(w, positions=sample_positions(w.P, count=2))
 
 
 # Ablation settings of the write-up's study (attention without global context,

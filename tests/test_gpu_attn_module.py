@@ -52,7 +52,7 @@ def W(name, F, N, P, heads, **kw):
 
 SMALL = [
     W("attnmod_F160_N10_P3_h2", 160, 10, 3, 2),          # fast attention path, 2 blocks
-    W("attnmod_F32_N4_P4_h1_L8", 32, 4, 4, 1),            # generic attention path
+    W("attnmod_F32_N8_P4_h1_L4", 32, 8, 4, 1, n_pre=4, n_post=4),   # generic attention path
     W("attnmod_F64_N4_P2_h5_ctx", 64, 4, 2, 5, n_pre=3, n_post=5, n_global=7),
 ]
 
@@ -68,6 +68,7 @@ FUSED = [
     W("attnmod_fused_F128_N8_P3_h4", 128, 8, 3, 4),
     W("attnmod_fused_F288_N18_P2_h5_halo16", 288, 18, 2, 5, n_pre=12, n_post=16, n_global=9),
     W("attnmod_fused_F256_N16_P2_h5_ctx", 256, 16, 2, 5, n_pre=0, n_post=3, n_global=16),
+    W("attnmod_fused_F72_N9_P3_h3_L8", 72, 9, 3, 3, n_pre=5, n_post=8, n_global=9),   # 8-frame clips
 ]
 
 
