@@ -14,7 +14,7 @@
 // neighbours' frames are simply the adjacent rows of the [P][F][C] layout.
 //
 // Fast path (bf16, d = 64, n_global <= 16; clips of L = 16 frames with
-// n_pre, n_post <= 16, or of L = 8 with n_pre, n_post <= 8):
+// n_pre, n_post <= 16, or of L = 8 or 32 with n_pre, n_post <= 8):
 //   CTA = (position p, block of 128 frames, head h), 8 warps.
 //   One thread issues five TMA loads (128B-swizzled, one mbarrier), for a
 //   window of H = 8 rows each side (H = 16 where a context exceeds 8):
@@ -22,9 +22,10 @@
 //     K,V rows f0-H .. f0+127+H ("window")        18 KB each (H = 8)
 //     K,V rows j*stride, j < 16 ("global")         2 KB each
 //   Rows outside [0, F) arrive as zeros and are masked out of the softmax.
-//   Warp w owns query rows 16w .. 16w+15 (one clip of 16 frames, or two of
-//   8) and window rows 16w .. 16w+2H+15 (C_pre | own | C_post of its clips)
-//   plus the 16 global rows.  S = Q K^T and O = P V run on tensor cores
+//   Warp w owns query rows 16w .. 16w+15 (one clip of 16 frames, two of 8,
+//   or half of one of 32) and the window rows of its clips' C_pre | own |
+//   C_post (2H + 16 rows from 16w; 48 from 32(w/2) for clips of 32) plus the
+//   16 global rows.  S = Q K^T and O = P V run on tensor cores
 //   (mma.sync m16n8k16, bf16 in, fp32 accumulate: 24 + 24 instructions per
 //   warp at H = 8), the softmax in fp32 registers with quad shuffles; P is
 //   rounded to bf16 for the PV product and the row sums use the rounded
@@ -263,13 +264,17 @@ static int fa_fast_launch(const bf16* q, const bf16* k, const bf16* v, bf16* out
 
 // The whole video on one GPU.  Clips of 16 frames: the narrower window (8
 // rows each side) where both context sizes fit it, else the 16-row one; clips
-// of 8 frames: the 8-row window, two clips per warp.
+// of 8 frames: the 8-row window, two clips per warp; of 32: the 8-row window,
+// two warps per clip.
 int dual_attn_bf16_fast(const bf16* q, const bf16* k, const bf16* v, bf16* out, int F, int N,
                         int P, int heads, int n_pre, int n_post, int n_global,
                         cudaStream_t stream) {
   if (F / N == 8)
     return fa_fast_launch<FA_HALO, 8>(q, k, v, out, F, N, P, heads, n_pre, n_post, n_global,
                                       stream);
+  if (F / N == 32)
+    return fa_fast_launch<FA_HALO, 32>(q, k, v, out, F, N, P, heads, n_pre, n_post, n_global,
+                                       stream);
   if (n_pre <= FA_HALO && n_post <= FA_HALO)
     return fa_fast_launch<FA_HALO, FA_L>(q, k, v, out, F, N, P, heads, n_pre, n_post, n_global,
                                          stream);
@@ -337,11 +342,11 @@ int dual_attn_bf16_shard(const bf16* q, const bf16* k_ext, const bf16* v_ext, co
   return VI_OK;
 }
 
-// Clips of 16 frames with up to 16 context frames on each side, or of 8 with
-// up to 8; at most 16 global frames; d = 64.
+// Clips of 16 frames with up to 16 context frames on each side, or of 8 or
+// 32 with up to 8; at most 16 global frames; d = 64.
 bool dual_attn_fast_ok(int F, int N, int d, int n_pre, int n_post, int n_global) {
   const int L = F / N;
-  const int ctx = L == FA_L ? FA_HALO_MAX : L == 8 ? FA_HALO : -1;
+  const int ctx = L == FA_L ? FA_HALO_MAX : (L == 8 || L == 32) ? FA_HALO : -1;
   return d == 64 && ctx >= 0 && n_pre <= ctx && n_post <= ctx && n_global <= FA_NG;
 }
 

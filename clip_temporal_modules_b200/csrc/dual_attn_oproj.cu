@@ -15,8 +15,9 @@
 //   Work item = (position p, block of 128 frames), every head.  One
 //   persistent CTA per SM walks its items; 10 warps:
 //     warps 0-7  the attention (warp w: frames 16w .. 16w+15 of the block, one
-//                clip of 16 frames or two of 8, the same per-warp code as
-//                the attention kernel), then the block's epilogue;
+//                clip of 16 frames, two of 8 or half of one of 32, the same
+//                per-warp code as the attention kernel), then the block's
+//                epilogue;
 //     warp 8     TMA producer: per head, its stage (Q, K/V window, K/V global)
 //                into a ring of 3 stages that runs on across blocks, and the
 //                columns 64h .. 64h+63 of W_out (C rows x 128 bytes) into one
@@ -85,7 +86,7 @@ struct FoMaps {
 };
 
 // Persistent: CTA c walks the blocks (position p, 128 frames) c, c + grid,
-// ... of the video (N clips of LQ = 16 or 8 frames, P positions); global head
+// ... of the video (N clips of LQ = 8, 16 or 32 frames, P positions); global head
 // g of the CTA is head g % heads of its block g / heads, staged in stage g % 3.
 // tmem_cols: a power of two >= C.
 template <int H, int LQ>
@@ -433,6 +434,9 @@ int dual_attn_oproj_bf16_launch(const bf16* q, const bf16* k, const bf16* v, con
   if (F / N == 8)
     return fo_launch<FA_HALO, 8>(q, k, v, w_out, b_out, out, F, N, P, heads, n_pre, n_post,
                                  n_global, stream);
+  if (F / N == 32)
+    return fo_launch<FA_HALO, 32>(q, k, v, w_out, b_out, out, F, N, P, heads, n_pre, n_post,
+                                  n_global, stream);
   if (n_pre <= FA_HALO && n_post <= FA_HALO)
     return fo_launch<FA_HALO, FA_L>(q, k, v, w_out, b_out, out, F, N, P, heads, n_pre, n_post,
                                     n_global, stream);

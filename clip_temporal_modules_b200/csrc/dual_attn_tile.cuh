@@ -53,6 +53,8 @@ __device__ __forceinline__ uint32_t sw128(uint32_t region, int row, int chunk) {
 // the same rows of the Q tile, in the tile's 128-byte swizzle.
 //   LQ = 16 (clips of 16 frames): the rows are clip `gclip` (its index in the
 //   whole video of n_total clips), its window keys C_pre | own | C_post.
+//   LQ = 32 (H = 8): the rows are half of clip `gclip`, whose 48 window keys
+//   start at window row 32 * (warp / 2).
 //   LQ = 8 (clips of 8 frames, H = 8): rows 0-7 are clip gclip and rows 8-15
 //   clip gclip + 1; their windows (8 | 8 | 8 keys) are window rows 0-23 and
 //   8-31 of the warp's 32.  In the mma.sync accumulator layout a thread holds
@@ -68,11 +70,18 @@ __device__ __forceinline__ void fa_attend_warp(uint32_t sQ, uint32_t sKW, uint32
                                                uint32_t sKG, uint32_t sVG, int warp, int lane,
                                                int gclip, int n_total, int n_pre, int n_post,
                                                int n_global, float scale_log2) {
-  constexpr int NW = 2 * H + FA_L;        // window keys of a clip
-  constexpr int NTW = NW / 8;             // their n-tiles (4 or 6)
-  constexpr int NT = NTW + FA_NG / 8;     // all n-tiles (6 or 8)
-  constexpr int KS = NT / 2;              // k-steps of P.V (3 or 4)
-  static_assert(LQ == FA_L || (LQ == 8 && H == 8), "clips of 16 frames, or of 8 with H = 8");
+  // Window keys of the warp: its clip's (L >= 16: H | L | H), or the union
+  // of its two clips' (L = 8: 32).
+  constexpr int NW = 2 * H + (LQ >= FA_L ? LQ : FA_L);
+  constexpr int NTW = NW / 8;             // their n-tiles
+  constexpr int NT = NTW + FA_NG / 8;     // all n-tiles, the 16 global keys included
+  constexpr int KS = NT / 2;              // k-steps of P.V
+  static_assert(LQ == FA_L || ((LQ == 8 || LQ == 32) && H == 8),
+                "clips of 16 frames, or of 8 or 32 with H = 8");
+  static_assert(NW % 16 == 0, "whole P.V k-steps over the window");
+  // First window row of the warp's keys: its clip's first pre row (L >= 16:
+  // warps 2m and 2m+1 share the clip of L = 32), or its first clip's (L = 8).
+  const int kbase = LQ > FA_L ? (16 * warp / LQ) * LQ : 16 * warp;
   const int g = lane >> 2, qd = lane & 3;
   // ---- S = Q K^T over 2H + 32 keys (NT n-tiles of 8), 4 k-steps of 16 dims ----
   uint32_t qa[4][4];
@@ -90,7 +99,7 @@ __device__ __forceinline__ void fa_attend_warp(uint32_t sQ, uint32_t sKW, uint32
     s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
     if (nt >= NTW && !has_global) continue;
     const uint32_t region = nt < NTW ? sKW : sKG;
-    const int row = nt < NTW ? warp * 16 + nt * 8 + (lane & 7) : (nt - NTW) * 8 + (lane & 7);
+    const int row = nt < NTW ? kbase + nt * 8 + (lane & 7) : (nt - NTW) * 8 + (lane & 7);
 #pragma unroll
     for (int kp = 0; kp < 2; ++kp) {
       uint32_t b0, b1, b2, b3;
@@ -109,10 +118,10 @@ __device__ __forceinline__ void fa_attend_warp(uint32_t sQ, uint32_t sKW, uint32
       bool v0, v1;                            // for rows g and g + 8
       if (kk >= NW) {
         v0 = v1 = kk - NW < n_global;
-      } else if constexpr (LQ == FA_L) {
+      } else if constexpr (LQ >= FA_L) {
         if (kk < H) v0 = gclip > 0 && kk >= H - n_pre;
-        else if (kk < H + FA_L) v0 = true;
-        else v0 = gclip < n_total - 1 && kk - (H + FA_L) < n_post;
+        else if (kk < H + LQ) v0 = true;
+        else v0 = gclip < n_total - 1 && kk - (H + LQ) < n_post;
         v1 = v0;
       } else {
         // clip gclip + hr sees window keys 8hr .. 8hr + 23 as pre | own | post
@@ -166,7 +175,7 @@ __device__ __forceinline__ void fa_attend_warp(uint32_t sQ, uint32_t sKW, uint32
   for (int ks = 0; ks < KS; ++ks) {
     if (ks == KS - 1 && !has_global) continue;
     const uint32_t region = ks < KS - 1 ? sVW : sVG;
-    const int row = (ks < KS - 1 ? warp * 16 + ks * 16 : 0) + (lane & 15);
+    const int row = (ks < KS - 1 ? kbase + ks * 16 : 0) + (lane & 15);
 #pragma unroll
     for (int nd = 0; nd < 8; nd += 2) {
       uint32_t b0, b1, b2, b3;

@@ -114,12 +114,12 @@ int vi_selftest_wait_timeout(int limit_us, vi_stream_t stream);
  *                n_global <= F.  Otherwise VI_ERR_INVALID_ARG, or
  *                VI_ERR_UNSUPPORTED for d != 64.
  * Paths        : bf16 with n_global <= 16 and either L == 16 with n_pre,
- *                n_post <= 16 or L == 8 with n_pre, n_post <= 8 (context up
- *                to a whole clip) runs on tensor cores (TMA-staged blocks,
- *                mma.sync; an 8-row window on each side when both context
- *                sizes are <= 8, else 16 rows; clips of 8 frames two to a
- *                warp); every other shape, and _f32, on CUDA cores, one warp
- *                per query frame (correct, much slower).
+ *                n_post <= 16 or L == 8 or 32 with n_pre, n_post <= 8 runs
+ *                on tensor cores (TMA-staged blocks, mma.sync; an 8-row
+ *                window on each side when both context sizes are <= 8, else
+ *                16 rows; clips of 8 frames two to a warp, of 32 two warps
+ *                to a clip); every other shape, and _f32, on CUDA cores, one
+ *                warp per query frame (correct, much slower).
  * Scratch      : none.
  */
 int vi_dual_attn(const void* q, const void* k, const void* v, void* out, int F, int N, int P,

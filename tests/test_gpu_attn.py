@@ -56,6 +56,11 @@ SMALL = [
     W("bf16_L8_short_ctx", "bf16", 64, 8, 4, 2, n_pre=3, n_post=5, n_global=7),
     W("bf16_L8_one_sided", "bf16", 96, 12, 3, 1, n_pre=0, n_post=8, n_global=0),
     W("bf16_L8_pre_only", "bf16", 48, 6, 2, 1, n_pre=8, n_post=1, n_global=16),
+    # clips of 32 frames on the fast path: two warps per clip
+    W("bf16_L32_1blk_ragged", "bf16", 96, 3, 4, 2),            # 3 of 4 clips in the block
+    W("bf16_L32_3blk_ctx", "bf16", 320, 10, 2, 3, n_pre=5, n_post=8, n_global=10),
+    W("bf16_L32_one_clip", "bf16", 32, 1, 5, 1, n_global=4),
+    W("bf16_L32_no_global", "bf16", 128, 4, 3, 2, n_global=0),
     # shapes outside the fast path: the generic kernel
     W("bf16_L4_generic", "bf16", 32, 8, 4, 2, n_pre=4, n_post=4),
     W("bf16_L32_generic", "bf16", 64, 2, 3, 1, n_pre=16, n_post=12, n_global=20),
@@ -78,6 +83,12 @@ def test_full_size_sampled_positions(cuda_device, w):
 def test_clips_of_8_frames_at_size(cuda_device):
     """F = 1024 in 128 clips of 8 frames (the fast path, two clips per warp)."""
     w = W("bf16_F1024_N128_P64_C320_L8", "bf16", 1024, 128, 64, 5)
+    run_case(w, positions=sample_positions(w.P, count=2))
+
+
+def test_clips_of_32_frames_at_size(cuda_device):
+    """F = 1024 in 32 clips of 32 frames (the fast path, two warps per clip)."""
+    w = W("bf16_F1024_N32_P64_C320_L32", "bf16", 1024, 32, 64, 5)
     run_case(w, positions=sample_positions(w.P, count=2))
 
 

@@ -69,6 +69,7 @@ FUSED = [
     W("attnmod_fused_F288_N18_P2_h5_halo16", 288, 18, 2, 5, n_pre=12, n_post=16, n_global=9),
     W("attnmod_fused_F256_N16_P2_h5_ctx", 256, 16, 2, 5, n_pre=0, n_post=3, n_global=16),
     W("attnmod_fused_F72_N9_P3_h3_L8", 72, 9, 3, 3, n_pre=5, n_post=8, n_global=9),   # 8-frame clips
+    W("attnmod_fused_F160_N5_P3_h4_L32", 160, 5, 3, 4, n_pre=8, n_post=2, n_global=5),  # 32-frame
 ]
 
 
