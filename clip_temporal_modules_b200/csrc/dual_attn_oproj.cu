@@ -13,16 +13,17 @@
 // it back: 2 x 2 bytes per channel and token on top of q, k, v and out.  Here
 // a never leaves the SM.
 //   Work item = (position p, block of 128 frames), every head.  One
-//   persistent CTA per SM walks its items; 10 warps:
-//     warps 0-7  the attention (warp w: frames 16w .. 16w+15 of the block, one
-//                clip of 16 frames, two of 8 or half of one of 32, the same
-//                per-warp code as the attention kernel), then the block's
-//                epilogue;
-//     warp 8     TMA producer: per head, its stage (Q, K/V window, K/V global)
-//                into a ring of 3 stages that runs on across blocks, and the
-//                columns 64h .. 64h+63 of W_out (C rows x 128 bytes) into one
-//                buffer; it also issues the blocks' output stores;
-//     warp 9     TMEM allocation and the MMA thread.
+//   persistent CTA per SM walks its items; 14 warps:
+//     warps 0-7    the attention (warp w: frames 16w .. 16w+15 of the block,
+//                  one clip of 16 frames, two of 8 or half of one of 32, the
+//                  same per-warp code as the attention kernel), head after
+//                  head and block after block;
+//     warp 8       TMA producer: per head, its stage (Q, K/V window of 8 rows
+//                  each side, K/V global) into a ring of 3 stages that runs on
+//                  across blocks, and the columns 64h .. 64h+63 of W_out
+//                  (C rows x 128 bytes) into one buffer;
+//     warp 9       TMEM allocation and the MMA thread;
+//     warps 10-13  the epilogue, one per TMEM lane quarter.
 //   Per head, the attention warps write O_h (128 x 64 bf16) over the Q tile
 //   of its stage.  That tile's 128-byte swizzle is also the K-major operand
 //   layout of tcgen05.mma, so the MMA thread accumulates
@@ -31,14 +32,15 @@
 //   M = 128, N = C/2, K = 16 per head).  When the MMAs of head g are done,
 //   its stage and the W_out buffer are free: the producer loads the W_out
 //   slice of head g+1 and the stage of head g+3.
-//   After a block's last head the attention warps read the accumulator (warp
-//   w: TMEM lanes 32(w%4) .. +31, columns (w/4)C/2 .. +C/2-1), hand TMEM back
-//   to the next block's MMAs, add b_out, round to bf16 and stage the rows in
-//   the last head's stage and the W_out buffer; the producer stores them with
-//   TMA (frames past the end fall outside the tensor map and are dropped) and
-//   refills that memory once the stores have read it.  Meanwhile the
-//   attention warps go on with the next block, whose first two stages are
-//   already loaded.
+//   After a block's last head the epilogue warps read the accumulator, add
+//   b_out, round to bf16 and park the packed rows in spare TMEM columns, so
+//   that the accumulator goes back to the next block's MMAs at once; then
+//   they store the rows through their own staging buffers with TMA (frames
+//   past the end fall outside the tensor map and are dropped).
+//   The attention warps never wait for the epilogue.
+// The three stages, the W_out slice and the staging fill the shared memory
+// with the 8-row window: contexts above 8 frames run the attention kernel
+// and the output GEMM instead.
 // HBM traffic per token: q, k, v read once and out written once (4 C x 2 B),
 // against 6 C x 2 B for the attention plus the output GEMM.  Every block
 // re-reads W_out (C x C x 2 B) from L2.
@@ -50,59 +52,56 @@
 
 namespace vi {
 
-constexpr int FO_THREADS = 320;                   // 8 attention warps, producer, MMA
+constexpr int FO_ATTN_WARPS = 8;                  // one per 16 query rows
+constexpr int FO_EPI_WARPS = 4;                   // one per TMEM lane quarter
+constexpr int FO_THREADS = 32 * (FO_ATTN_WARPS + 2 + FO_EPI_WARPS);   // + producer, MMA
 constexpr int FO_C_MAX = 320;                     // channels (5 heads of 64)
 constexpr int FO_STAGES = 3;
-constexpr int FO_G_MAX = FO_C_MAX / 64;           // 32-column groups per epilogue warp
+constexpr int FO_H = 8;                           // window rows each side (context <= 8)
+constexpr uint32_t FO_EPI_BUF = 32 * 64;          // 32 frames x 32 channels of bf16
 
 // Shared memory: 3 stages of the attention kernel's layout (without its
-// barrier) | W_out slice of one head (up to FO_C_MAX rows x 128 B) | barriers.
-// The output staging of a block (C/64 boxes of 128 frames x 64 channels,
-// 16 KB each) reuses the stage of its last head (boxes 0-2) and the W_out
-// buffer (boxes 3-4), both idle from the last head's MMAs until the stores
-// have read them.
-template <int H>
+// barrier) | W_out slice of one head (up to FO_C_MAX rows x 128 B) | two
+// output staging buffers per epilogue warp | barriers | b_out in fp32.
 struct FoLayout {
-  static constexpr uint32_t STAGE = FaLayout<H>::STAGE;
+  static constexpr uint32_t STAGE = FaLayout<FO_H>::STAGE;
   static constexpr uint32_t OFF_W = FO_STAGES * STAGE;
-  static constexpr uint32_t OFF_BAR = OFF_W + FO_C_MAX * FA_ROW_BYTES;
-  static constexpr uint32_t BOX = FA_ROWS_Q * FA_ROW_BYTES;     // one output box
-  static constexpr int BOXES_IN_STAGE = STAGE / BOX;            // 3
-  // full[3], o_full[3], w_full, m_done, acc_full, tmem_empty, staged, drain
-  // (8 bytes each), TMEM slot; then b_out in fp32
+  static constexpr uint32_t OFF_EPI = OFF_W + FO_C_MAX * FA_ROW_BYTES;
+  static constexpr uint32_t OFF_BAR = OFF_EPI + FO_EPI_WARPS * 2 * FO_EPI_BUF;
+  // full[3], o_full[3], w_full, m_done, acc_full, tmem_empty, drain (8 bytes
+  // each), TMEM slot
   static constexpr uint32_t OFF_BIAS = OFF_BAR + 128;
   static constexpr uint32_t SMEM = OFF_BIAS + FO_C_MAX * 4 + 1024;   // + slack for alignment
-  static_assert(OFF_W % 1024 == 0, "the W_out slice is 128B-swizzled");
-  static_assert(BOXES_IN_STAGE >= 3 &&
-                    (FO_C_MAX / 64 - BOXES_IN_STAGE) * BOX <= FO_C_MAX * FA_ROW_BYTES,
-                "a block's output staging fits one stage and the W_out buffer");
+  static_assert(OFF_W % 1024 == 0 && OFF_EPI % 1024 == 0,
+                "the W_out slice is 128B-swizzled, the staging 64B-swizzled");
   static_assert(SMEM <= 232448, "one CTA per SM must fit");
 };
 
 struct FoMaps {
   CUtensorMap q, k, v, kg, vg;   // as in the attention kernel
   CUtensorMap w;                 // W_out [C][C]: box of 64 input channels x C/2 rows
-  CUtensorMap y;                 // out [P][F][C]: box of 64 channels x 128 frames
+  CUtensorMap y;                 // out [P][F][C]: box of 32 channels x 32 frames
 };
 
 // Persistent: CTA c walks the blocks (position p, 128 frames) c, c + grid,
-// ... of the video (N clips of LQ = 8, 16 or 32 frames, P positions); global head
-// g of the CTA is head g % heads of its block g / heads, staged in stage g % 3.
-// tmem_cols: a power of two >= C.
-template <int H, int LQ>
+// ... of the video (N clips of LQ = 8, 16 or 32 frames, P positions); global
+// head g of the CTA is head g % heads of its block g / heads, staged in stage
+// g % 3.  tmem_cols: a power of two >= 3C/2.
+template <int LQ>
 __global__ void __launch_bounds__(FO_THREADS, 1)
     dual_attn_oproj_bf16(const __grid_constant__ FoMaps maps, const bf16* __restrict__ b_out,
                          int N, int P, int heads, int n_pre, int n_post, int n_global,
                          float scale_log2, uint32_t tmem_cols, unsigned int* err_word) {
-  using Lay = FaLayout<H>;
-  using FL = FoLayout<H>;
+  using Lay = FaLayout<FO_H>;
+  using FL = FoLayout;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
-  const uint32_t sW = base + FL::OFF_W, bars = base + FL::OFF_BAR, sBias = base + FL::OFF_BIAS;
+  const uint32_t sW = base + FL::OFF_W, sEpi = base + FL::OFF_EPI;
+  const uint32_t bars = base + FL::OFF_BAR, sBias = base + FL::OFF_BIAS;
   const uint32_t o_full0 = bars + 8 * FO_STAGES, w_full = bars + 16 * FO_STAGES;
   const uint32_t m_done = w_full + 8, acc_full = w_full + 16, tmem_empty = w_full + 24;
-  const uint32_t staged = w_full + 32, drain = w_full + 40, tmem_slot = w_full + 48;
-  const int C = heads * 64, NH = C / 2;           // NH: N of one MMA, columns of one warp
+  const uint32_t drain = w_full + 32, tmem_slot = w_full + 40;
+  const int C = heads * 64, NH = C / 2;           // NH: N of one MMA
   const int cpb = FA_ROWS_Q / LQ;                 // clips per block
   const int nblk = (N + cpb - 1) / cpb;
   const long long n_items = (long long)P * nblk;
@@ -115,32 +114,24 @@ __global__ void __launch_bounds__(FO_THREADS, 1)
     p = (int)(it / nblk);
     f0 = (int)(it % nblk) * FA_ROWS_Q;
   };
-  // Output box b of a block staged where its last head's stage and the W_out
-  // buffer are.
-  auto box_addr = [&](int i, int b) -> uint32_t {
-    const int s_last = (i * heads + heads - 1) % FO_STAGES;
-    return b < FL::BOXES_IN_STAGE ? base + (uint32_t)s_last * Lay::STAGE + (uint32_t)b * FL::BOX
-                                  : sW + (uint32_t)(b - FL::BOXES_IN_STAGE) * FL::BOX;
-  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < FO_STAGES; ++s) {
       mbar_init(bars + 8 * s, 1);
-      mbar_init(o_full0 + 8 * s, FA_CLIPS);       // one arrive per attention warp
+      mbar_init(o_full0 + 8 * s, FO_ATTN_WARPS);  // one arrive per attention warp
     }
     mbar_init(w_full, 1);
     mbar_init(m_done, 1);
     mbar_init(acc_full, 1);
-    mbar_init(tmem_empty, FA_CLIPS);
-    mbar_init(staged, FA_CLIPS);
+    mbar_init(tmem_empty, FO_EPI_WARPS);
     mbar_init(drain, 1);
     fence_barrier_init();
   }
-  if (warp == 9) {
+  if (warp == FO_ATTN_WARPS + 1) {
     tmem_alloc(tmem_slot, tmem_cols);
     tmem_relinquish();
   }
-  if ((int)threadIdx.x < C)                       // C <= FO_C_MAX = FO_THREADS
+  if ((int)threadIdx.x < C)                       // C <= FO_C_MAX <= FO_THREADS
     asm volatile("st.shared.f32 [%0], %1;" ::"r"(sBias + 4u * threadIdx.x),
                  "f"(__bfloat162float(b_out[threadIdx.x])));
   tc_fence_before();
@@ -149,7 +140,7 @@ __global__ void __launch_bounds__(FO_THREADS, 1)
   uint32_t tmem_base;
   asm volatile("ld.shared.u32 %0, [%1];" : "=r"(tmem_base) : "r"(tmem_slot));
 
-  if (warp == 8) {
+  if (warp == FO_ATTN_WARPS) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       const uint32_t stage_bytes = (FA_ROWS_Q + 2 * Lay::ROWS_W) * FA_ROW_BYTES +
@@ -162,8 +153,8 @@ __global__ void __launch_bounds__(FO_THREADS, 1)
         const uint32_t bar = bars + 8 * (g % FO_STAGES);
         mbar_arrive_expect_tx(bar, stage_bytes);
         tma_load_3d(st + Lay::OFF_Q, &maps.q, h * 64, f0, p, bar);
-        tma_load_3d(st + Lay::OFF_KW, &maps.k, h * 64, f0 - H, p, bar);
-        tma_load_3d(st + Lay::OFF_VW, &maps.v, h * 64, f0 - H, p, bar);
+        tma_load_3d(st + Lay::OFF_KW, &maps.k, h * 64, f0 - FO_H, p, bar);
+        tma_load_3d(st + Lay::OFF_VW, &maps.v, h * 64, f0 - FO_H, p, bar);
         if (n_global > 0) {
           tma_load_3d(st + Lay::OFF_KG, &maps.kg, h * 64, 0, p, bar);
           tma_load_3d(st + Lay::OFF_VG, &maps.vg, h * 64, 0, p, bar);
@@ -175,50 +166,23 @@ __global__ void __launch_bounds__(FO_THREADS, 1)
         tma_load_2d(sW, &maps.w, h * 64, 0, w_full);
         tma_load_2d(sW + (uint32_t)NH * FA_ROW_BYTES, &maps.w, h * 64, NH, w_full);
       };
-      // Block i's output, once the attention warps have staged it: one TMA
-      // store per 64 channels (frames past the end are dropped), the boxes in
-      // the W_out buffer first, each region in a bulk group of its own, so
-      // that the buffer can be refilled as soon as its boxes have been read.
-      const int n_box = C / 64, n_box_w = n_box > FL::BOXES_IN_STAGE ? n_box - FL::BOXES_IN_STAGE : 0;
-      auto store_item = [&](int i) -> bool {
-        if (!mbar_wait_bounded(staged, (uint32_t)(i & 1), err_word, VI_DEV_ERR_MMA_TIMEOUT))
-          return false;
-        int p, f0;
-        item_pos(i, p, f0);
-        for (int b = n_box - n_box_w; b < n_box; ++b)
-          tma_store_3d(&maps.y, box_addr(i, b), 64 * b, f0, p);
-        bulk_commit();
-        for (int b = 0; b < n_box - n_box_w; ++b)
-          tma_store_3d(&maps.y, box_addr(i, b), 64 * b, f0, p);
-        bulk_commit();
-        return true;
-      };
       int n_stage = total < FO_STAGES ? total : FO_STAGES;
       for (int g = 0; g < n_stage; ++g) load_stage(g);
       load_w(0);
       int n_w = 1;
-      bool ok = true;
       for (int g = 1; g < total; ++g) {
         // The MMAs of head g-1 are done: the W_out buffer and the stage of
-        // head g-1 (= that of head g+2) are free -- after the stores of the
-        // block's output staged there, if head g-1 was a block's last.
-        const bool edge = g % heads == 0;
+        // head g-1 (= that of head g+2) are free.
         if (!mbar_wait_bounded(m_done, (uint32_t)((g - 1) & 1), err_word,
-                               VI_DEV_ERR_MMA_TIMEOUT) ||
-            (edge && !store_item(g / heads - 1))) {
-          ok = false;
+                               VI_DEV_ERR_MMA_TIMEOUT))
           break;
-        }
-        if (edge) bulk_wait_read_le1();        // the W_out buffer's boxes have been read
         load_w(g);
         ++n_w;
-        if (edge) bulk_wait_read_all();        // and the stage's
         if (g + 2 < total) {
           load_stage(g + 2);
           ++n_stage;
         }
       }
-      if (ok && store_item(my_items - 1)) bulk_wait_read_all();
       // Every copy issued lands before the CTA may end (on an error path the
       // consumers may have stopped waiting for them).
       for (int s = 0; s < FO_STAGES && s < n_stage; ++s) {
@@ -228,7 +192,7 @@ __global__ void __launch_bounds__(FO_THREADS, 1)
       }
       mbar_wait_bounded(w_full, (uint32_t)((n_w - 1) & 1), err_word, VI_DEV_ERR_TMA_TIMEOUT);
     }
-  } else if (warp == 9) {
+  } else if (warp == FO_ATTN_WARPS + 1) {
     // ------------------------------------------------------------ MMA thread
     if (lane == 0) {
       const uint32_t idesc = umma_idesc_bf16_f32(128, NH);
@@ -260,16 +224,14 @@ __global__ void __launch_bounds__(FO_THREADS, 1)
       umma_commit(drain);
       mbar_wait_bounded(drain, 0, err_word, VI_DEV_ERR_MMA_TIMEOUT);
     }
-  } else {
+  } else if (warp < FO_ATTN_WARPS) {
     // ------------------------------------------------------------ attention
-    const int q = warp & 3, c = warp >> 2;   // epilogue: TMEM lane quarter, column half
-    const int G = NH / 32;                   // 32-column groups of this warp (<= FO_G_MAX)
-    bool ok = true;
     int g = 0;
-    for (int i = 0; i < my_items && ok; ++i) {
+    for (int i = 0; i < my_items; ++i) {
       int p, f0;
       item_pos(i, p, f0);
       const int clip = (f0 + 16 * warp) / LQ;  // the warp's (first) clip
+      bool ok = true;
       for (int h = 0; h < heads; ++h, ++g) {
         const int s = g % FO_STAGES;
         const uint32_t st = base + (uint32_t)s * Lay::STAGE;
@@ -278,69 +240,108 @@ __global__ void __launch_bounds__(FO_THREADS, 1)
                                                        err_word, VI_DEV_ERR_TMA_TIMEOUT));
         if (!ok) break;
         if (clip < N)
-          fa_attend_warp<H, LQ>(st + Lay::OFF_Q, st + Lay::OFF_KW, st + Lay::OFF_VW,
-                            st + Lay::OFF_KG, st + Lay::OFF_VG, warp, lane, clip, N, n_pre,
-                            n_post, n_global, scale_log2);
+          fa_attend_warp<FO_H, LQ>(st + Lay::OFF_Q, st + Lay::OFF_KW, st + Lay::OFF_VW,
+                                   st + Lay::OFF_KG, st + Lay::OFF_VG, warp, lane, clip, N,
+                                   n_pre, n_post, n_global, scale_log2);
         fence_proxy_async_smem();            // O_h is visible to the tensor core
         __syncwarp();
         if (lane == 0) mbar_arrive(o_full0 + 8 * s);
       }
       if (!ok) break;
-      // ---------------------------------------------------------- epilogue
-      ok = __all_sync(0xffffffffu, mbar_wait_bounded(acc_full, (uint32_t)(i & 1), err_word,
-                                                     VI_DEV_ERR_MMA_TIMEOUT));
-      if (!ok) break;
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    // Warp q (= its index mod 4, the TMEM lane quarter it may read) writes
+    // frames 32q .. 32q+31 of each block, all C channels, in two phases:
+    //   1. the accumulator, 32 columns at a time (the next group's load in
+    //      flight during each store), + b_out, -> bf16 pairs, -> TMEM columns
+    //      C .. C + C/2 - 1 (spare beside the accumulator); then the
+    //      accumulator goes back to the next block's MMAs;
+    //   2. the packed rows, 16 columns (32 channels) at a time, -> one of its
+    //      two staging buffers (64-byte rows, chunk i of row r at
+    //      i ^ ((r >> 1) & 3)), -> one TMA store (frames past the end are
+    //      dropped); a buffer is written again once its previous store has
+    //      read it.
+    // Loops unrolled: registers indexed at compile time only.
+    const int q = warp & 3;
+    const uint32_t my_buf = sEpi + (uint32_t)(warp - FO_ATTN_WARPS - 2) * 2u * FO_EPI_BUF;
+    const int G = C / 32;                    // 32-channel groups
+    const uint32_t t_acc = tmem_base + ((uint32_t)(32 * q) << 16);
+    const uint32_t t_out = t_acc + (uint32_t)C;
+    int ob = 0;
+    for (int i = 0; i < my_items; ++i) {
+      int p, f0;
+      item_pos(i, p, f0);
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(acc_full, (uint32_t)(i & 1), err_word,
+                                                     VI_DEV_ERR_MMA_TIMEOUT)))
+        break;
       tc_fence_after();
-      // Group by group (32 columns): TMEM -> registers (the next group's load
-      // in flight meanwhile), + b_out, -> bf16 pairs, -> row 32q + lane of the
-      // output boxes in the 128-byte swizzle (chunk j of row r at j ^ (r mod
-      // 8)).  The producer stores the boxes.  Loops unrolled: registers
-      // indexed at compile time only.
-      const uint32_t taddr = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(c * NH);
-      const int row = 32 * q + lane;
-      uint32_t ra[32], rb[32];
-      tmem_ld32(taddr, ra);
+      {
+        uint32_t r[32];
+        tmem_ld32(t_acc, r);
 #pragma unroll
-      for (int gg = 0; gg < FO_G_MAX; ++gg) {
-        if (gg >= G) break;
-        uint32_t (&r)[32] = (gg & 1) ? rb : ra;
-        uint32_t (&rn)[32] = (gg & 1) ? ra : rb;
-        tmem_wait_ld_dep(r);
-        if (gg + 1 < G) tmem_ld32(taddr + 32u * (gg + 1), rn);
-        const int col = c * NH + 32 * gg;
-        const uint32_t rowb = box_addr(i, col / 64) + (uint32_t)row * FA_ROW_BYTES;
-        const int j0 = (col % 64) / 8;           // first 16-byte chunk of the group
+        for (int gg = 0; gg < FO_C_MAX / 32; ++gg) {
+          if (gg >= G) break;
+          tmem_wait_ld_dep(r);
+          uint32_t pk[16];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          float bv[8];                           // (the same address in every lane)
-          asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];"
-                       : "=f"(bv[0]), "=f"(bv[1]), "=f"(bv[2]), "=f"(bv[3])
-                       : "r"(sBias + 4u * (col + 8 * e)));
-          asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];"
-                       : "=f"(bv[4]), "=f"(bv[5]), "=f"(bv[6]), "=f"(bv[7])
-                       : "r"(sBias + 4u * (col + 8 * e + 4)));
-          uint32_t w[4];
+          for (int e = 0; e < 4; ++e) {
+            float bv[8];                         // (the same address in every lane)
+            asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];"
+                         : "=f"(bv[0]), "=f"(bv[1]), "=f"(bv[2]), "=f"(bv[3])
+                         : "r"(sBias + 4u * (32 * gg + 8 * e)));
+            asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];"
+                         : "=f"(bv[4]), "=f"(bv[5]), "=f"(bv[6]), "=f"(bv[7])
+                         : "r"(sBias + 4u * (32 * gg + 8 * e + 4)));
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int t = 8 * e + 2 * u;           // column t of the group
-            w[u] = pack2_bf16(__uint_as_float(r[t]) + bv[2 * u],
-                              __uint_as_float(r[t + 1]) + bv[2 * u + 1]);
+            for (int u = 0; u < 4; ++u) {
+              const int t = 8 * e + 2 * u;         // column t of the group
+              pk[4 * e + u] = pack2_bf16(__uint_as_float(r[t]) + bv[2 * u],
+                                         __uint_as_float(r[t + 1]) + bv[2 * u + 1]);
+            }
           }
-          sts128(rowb + ((uint32_t)((j0 + e) ^ (row & 7)) << 4), make_uint4(w[0], w[1], w[2], w[3]));
+          // r is consumed: the next group's load goes in flight during the store.
+          if (gg + 1 < G) tmem_ld32(t_acc + 32u * (gg + 1), r);
+          tmem_st16(t_out + 16u * gg, pk);
         }
       }
+      tmem_wait_st();
       tc_fence_before();
-      fence_proxy_async_smem();              // the staging is visible to the TMA stores
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(tmem_empty);             // the next block's MMAs may start
-        mbar_arrive(staged);
+      if (lane == 0) mbar_arrive(tmem_empty);  // the next block's MMAs may start
+      {
+        uint32_t pa[16], pb[16];
+        tmem_ld16(t_out, pa);
+#pragma unroll
+        for (int gg = 0; gg < FO_C_MAX / 32; ++gg) {
+          if (gg >= G) break;
+          uint32_t (&pc)[16] = (gg & 1) ? pb : pa;
+          uint32_t (&pn)[16] = (gg & 1) ? pa : pb;
+          tmem_wait_ld_dep16(pc);
+          if (gg + 1 < G) tmem_ld16(t_out + 16u * (gg + 1), pn);
+          const uint32_t buf = my_buf + (uint32_t)ob * FO_EPI_BUF;
+          if (lane == 0) bulk_wait_read_le1();   // the store that last read this buffer is done
+          __syncwarp();
+          const uint32_t row = buf + (uint32_t)lane * 64u, sw = (uint32_t)((lane >> 1) & 3);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            sts128(row + (((uint32_t)e ^ sw) << 4),
+                   make_uint4(pc[4 * e], pc[4 * e + 1], pc[4 * e + 2], pc[4 * e + 3]));
+          fence_proxy_async_smem();              // the writes are visible to the TMA store
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_3d(&maps.y, buf, 32 * gg, f0 + 32 * q, p);
+            bulk_commit();
+          }
+          ob ^= 1;
+        }
       }
     }
+    if (lane == 0) bulk_wait_read_all();       // the staging is read before the CTA ends
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == FO_ATTN_WARPS + 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, tmem_cols);
   }
@@ -350,21 +351,21 @@ bool encode_tmap(CUtensorMap* map, const void* base, int rank, const uint64_t* d
                  const uint64_t* strides_bytes, const uint32_t* box, CUtensorMapSwizzle swz,
                  CUtensorMapDataType dt);
 
-template <int H, int LQ>
+template <int LQ>
 static int fo_prepare() {
   static std::atomic<bool> attr_set[64] = {};
   int dev = 0;
   VI_CUDA_TRY(cudaGetDevice(&dev));
   if (dev < 0 || dev >= 64 || !attr_set[dev].load(std::memory_order_acquire)) {
-    VI_CUDA_TRY(cudaFuncSetAttribute(dual_attn_oproj_bf16<H, LQ>,
+    VI_CUDA_TRY(cudaFuncSetAttribute(dual_attn_oproj_bf16<LQ>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     FoLayout<H>::SMEM));
+                                     FoLayout::SMEM));
     if (dev >= 0 && dev < 64) attr_set[dev].store(true, std::memory_order_release);
   }
   return VI_OK;
 }
 
-template <int H, int LQ>
+template <int LQ>
 static int fo_launch(const bf16* q, const bf16* k, const bf16* v, const bf16* w_out,
                      const bf16* b_out, bf16* out, int F, int N, int P, int heads, int n_pre,
                      int n_post, int n_global, cudaStream_t stream) {
@@ -372,14 +373,14 @@ static int fo_launch(const bf16* q, const bf16* k, const bf16* v, const bf16* w_
   FoMaps maps;
   const uint64_t dims[3] = {(uint64_t)C, (uint64_t)F, (uint64_t)P};
   const uint64_t strides[2] = {(uint64_t)C * 2, (uint64_t)F * C * 2};
-  const uint32_t boxQ[3] = {64, FA_ROWS_Q, 1}, boxW[3] = {64, FaLayout<H>::ROWS_W, 1};
-  const uint32_t boxY[3] = {64, FA_ROWS_Q, 1};
+  const uint32_t boxQ[3] = {64, FA_ROWS_Q, 1}, boxW[3] = {64, FaLayout<FO_H>::ROWS_W, 1};
+  const uint32_t boxY[3] = {32, 32, 1};
   const CUtensorMapDataType BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const CUtensorMapSwizzle SW = CU_TENSOR_MAP_SWIZZLE_128B;
   bool ok = encode_tmap(&maps.q, q, 3, dims, strides, boxQ, SW, BF) &&
             encode_tmap(&maps.k, k, 3, dims, strides, boxW, SW, BF) &&
             encode_tmap(&maps.v, v, 3, dims, strides, boxW, SW, BF) &&
-            encode_tmap(&maps.y, out, 3, dims, strides, boxY, SW, BF);
+            encode_tmap(&maps.y, out, 3, dims, strides, boxY, CU_TENSOR_MAP_SWIZZLE_64B, BF);
   {
     const uint64_t wdims[2] = {(uint64_t)C, (uint64_t)C};
     const uint64_t wstrides[1] = {(uint64_t)C * 2};
@@ -398,7 +399,7 @@ static int fo_launch(const bf16* q, const bf16* k, const bf16* v, const bf16* w_
     maps.vg = maps.v;
   }
   if (!ok) return VI_ERR_CUDA;
-  int st = fo_prepare<H, LQ>();
+  int st = fo_prepare<LQ>();
   if (st != VI_OK) return st;
   const int cpb = FA_ROWS_Q / LQ;
   const int nblk = (N + cpb - 1) / cpb;
@@ -409,12 +410,13 @@ static int fo_launch(const bf16* q, const bf16* k, const bf16* v, const bf16* w_
   // with at most 2^31 / heads heads of work.
   const int64_t grid = n_items < sms ? n_items : sms;
   if ((n_items + grid - 1) / grid * heads > 0x7fffffff) return VI_ERR_UNSUPPORTED;
+  // The accumulator (C columns) and the epilogue's packed bf16 rows (C / 2).
   uint32_t tmem_cols = 64;
-  while ((int)tmem_cols < C) tmem_cols <<= 1;
+  while ((int)tmem_cols < C + C / 2) tmem_cols <<= 1;
   const float scale_log2 = 1.4426950408889634f / 8.0f;    // log2(e) / sqrt(64)
   unsigned int* err = device_error_word();
   if (!err) return VI_ERR_CUDA;
-  dual_attn_oproj_bf16<H, LQ><<<(unsigned)grid, FO_THREADS, FoLayout<H>::SMEM, stream>>>(
+  dual_attn_oproj_bf16<LQ><<<(unsigned)grid, FO_THREADS, FoLayout::SMEM, stream>>>(
       maps, b_out, N, P, heads, n_pre, n_post, n_global, scale_log2, tmem_cols, err);
   VI_LAUNCHED();
   return VI_OK;
@@ -422,9 +424,11 @@ static int fo_launch(const bf16* q, const bf16* k, const bf16* v, const bf16* w_
 
 bool dual_attn_fast_ok(int F, int N, int d, int n_pre, int n_post, int n_global);
 
-// The attention fast path's shapes with at most FO_C_MAX channels.
+// The attention fast path's shapes with at most FO_C_MAX channels and context
+// of at most FO_H frames on each side (the 8-row window: three stages, the
+// W_out slice and the epilogue staging fill the shared memory).
 bool dual_attn_oproj_ok(int F, int N, int d, int heads, int n_pre, int n_post, int n_global) {
-  return heads >= 1 && heads * 64 <= FO_C_MAX &&
+  return heads >= 1 && heads * 64 <= FO_C_MAX && n_pre <= FO_H && n_post <= FO_H &&
          dual_attn_fast_ok(F, N, d, n_pre, n_post, n_global);
 }
 
@@ -432,16 +436,13 @@ int dual_attn_oproj_bf16_launch(const bf16* q, const bf16* k, const bf16* v, con
                                 const bf16* b_out, bf16* out, int F, int N, int P, int heads,
                                 int n_pre, int n_post, int n_global, cudaStream_t stream) {
   if (F / N == 8)
-    return fo_launch<FA_HALO, 8>(q, k, v, w_out, b_out, out, F, N, P, heads, n_pre, n_post,
-                                 n_global, stream);
+    return fo_launch<8>(q, k, v, w_out, b_out, out, F, N, P, heads, n_pre, n_post, n_global,
+                        stream);
   if (F / N == 32)
-    return fo_launch<FA_HALO, 32>(q, k, v, w_out, b_out, out, F, N, P, heads, n_pre, n_post,
-                                  n_global, stream);
-  if (n_pre <= FA_HALO && n_post <= FA_HALO)
-    return fo_launch<FA_HALO, FA_L>(q, k, v, w_out, b_out, out, F, N, P, heads, n_pre, n_post,
-                                    n_global, stream);
-  return fo_launch<FA_HALO_MAX, FA_L>(q, k, v, w_out, b_out, out, F, N, P, heads, n_pre, n_post,
-                                      n_global, stream);
+    return fo_launch<32>(q, k, v, w_out, b_out, out, F, N, P, heads, n_pre, n_post, n_global,
+                         stream);
+  return fo_launch<FA_L>(q, k, v, w_out, b_out, out, F, N, P, heads, n_pre, n_post, n_global,
+                         stream);
 }
 
 }  // namespace vi

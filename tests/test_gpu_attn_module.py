@@ -66,7 +66,7 @@ FUSED = [
     W("attnmod_fused_F48_N3_P5_h1_noglobal", 48, 3, 5, 1, n_global=0),
     W("attnmod_fused_F16_N1_P7_h3_oneclip", 16, 1, 7, 3, n_global=4),
     W("attnmod_fused_F128_N8_P3_h4", 128, 8, 3, 4),
-    W("attnmod_fused_F288_N18_P2_h5_halo16", 288, 18, 2, 5, n_pre=12, n_post=16, n_global=9),
+    W("attnmod_fused_F288_N18_P2_h5_ctx8", 288, 18, 2, 5, n_pre=8, n_post=7, n_global=9),
     W("attnmod_fused_F256_N16_P2_h5_ctx", 256, 16, 2, 5, n_pre=0, n_post=3, n_global=16),
     W("attnmod_fused_F72_N9_P3_h3_L8", 72, 9, 3, 3, n_pre=5, n_post=8, n_global=9),   # 8-frame clips
     W("attnmod_fused_F160_N5_P3_h4_L32", 160, 5, 3, 4, n_pre=8, n_post=2, n_global=5),  # 32-frame
@@ -114,6 +114,25 @@ def test_fused_kernel_alone_elementwise(cuda_device, w):
 def test_fused_kernel_alone_full_size_sampled_positions(cuda_device):
     w = synth.BY_NAME["bf16_F1024_P2560_C320"]
     oproj_case(w, positions=sample_positions(w.P, count=3))
+
+
+def test_fused_form_refuses_context_above_8(cuda_device):
+    """Context above 8 frames needs the 16-row window, whose stages do not fit
+    beside the fused kernel's W_out slice and staging: the forced fused form is
+    refused before any launch, and the library's choice runs the attention
+    kernel (16-row window) and the output GEMM (checked against the oracle)."""
+    from clip_temporal_modules_b200._binding import dual_attn_oproj, temporal_attention_forced_form
+    w = W("attnmod_F288_N18_P2_h5_halo16", 288, 18, 2, 5, n_pre=12, n_post=16, n_global=9)
+    x, wq, bq, wo, bo = (to_device(synth.make(w, t), w.dtype) for t in NAMES)
+    n0 = vi.launch_count()
+    with pytest.raises(vi.ViError):
+        temporal_attention_forced_form(x, wq, bq, wo, bo, N=w.N, heads=w.heads, fused=True,
+                                       n_pre=w.n_pre, n_post=w.n_post, n_global=w.n_global)
+    with pytest.raises(vi.ViError):
+        dual_attn_oproj(x, x, x, wo, bo, N=w.N, heads=w.heads, n_pre=w.n_pre, n_post=w.n_post,
+                        n_global=w.n_global)
+    assert vi.launch_count() == n0
+    run_case(w)
 
 
 def test_fused_form_refuses_more_than_five_heads(cuda_device):
