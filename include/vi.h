@@ -183,14 +183,19 @@ int vi_groupnorm_global_f32(const void* x, const void* gamma, const void* beta, 
  *   out = a Wo^T + bo
  * The three input projections are ONE tensor-core GEMM of N = 3C over x
  * (the temporal-conv kernel with a single tap, its output channels split
- * into the q, k and v tensors), then the attention kernel, then the output
- * projection GEMM; each stage writes a bf16 tensor.
+ * into the q, k and v tensors), each written as a bf16 tensor.  Then, where
+ * C <= 320 and the attention takes its tensor-core path with n_pre, n_post
+ * <= 8, one kernel runs the attention and the output projection (a is
+ * rounded to bf16 on chip and never written); otherwise the attention kernel
+ * writes a (bf16) and the output projection GEMM follows.  The two forms
+ * differ only in the fp32 summation order of the output projection.
  *
  * x, out : [P][F][C], C = heads*d;  w_qkv : [3C][C] (rows Wq, Wk, Wv, PyTorch
  * Linear layout);  b_qkv : [3C];  w_out : [C][C];  b_out : [C].
  * workspace : device buffer of vi_temporal_attention_workspace_bytes(F, P, C)
  *             bytes (16-byte aligned), owned by the caller, holding q, k, v
- *             and a between the stages; contents undefined after the call.
+ *             (and a, when the projection is not fused) between the stages;
+ *             contents undefined after the call.
  * Requirements : those of vi_dual_attn; C % 64 == 0; out, x, weights and
  *                workspace must not overlap.
  */
