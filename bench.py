@@ -561,7 +561,7 @@ def attn_generic_path(w, d, out, stream, reps=2):
     ms = e0.elapsed_time(e1) / reps
     S = w.P * w.F * w.C * w.elem_bytes
     return {"n_pre": n_pre, "n_post": n_post, "n_global": n_global, "ms": round(ms, 4),
-            "GB/s": round(4 * S / (ms / 1e3) / 1e9, 1), "path": "dual_attn_generic (CUDA cores)"}
+            "GB/s": round(4 * S / (ms / 1e3) / 1e9, 1), "path": "dual_attn_generic_staged (CUDA cores, key lists staged in shared memory)"}
 
 
 def attn_halo16(w, d, out, stream, reps=10):

@@ -33,8 +33,10 @@
 //   HBM traffic per token and head: q, k, v, out once each (4 x 128 B); the
 //   halo and global rows are re-read by neighbouring CTAs from L2.
 // Generic path (fp32 I/O, or shapes outside the fast path): one warp per
-//   (position, head, query frame), keys streamed with an online softmax in
-//   fp32, expf, and the exact key list walked in order.
+//   (position, head, query frame), keys walked in list order with an online
+//   softmax in fp32 and expf; a clip's key list is staged in shared memory
+//   once per CTA of (position, head, clip) where it fits (96 KB of K and V),
+//   else read from global memory by every query.
 #include <atomic>
 
 #include "dual_attn_tile.cuh"
@@ -110,19 +112,109 @@ __global__ void __launch_bounds__(256) dual_attn_generic(const T* __restrict__ q
   for (int e = 0; e < DPL; ++e) out[pbase + (int64_t)f * C + e] = from_f32<T>(acc[e] * inv);
 }
 
+// The same computation with each clip's key list staged in shared memory:
+// CTA = (position, head, clip), 4 warps.  The K and V rows of the clip's list
+// (own, C_pre, C_post, C_global, in list order) are copied in once; then one
+// warp per query frame of the clip walks them exactly as above (the same
+// arithmetic in the same order: identical results), reading shared memory
+// instead of re-reading the rows from L2 for every query.  nk_max: the
+// longest key list of the video (rows of each staging buffer).
+template <typename T, int DPL>
+__global__ void __launch_bounds__(128) dual_attn_generic_staged(
+    const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v, T* __restrict__ out,
+    int F, int N, int heads, int n_pre, int n_post, int n_global, int nk_max, float scale) {
+  constexpr int D = 32 * DPL;
+  constexpr int VPR = D * (int)sizeof(T) / 16;   // 16-byte vectors per row
+  extern __shared__ uint4 smem_vec[];
+  T* sK = reinterpret_cast<T*>(smem_vec);
+  T* sV = sK + (size_t)nk_max * D;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int i = (int)(blockIdx.x % N);
+  const int h = (int)((blockIdx.x / N) % heads);
+  const int64_t p = blockIdx.x / ((int64_t)N * heads);
+  const int C = heads * D, L = F / N;
+  const int64_t base = p * F * C + (int64_t)h * D;
+  const int gstride = n_global > 0 ? F / n_global : 1;
+  const int nk = L + (i > 0 ? n_pre : 0) + (i < N - 1 ? n_post : 0) + n_global;
+  for (int idx = threadIdx.x; idx < nk * VPR; idx += blockDim.x) {
+    const int t = idx / VPR, c = idx % VPR;
+    const int64_t off = base + (int64_t)key_frame(t, i, L, N, n_pre, n_post, gstride) * C;
+    reinterpret_cast<uint4*>(sK + (size_t)t * D)[c] = reinterpret_cast<const uint4*>(k + off)[c];
+    reinterpret_cast<uint4*>(sV + (size_t)t * D)[c] = reinterpret_cast<const uint4*>(v + off)[c];
+  }
+  __syncthreads();
+  for (int fl = warp; fl < L; fl += 4) {
+    const int64_t qo = base + (int64_t)(i * L + fl) * C + lane * DPL;
+    float qv[DPL], acc[DPL];
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) {
+      qv[e] = to_f32(q[qo + e]);
+      acc[e] = 0.f;
+    }
+    float m = -INFINITY, l = 0.f;
+    for (int t = 0; t < nk; ++t) {
+      const T* kr = sK + (size_t)t * D + lane * DPL;
+      float dot = 0.f;
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) dot = fmaf(qv[e], to_f32(kr[e]), dot);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+      const float s = dot * scale;
+      const float mn = fmaxf(m, s);
+      const float alpha = expf(m - mn);      // exp(-inf) = 0 on the first key
+      const float pe = expf(s - mn);
+      l = l * alpha + pe;
+      const T* vr = sV + (size_t)t * D + lane * DPL;
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) acc[e] = fmaf(pe, to_f32(vr[e]), acc[e] * alpha);
+      m = mn;
+    }
+    const float inv = 1.f / l;
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) out[qo + e] = from_f32<T>(acc[e] * inv);
+  }
+}
+
+// Shared memory of the staged kernel: up to this much per CTA (K and V of the
+// longest key list), else the unstaged kernel.
+constexpr int GA_SMEM_MAX = 96 * 1024;
+
+template <typename T>
+static int ga_staged_prepare() {
+  static std::atomic<bool> attr_set[64] = {};
+  int dev = 0;
+  VI_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64 || !attr_set[dev].load(std::memory_order_acquire)) {
+    VI_CUDA_TRY(cudaFuncSetAttribute(dual_attn_generic_staged<T, 2>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, GA_SMEM_MAX));
+    if (dev >= 0 && dev < 64) attr_set[dev].store(true, std::memory_order_release);
+  }
+  return VI_OK;
+}
+
 template <typename T>
 int dual_attn_generic_launch(const T* q, const T* k, const T* v, T* out, int F, int N, int P,
                              int heads, int d, int n_pre, int n_post, int n_global,
                              cudaStream_t stream) {
+  if (d != 64) return VI_ERR_UNSUPPORTED;
+  const float scale = 1.0f / sqrtf((float)d);
+  const int L = F / N;
+  const int nk_max = L + (N > 1 ? n_pre + n_post : 0) + n_global;
+  const int64_t smem = 2 * (int64_t)nk_max * d * (int64_t)sizeof(T);
+  const int64_t ctas = (int64_t)P * heads * N;
+  if (smem <= GA_SMEM_MAX && ctas <= 0x7fffffff) {
+    int st = ga_staged_prepare<T>();
+    if (st != VI_OK) return st;
+    dual_attn_generic_staged<T, 2><<<(unsigned)ctas, 128, (size_t)smem, stream>>>(
+        q, k, v, out, F, N, heads, n_pre, n_post, n_global, nk_max, scale);
+    VI_LAUNCHED();
+    return VI_OK;
+  }
   const int64_t warps = (int64_t)P * heads * F;
   const int64_t blocks = (warps + 7) / 8;
   if (blocks > 0x7fffffff) return VI_ERR_UNSUPPORTED;
-  const float scale = 1.0f / sqrtf((float)d);
-  if (d == 64)
-    dual_attn_generic<T, 2><<<(unsigned)blocks, 256, 0, stream>>>(q, k, v, out, F, N, P, heads,
-                                                                  n_pre, n_post, n_global, scale);
-  else
-    return VI_ERR_UNSUPPORTED;
+  dual_attn_generic<T, 2><<<(unsigned)blocks, 256, 0, stream>>>(q, k, v, out, F, N, P, heads,
+                                                                n_pre, n_post, n_global, scale);
   VI_LAUNCHED();
   return VI_OK;
 }

@@ -65,6 +65,8 @@ SMALL = [
     W("bf16_L4_generic", "bf16", 32, 8, 4, 2, n_pre=4, n_post=4),
     W("bf16_L32_generic", "bf16", 64, 2, 3, 1, n_pre=16, n_post=12, n_global=20),
     W("bf16_L8_global20_generic", "bf16", 64, 8, 2, 1, n_global=20),
+    # key lists too long to stage in shared memory: the unstaged generic kernel
+    W("bf16_L128_ctx128_unstaged", "bf16", 256, 2, 2, 1, n_pre=128, n_post=128, n_global=16),
     W("f32_generic", "f32", 48, 3, 3, 2),
     W("f32_L16_short", "f32", 64, 4, 2, 1, n_pre=2, n_post=0, n_global=5),
 ]
