@@ -188,6 +188,12 @@ def test_no_global_tuning_state_in_the_abi(L):
     oproj.argtypes = [ctypes.c_void_p] * 6 + [ctypes.c_int] * 8 + [ctypes.c_void_p]
     assert oproj(A, B, Cp, D, A, B, 64, 4, 2, 6, 64, 8, 8, 16, None) == UNSUP   # C = 384
     assert oproj(A, B, Cp, D, A, B, 64, 16, 2, 1, 64, 4, 4, 16, None) == UNSUP  # L = 4
+    assert oproj(A, B, Cp, D, A, B, 64, 4, 2, 1, 64, 12, 8, 16, None) == UNSUP  # context 12
+    assert oproj(A, B, Cp, D, A, B, 64, 4, 2, 1, 64, 8, 8, 17, None) == UNSUP   # n_global 17
+    # the forced fused form of the module refuses the same shapes before any launch
+    # (seven distinct, far-apart buffers: the module checks that none overlap)
+    bufs = [(i + 1) << 40 for i in range(7)]
+    assert form_t(*bufs, 64, 4, 2, 1, 64, 12, 8, 16, 1, None) == UNSUP
     assert oproj(None, None, None, None, None, None, 64, 4, 0, 1, 64, 8, 8, 16, None) == OK
     assert conv_t(None, None, None, None, 64, 4, 0, 64, 3, 1, None) == OK     # empty
     assert conv_t(A, B, Cp, D, 64, 4, 2, 64, 2, 1, None) == INVALID         # even k
