@@ -136,3 +136,24 @@ def test_tensor_peak_follows_the_timed_region():
     assert bench.choose_tensor_peak(peaks, 5.0, capped) == (1373.6, "bf16_tflops_sustained")
     assert bench.choose_tensor_peak(peaks, 5.0, {"sm_mhz": None, "sm_max_mhz": None}) == \
         (1610.6, "bf16_tflops")
+
+
+def test_traffic_record_holds_only_for_the_sources_it_was_taken_with(tmp_path, monkeypatch):
+    """roofline.traffic comes from profiles/traffic.json only while the
+    kernel's source files hash to what the capture recorded; any change to
+    them turns it into null, and a workload without a capture is null too."""
+    import shutil
+    w = synth.BY_NAME["bf16_F1024_P2560_C320"]
+    real = bench.load_traffic("temporal_conv", w)
+    assert isinstance(real, int) and real > 0            # the committed record holds
+    assert bench.load_traffic("temporal_conv", synth.BY_NAME["bf16_F128_P2560_C320"]) is None
+    # a copy of the tree whose conv source differs by one byte
+    root = tmp_path / "tree"
+    shutil.copytree(os.path.join(ROOT, "profiles"), root / "profiles")
+    shutil.copytree(os.path.join(ROOT, "clip_temporal_modules_b200", "csrc"),
+                    root / "clip_temporal_modules_b200" / "csrc")
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    assert bench.load_traffic("temporal_conv", w) == real
+    src = root / "clip_temporal_modules_b200" / "csrc" / "temporal_conv_tc.cu"
+    src.write_bytes(src.read_bytes() + b"\n")
+    assert bench.load_traffic("temporal_conv", w) is None
